@@ -1,0 +1,88 @@
+"""Planted mistakes: each plausible error in the oracle must fail a pin.
+
+The mistakes are planted in the oracle, on the CPU, through monkeypatching;
+each test checks that one of the pins of test_oracle_*.py sees it.  This is
+what makes the pins trustworthy: a dropped term, a wrong sign or index, or a
+transposed operand does not pass silently.
+"""
+import numpy as np
+
+from oracle import cg as cgmod
+from oracle import conv
+from oracle import sh as shmod
+from tests.helpers import block_wigner, random_rotation, small_problem
+from tests.test_oracle_sh import closed_forms
+
+
+def _equivariance_error(prob, N, s, rcv, r, x, w):
+    R = random_rotation(11)
+    Din, Dout = block_wigner(R, prob.irreps_in), block_wigner(R, prob.irreps_out)
+    y = conv.forward_bruteforce(prob, N, s, rcv, r, x, w)
+    y_rot = conv.forward_bruteforce(prob, N, s, rcv, r.astype(np.float64) @ R.T,
+                                    np.einsum("ab,nbc->nac", Din, x.astype(np.float64)), w)
+    return np.max(np.abs(y_rot - np.einsum("ab,nbc->nac", Dout, y))) / np.max(np.abs(y))
+
+
+def test_sign_error_in_sh_fails_closed_forms(monkeypatch):
+    real = shmod.sh
+
+    def bad(r, L):
+        Y = real(r, L)
+        Y[..., 5] = -Y[..., 5]             # flip Y_{2,-1}
+        return Y
+    u = np.random.default_rng(0).standard_normal((20, 3))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    assert np.max(np.abs(real(u, 3) - closed_forms(u))) < 1e-12
+    assert np.max(np.abs(bad(u, 3) - closed_forms(u))) > 1e-3
+
+
+def test_reversed_m2_in_one_cg_fails_equivariance(monkeypatch):
+    N = 8
+    prob, s, rcv, r, x, w, gy = small_problem(N=N, E=30, C=3)
+    assert _equivariance_error(prob, N, s, rcv, r, x, w) < 1e-10
+    real = cgmod.real_cg
+
+    def bad(l1, l2, l3):
+        C = real(l1, l2, l3)
+        return C[:, ::-1, :].copy() if (l1, l2, l3) == (1, 2, 1) else C
+    monkeypatch.setattr(conv, "real_cg", bad)
+    assert _equivariance_error(prob, N, s, rcv, r, x, w) > 1e-3
+
+
+def test_transposition_mistakes_are_harmless_or_shape_errors():
+    """m1 <-> m3 transposition: for l1 != l3 the shapes differ (the mistake
+    cannot run); for every natural-parity path with l1 = l3 the coupling is
+    symmetric in m1 <-> m3, so the transposed tensor gives the same result.
+    Odd paths (both-parity variant) are antisymmetric there."""
+    import itertools
+    for l1, l2 in itertools.product(range(4), repeat=2):
+        for l3 in [l1]:
+            if abs(l1 - l2) <= l3 <= l1 + l2:
+                C = cgmod.real_cg(l1, l2, l3)
+                sign = 1 if (l1 + l2 + l3) % 2 == 0 else -1
+                assert np.max(np.abs(C - sign * C.transpose(2, 1, 0))) < 1e-13
+
+
+def test_dropped_path_in_forward_fails_bilinearity(monkeypatch):
+    N = 9
+    prob, s, rcv, r, x, w, gy = small_problem(N=N, E=40, C=4)
+    y, dx, dw, dr = conv.full(prob, N, s, rcv, r, x, w, gy)
+    w_dropped = w.copy()
+    w_dropped[:, 4, :] = 0.0               # forward silently skips path 4
+    y_bad = conv.full(prob, N, s, rcv, r, x, w_dropped)
+    a, b = float((gy * y_bad).sum()), float((w * dw).sum())
+    assert abs(a - b) > 1e-6 * abs(b)
+
+
+def test_missing_radial_projection_fails_finite_differences(monkeypatch):
+    rng = np.random.default_rng(2)
+    r = rng.standard_normal((10, 3)) * 2.0
+    g = shmod.sh_grad(r, 2)
+    u = r / np.linalg.norm(r, axis=1, keepdims=True)
+    radial = np.einsum("ekj,ej->ek", g, u)
+    assert np.max(np.abs(radial)) < 1e-12
+    # a gradient that forgot the projection (grad f(u) / |r| only) differs
+    # from finite differences in the radial direction:
+    h = 1e-6
+    fd_radial = (shmod.sh(r + h * u, 2) - shmod.sh(r - h * u, 2)) / (2 * h)
+    assert np.max(np.abs(fd_radial)) < 1e-8
