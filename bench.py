@@ -1,0 +1,489 @@
+#!/usr/bin/env python
+"""Benchmark of the equivariant message-passing convolution hot path on B200.
+
+One step = the whole path over one batch of synthetic input: edge layout
+(receiver and sender CSR + stable permutations), fused forward, fused
+deterministic backward (dx, dw, dr).  Default workload: the lmax=2 setting of
+the e3j page's Table 1 (N=32768 nodes, C=128 channels, Poisson(45) in-degree,
+irreps 0e+1o+2e, L_sh=2; E ~ 1.47M edges, 11 paths, w = 8.3 GB).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Throughput is unique bytes (every tensor the step reads or writes, counted
+once) per second, and edges per second.  Multi-GPU runs are independent
+replicas (the convolution needs no collective); the timed region is bracketed
+by a barrier and a device synchronize, and the time is the max over ranks.
+``--impl reference`` times the CPU oracle (fp64 C loops) on a bounded sample of
+the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from equivariant_gnn_message_edge_b200 import workloads as wl  # noqa: E402
+
+METRIC = "conv fwd / fwd+bwd GB/s and edges/s at lmax=2 C=128; % of B200 HBM peak"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------- sizes
+
+def tensor_bytes(N, E, C, D_in, D_out, P):
+    f = 4
+    return dict(
+        senders=4 * E, receivers=4 * E, recv_ptr=4 * (N + 1), recv_perm=4 * E, send_ptr=4 * (N + 1),
+        send_perm=4 * E, x=f * N * D_in * C, r=f * E * 3, w=f * E * P * C, gy=f * N * D_out * C,
+        y=f * N * D_out * C, dx=f * N * D_in * C, dw=f * E * P * C, dr=f * E * 3)
+
+
+def byte_counts(N, E, C, D_in, D_out, P):
+    t = tensor_bytes(N, E, C, D_in, D_out, P)
+    fwd = sum(t[k] for k in ("x", "r", "w", "recv_ptr", "recv_perm", "senders", "y"))
+    bwd = sum(t[k] for k in ("x", "r", "w", "gy", "send_ptr", "send_perm", "receivers", "dx", "dw", "dr"))
+    graph = sum(t[k] for k in ("senders", "receivers", "recv_ptr", "recv_perm", "send_ptr", "send_perm"))
+    step = sum(t.values())
+    h2d = sum(t[k] for k in ("senders", "receivers", "x", "r", "w", "gy"))
+    d2h = sum(t[k] for k in ("y", "dx", "dw", "dr"))
+    return dict(fwd=fwd, bwd=bwd, graph=graph, step=step, h2d=h2d, d2h=d2h)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------------- inputs
+
+class Inputs:
+    """Seeded synthetic workload on the host (pinned when asked)."""
+
+    def __init__(self, name, P, D_in, D_out, pinned):
+        import torch
+        W = wl.WORKLOADS[name]
+        self.W = W
+        s, rcv, r = wl.make_graph(W)
+        self.N, self.E, self.C = W.N, len(s), W.C
+        mk = (lambda shape, dt: torch.empty(shape, dtype=dt, pin_memory=True)) if pinned else \
+            (lambda shape, dt: torch.empty(shape, dtype=dt))
+        self.senders = mk((self.E,), torch.int32)
+        self.receivers = mk((self.E,), torch.int32)
+        self.r = mk((self.E, 3), torch.float32)
+        self.senders.numpy()[:] = s
+        self.receivers.numpy()[:] = rcv
+        self.r.numpy()[:] = r
+        self.x = mk((W.N, D_in, W.C), torch.float32)
+        self.x.numpy()[:] = wl.features(W.N, D_in, W.C, wl.SEED_X)
+        self.gy = mk((W.N, D_out, W.C), torch.float32)
+        self.gy.numpy()[:] = wl.features(W.N, D_out, W.C, wl.SEED_GY)
+        self.w = mk((self.E, P, W.C), torch.float32)
+        wl.weights_into(self.w.numpy())
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- native
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from equivariant_gnn_message_edge_b200 import binding as B
+    from equivariant_gnn_message_edge_b200.conv import EqConv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    W = wl.WORKLOADS[args.workload]
+    conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    if args.vec:
+        conv.set_vec(*[int(v) for v in args.vec.split(",")])
+    P, D_in, D_out = conv.P, conv.D_in, conv.D_out
+    inp = Inputs(args.workload, P, D_in, D_out, pinned=True)
+    N, E, C = inp.N, inp.E, inp.C
+    bc = byte_counts(N, E, C, D_in, D_out, P)
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        s_d = inp.senders.to(dev, non_blocking=True)
+        r_d = inp.receivers.to(dev, non_blocking=True)
+        x_d = inp.x.to(dev, non_blocking=True)
+        rv_d = inp.r.to(dev, non_blocking=True)
+        w_d = inp.w.to(dev, non_blocking=True)
+        gy_d = inp.gy.to(dev, non_blocking=True)
+        g = conv.graph(s_d, r_d, N, stream=stream)
+        y_d = torch.empty((N, D_out, C), dtype=torch.float32, device=dev)
+        dx_d = torch.empty_like(x_d)
+        dw_d = torch.empty_like(w_d)
+        dr_d = torch.empty_like(rv_d)
+        gws_n = B.eqconv_graph_workspace_bytes(N, E)
+        gws = torch.empty(max(gws_n, 1), dtype=torch.uint8, device=dev)
+        bws_n = B.eqconv_backward_workspace_bytes(conv.plan, E)
+        bws = torch.empty(max(bws_n, 1), dtype=torch.uint8, device=dev)
+    stream.synchronize()
+    sh = stream.cuda_stream
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        B.eqconv_graph_build(conv.plan, g.c, gws, gws_n, sh)
+        if ev is not None:
+            ev[1].record(stream)
+        B.eqconv_forward(conv.plan, g.c, x_d, rv_d, w_d, y_d, 0, sh)
+        if ev is not None:
+            ev[2].record(stream)
+        B.eqconv_backward(conv.plan, g.c, x_d, rv_d, w_d, gy_d, dx_d, dw_d, dr_d, bws, bws_n,
+                          B.EQCONV_DETERMINISTIC, sh)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    stream.synchronize()
+    assert B.eqconv_get_device_error(conv.plan, sh) == B.EQCONV_OK
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_id = None
+    try:
+        gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_id.startswith("GPU-"):
+            gpu_id = "GPU-" + gpu_id
+    except Exception:
+        gpu_id = None
+    barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = B.eqconv_launch_count()
+    with ClockSampler(gpu_id) as clk:
+        t0.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    launches = B.eqconv_launch_count() - launches0
+    total_ms = t0.elapsed_time(t1)
+    graph_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    t_max = total_ms
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+
+    # non-deterministic backward, timed separately (not part of the step)
+    nd_ms = []
+    for _ in range(max(2, args.steps // 2)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        B.eqconv_backward(conv.plan, g.c, x_d, rv_d, w_d, gy_d, dx_d, dw_d, dr_d, bws, bws_n, 0, sh)
+        b.record(stream)
+        nd_ms.append((a, b))
+    stream.synchronize()
+    nd_ms = [a.elapsed_time(b) for a, b in nd_ms[1:]]
+
+    # end-to-end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        y_h = torch.empty((N, D_out, C), dtype=torch.float32, pin_memory=True)
+        dx_h = torch.empty((N, D_in, C), dtype=torch.float32, pin_memory=True)
+        dw_h = torch.empty((E, P, C), dtype=torch.float32, pin_memory=True)
+        dr_h = torch.empty((E, 3), dtype=torch.float32, pin_memory=True)
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for dst, src in ((s_d, inp.senders), (r_d, inp.receivers), (x_d, inp.x), (rv_d, inp.r),
+                                 (w_d, inp.w), (gy_d, inp.gy)):
+                    dst.copy_(src, non_blocking=True)
+                step()
+                for dst, src in ((y_h, y_d), (dx_h, dx_d), (dw_h, dw_d), (dr_h, dr_d)):
+                    dst.copy_(src, non_blocking=True)
+
+        e2e_steps = max(2, min(args.steps, 5))
+        for _ in range(2):
+            e2e_step()
+        stream.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        stream.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": bc["step"] * e2e_steps * world / (e_ms * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": bc["h2d"], "d2h_bytes_per_step": bc["d2h"],
+               "ms_per_step": e_ms / e2e_steps}
+
+    peak, peak_kind = measured_peak()
+    ms_step = t_max / args.steps
+    med = statistics.median
+    value = bc["step"] * args.steps * world / (t_max * 1e-3) / 1e9
+    fwd_gbs = bc["fwd"] / (med(fwd_ms) * 1e-3) / 1e9
+    bwd_gbs = bc["bwd"] / (med(bwd_ms) * 1e-3) / 1e9
+    fb_gbs = (bc["fwd"] + bc["bwd"]) / ((med(fwd_ms) + med(bwd_ms)) * 1e-3) / 1e9
+    bwd_avg = sum(bwd_ms) / len(bwd_ms)
+    fwd_avg = sum(fwd_ms) / len(fwd_ms)
+    traffic = load_traffic()
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded NumPy PCG64)",
+        "config": {
+            "workload": f"{W.name}: N={N}, C={C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}, L_sh={W.L_sh}, "
+                        f"P={P}, in-degree Poisson({W.mean_degree:g}), uniform senders",
+            "step": "graph build (recv+send CSR) + fused forward + fused deterministic backward",
+            "l2": "inputs larger than L2 (w alone is %.1f GB)" % (bc["step"] and 4 * E * P * C / 1e9),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "unique_bytes_per_step": bc["step"],
+        },
+        "fwd_gbps": round(fwd_gbs, 1), "bwd_gbps": round(bwd_gbs, 1), "fwd_bwd_gbps": round(fb_gbs, 1),
+        "hbm_frac_fwd_bwd": round(fb_gbs / peak, 4),
+        "edges_per_s_fwd": round(E / (med(fwd_ms) * 1e-3), 1),
+        "edges_per_s_fwd_bwd": round(E / ((med(fwd_ms) + med(bwd_ms)) * 1e-3), 1),
+        "ms": {"graph": round(med(graph_ms), 4), "fwd": round(med(fwd_ms), 4), "bwd_det": round(med(bwd_ms), 4),
+               "bwd_atomic": round(med(nd_ms), 4) if nd_ms else None},
+        "roofline": {"bound": "hbm", "kernel": "eqconv_bwd_kernel (deterministic, fused dr)",
+                     "achieved": round(bc["bwd"] / (bwd_avg * 1e-3) / 1e9, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(bc["bwd"] / (bwd_avg * 1e-3) / 1e9 / peak, 4),
+                     "traffic": traffic.get("bwd"), "algorithmic_bytes": bc["bwd"], "peak_kind": peak_kind},
+        "roofline_fwd": {"bound": "hbm", "kernel": "eqconv_fwd_kernel",
+                         "achieved": round(bc["fwd"] / (fwd_avg * 1e-3) / 1e9, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(bc["fwd"] / (fwd_avg * 1e-3) / 1e9 / peak, 4), "traffic": traffic.get("fwd"),
+                         "algorithmic_bytes": bc["fwd"]},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        result["e2e"] = e2e
+    return result, inp, (N, E, C, D_in, D_out, P)
+
+
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu summary (None if absent)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
+# --------------------------------------------------------------------- oracle
+
+def oracle_sample_step(name, n_recv, D_in, D_out, P, x=None, gy=None, nthreads=0):
+    """The whole path on the CPU oracle for the in-edges of receivers
+    0..n_recv-1 of the workload: CSR of the sample, harmonics, forward rows,
+    backward dx rows, dw/gY per edge, dr.  Returns (seconds, sample edges)."""
+    from oracle import conv as oconv
+    from oracle.csr import csr
+    from oracle.sh import sh
+    W = wl.WORKLOADS[name]
+    s, rcv, r = wl.make_graph(W)
+    k = int(np.searchsorted(rcv, n_recv))      # receiver-sorted workload
+    s_s, r_s, rv_s = s[:k], rcv[:k], r[:k]
+    w_s = wl.weights(k, P, W.C)
+    if x is None:
+        x = wl.features(W.N, D_in, W.C, wl.SEED_X)
+    if gy is None:
+        gy = wl.features(W.N, D_out, W.C, wl.SEED_GY)
+    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    t = time.perf_counter()
+    rp, rperm = csr(r_s, W.N)
+    sp, sperm = csr(s_s, W.N)
+    Y = sh(rv_s, W.L_sh)
+    oconv.forward(prob, rp, rperm, s_s, Y, x, w_s, rows=np.unique(r_s), nthreads=nthreads)
+    oconv.backward_dx(prob, sp, sperm, r_s, Y, gy, w_s, rows=np.unique(s_s), nthreads=nthreads)
+    _, gY = oconv.backward_edges(prob, s_s, r_s, Y, x, gy, w_s, nthreads=nthreads)
+    oconv.dr_from_gY(rv_s, gY, W.L_sh)
+    return time.perf_counter() - t, k
+
+
+def cpu_baseline(name, D_in, D_out, P, target_s, bytes_step, E_full):
+    from oracle import conv as oconv
+    W = wl.WORKLOADS[name]
+    x = wl.features(W.N, D_in, W.C, wl.SEED_X)
+    gy = wl.features(W.N, D_out, W.C, wl.SEED_GY)
+    t0, k0 = oracle_sample_step(name, 16, D_in, D_out, P, x, gy)
+    n_recv = int(min(W.N, max(16, 16 * target_s / max(t0, 1e-3))))
+    t, k = oracle_sample_step(name, n_recv, D_in, D_out, P, x, gy)
+    frac = k / E_full
+    return {"value": round(bytes_step * frac / t / 1e9, 4), "unit": UNIT, "cores": oconv.max_threads(),
+            "kind": "oracle", "edges_per_s": round(k / t, 1), "seconds": round(t, 2),
+            "sample": f"in-edges of receivers 0..{n_recv - 1} ({k} of {E_full} edges): CSR, SH, forward rows, "
+                      f"backward dx/dw/dr; bytes scaled by the edge fraction {frac:.5f}"}
+
+
+def run_reference(args, rank, world):
+    """CPU oracle as the reference arm: each step is a bounded sample."""
+    from oracle import build as obuild
+    from oracle import conv as oconv
+    obuild.build()
+    W = wl.WORKLOADS[args.workload]
+    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    s, rcv, r = wl.make_graph(W)
+    E = len(s)
+    bc = byte_counts(W.N, E, W.C, prob.D_in, prob.D_out, prob.P)
+    x = wl.features(W.N, prob.D_in, W.C, wl.SEED_X)
+    gy = wl.features(W.N, prob.D_out, W.C, wl.SEED_GY)
+    t0, _ = oracle_sample_step(args.workload, 16, prob.D_in, prob.D_out, prob.P, x, gy)
+    budget = max(1.0, args.ref_seconds / max(1, args.steps + args.warmup))
+    n_recv = int(min(W.N, max(16, 16 * budget / max(t0, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample_step(args.workload, n_recv, prob.D_in, prob.D_out, prob.P, x, gy)
+    tot, k = 0.0, 0
+    for _ in range(args.steps):
+        t, k = oracle_sample_step(args.workload, n_recv, prob.D_in, prob.D_out, prob.P, x, gy)
+        tot += t
+    frac = k / E
+    value = bc["step"] * frac * args.steps / tot / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot / args.steps, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded NumPy PCG64)",
+        "config": {"workload": f"{W.name}: N={W.N}, C={W.C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}, "
+                               f"L_sh={W.L_sh}, P={prob.P}",
+                   "step": "graph build + forward + backward (dx, dw, dr), oracle on a bounded sample"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oconv.max_threads(), "kind": "oracle",
+                         "sample": f"in-edges of receivers 0..{n_recv - 1} ({k} of {E} edges) per step; "
+                                   f"bytes scaled by {frac:.5f}"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+# --------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="lmax2", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--vec", default=None, help="fwd,bwd channel vector widths (2 or 4)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        result, inp, dims = run_native(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            from oracle import build as obuild
+            obuild.build()
+            N, E, C, D_in, D_out, P = dims
+            result["cpu_baseline"] = cpu_baseline(args.workload, D_in, D_out, P, args.cpu_seconds,
+                                                  byte_counts(N, E, C, D_in, D_out, P)["step"], E)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,101 @@
+"""User-level API over the C ABI: plans, edge layouts and the convolution as a
+torch.autograd.Function.  Device memory and streams come from PyTorch; every
+step of the convolution runs in libeqconv's kernels (see binding.py).
+
+    conv = EqConv("0e+1o+2e", 2, "0e+1o+2e", C=128)
+    g = conv.graph(senders, receivers, N)           # CSR + permutations, on device
+    y = conv(g, x, r, w)                            # differentiable in x, r, w
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+class Graph:
+    """Edge layout on one device: the caller's senders/receivers (int32, kept
+    alive here) plus the receiver/sender CSR built by eqconv_graph_build."""
+
+    def __init__(self, plan: int, senders: torch.Tensor, receivers: torch.Tensor, N: int, stream=None):
+        if senders.dtype != torch.int32 or receivers.dtype != torch.int32:
+            raise ValueError("senders and receivers must be int32")
+        if senders.shape != receivers.shape or senders.dim() != 1:
+            raise ValueError("senders and receivers must be 1-D of equal length")
+        dev = senders.device
+        E = senders.numel()
+        self.N, self.E = int(N), int(E)
+        self.senders = senders.contiguous()
+        self.receivers = receivers.contiguous()
+        self.recv_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+        self.send_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+        self.recv_perm = torch.empty(max(E, 1), dtype=torch.int32, device=dev)
+        self.send_perm = torch.empty(max(E, 1), dtype=torch.int32, device=dev)
+        self.c = B.eqconv_graph_t(self.N, self.E, self.senders.data_ptr() if E else 0,
+                                  self.receivers.data_ptr() if E else 0, self.recv_ptr.data_ptr(),
+                                  self.recv_perm.data_ptr(), self.send_ptr.data_ptr(), self.send_perm.data_ptr())
+        nbytes = B.eqconv_graph_workspace_bytes(self.N, self.E)
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+        B.eqconv_graph_build(plan, self.c, ws, nbytes, stream)
+        self._ws = ws  # freed with the graph; the build is stream-ordered
+
+
+class EqConv:
+    """One convolution configuration (irreps, L_sh, C) on the current device."""
+
+    def __init__(self, irreps_in: str, L_sh: int, irreps_out: str, C: int):
+        self.irreps_in, self.L_sh, self.irreps_out, self.C = irreps_in, L_sh, irreps_out, C
+        self.plan = B.eqconv_plan_create(irreps_in, L_sh, irreps_out, C)
+        info = B.eqconv_plan_info(self.plan)
+        self.P, self.D_in, self.D_sh, self.D_out = info["P"], info["D_in"], info["D_sh"], info["D_out"]
+        self.paths = info["paths"]
+
+    def __del__(self):
+        try:
+            B.eqconv_plan_destroy(self.plan)
+        except Exception:
+            pass
+
+    def set_vec(self, fwd_vec: int, bwd_vec: int):
+        B.eqconv_plan_set_vec(self.plan, fwd_vec, bwd_vec)
+
+    def graph(self, senders: torch.Tensor, receivers: torch.Tensor, N: int, stream=None) -> Graph:
+        return Graph(self.plan, senders, receivers, N, stream)
+
+    def forward_raw(self, g: Graph, x, r, w, y=None, stream=None):
+        if y is None:
+            y = torch.empty((g.N, self.D_out, self.C), dtype=torch.float32, device=x.device)
+        B.eqconv_forward(self.plan, g.c, x, r, w, y, 0, stream)
+        return y
+
+    def backward_raw(self, g: Graph, x, r, w, gy, deterministic=True, out=None, workspace=None, stream=None):
+        if out is None:
+            dx = torch.empty_like(x)
+            dw = torch.empty_like(w)
+            dr = torch.empty_like(r)
+        else:
+            dx, dw, dr = out
+        nbytes = B.eqconv_backward_workspace_bytes(self.plan, g.E)
+        if nbytes and workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+        B.eqconv_backward(self.plan, g.c, x, r, w, gy, dx, dw, dr, workspace, nbytes,
+                          B.EQCONV_DETERMINISTIC if deterministic else 0, stream)
+        return dx, dw, dr
+
+    def __call__(self, g: Graph, x, r, w, deterministic=True):
+        return _EqConvFn.apply(self, g, deterministic, x, r, w)
+
+
+class _EqConvFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, conv: EqConv, g: Graph, deterministic: bool, x, r, w):
+        x, r, w = x.contiguous(), r.contiguous(), w.contiguous()
+        ctx.conv, ctx.g, ctx.det = conv, g, deterministic
+        ctx.save_for_backward(x, r, w)
+        return conv.forward_raw(g, x, r, w)
+
+    @staticmethod
+    def backward(ctx, gy):
+        x, r, w = ctx.saved_tensors
+        dx, dw, dr = ctx.conv.backward_raw(ctx.g, x, r, w, gy.contiguous(), ctx.det)
+        return None, None, None, dx, dr, dw

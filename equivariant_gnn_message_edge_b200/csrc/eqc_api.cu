@@ -1,0 +1,388 @@
+// C ABI of libeqconv (declarations and contracts in include/eqconv.h).
+//
+// The plan validates the irreps, enumerates the natural-parity paths
+// (FlashCart, arXiv 2610.06409, App. B: triangle rule, natural parity) and
+// selects the compiled kernel instance; forward / backward validate their
+// arguments and enqueue the fused kernels of eqc_conv.cuh on the caller's
+// stream.  Nothing here allocates per call.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cctype>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "eqc_conv.cuh"
+#include "eqc_dispatch.h"
+#include "eqc_graph.h"
+#include "eqconv.h"
+
+namespace eqc {
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+template <int LSH>
+static cudaError_t dr_epi(const float* gy_part, int T, const float* r, float* dr, int E, cudaStream_t st) {
+    if (E <= 0) return cudaSuccess;
+    eqconv_dr_epilogue<LSH><<<(E + 255) / 256, 256, 0, st>>>(gy_part, T, r, dr, E);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dr_epilogue(int lsh, const float* gy_part, int T, const float* r, float* dr, int E,
+                               cudaStream_t st) {
+    switch (lsh) {
+        case 0: return dr_epi<0>(gy_part, T, r, dr, E, st);
+        case 1: return dr_epi<1>(gy_part, T, r, dr, E, st);
+        case 2: return dr_epi<2>(gy_part, T, r, dr, E, st);
+        case 3: return dr_epi<3>(gy_part, T, r, dr, E, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int LSH>
+static cudaError_t sh_k(const float* r, float* Y, int E, cudaStream_t st) {
+    if (E <= 0) return cudaSuccess;
+    eqconv_sh_kernel<LSH><<<(E + 255) / 256, 256, 0, st>>>(r, Y, E);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sh(int lsh, const float* r, float* Y, int E, cudaStream_t st) {
+    switch (lsh) {
+        case 0: return sh_k<0>(r, Y, E, st);
+        case 1: return sh_k<1>(r, Y, E, st);
+        case 2: return sh_k<2>(r, Y, E, st);
+        case 3: return sh_k<3>(r, Y, E, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+__global__ void k_zero_f4(float4* p, int64_t n4) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n4) p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+}  // namespace eqc
+
+struct eqconv_plan_s {
+    int lin, lsh, lout, C;
+    int fwd_vec, bwd_vec;
+    int P, D_in, D_sh, D_out;
+    int paths[eqc::kMaxPaths][3];
+    int device;
+    unsigned* d_status;
+    const eqc::KernelSet* fwd_ks;
+    const eqc::KernelSet* bwd_ks;
+};
+
+namespace {
+
+// "0e+1o+2e" (optionally "1x0e + 1x1o ...") -> L when it is the natural-parity
+// prefix 0..L; -1 if malformed, -2 if well formed but not such a prefix.
+int parse_natural_prefix(const char* s) {
+    if (!s) return -1;
+    std::string t;
+    for (const char* c = s; *c; ++c)
+        if (!std::isspace((unsigned char)*c)) t.push_back(*c);
+    if (t.empty()) return -1;
+    int expect = 0;
+    size_t i = 0;
+    bool prefix = true;
+    while (i < t.size()) {
+        size_t j = t.find('+', i);
+        if (j == std::string::npos) j = t.size();
+        std::string tok = t.substr(i, j - i);
+        if (tok.size() >= 2 && tok[0] == '1' && tok[1] == 'x') tok = tok.substr(2);
+        if (tok.size() < 2) return -1;
+        const char par = tok.back();
+        if (par != 'e' && par != 'o') return -1;
+        const std::string num = tok.substr(0, tok.size() - 1);
+        if (num.empty() || num.size() > 2) return -1;
+        for (char ch : num)
+            if (!std::isdigit((unsigned char)ch)) return -1;
+        const int l = std::stoi(num);
+        const char nat = (l % 2 == 0) ? 'e' : 'o';
+        if (l != expect || par != nat) prefix = false;
+        ++expect;
+        i = j + 1;
+        if (j == t.size()) break;
+    }
+    if (!prefix) return -2;
+    return expect - 1;
+}
+
+int default_vec(int C) { return C >= 128 ? 4 : 2; }
+
+int tiles_for(int C, int vec) { return (C + 32 * vec - 1) / (32 * vec); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device(eqconv_plan_t plan) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return EQCONV_ERR_CUDA;
+    return dev == plan->device ? EQCONV_OK : EQCONV_ERR_INVALID_ARG;
+}
+
+int check_graph(const eqconv_graph_t* g) {
+    if (!g || g->N < 0 || g->E < 0) return EQCONV_ERR_INVALID_ARG;
+    if (!g->recv_ptr || !g->send_ptr) return EQCONV_ERR_INVALID_ARG;
+    if (g->E > 0 && (!g->senders || !g->receivers || !g->recv_perm || !g->send_perm)) return EQCONV_ERR_INVALID_ARG;
+    return EQCONV_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? EQCONV_OK : EQCONV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh, const char* irreps_out, int C) {
+    if (!out) return EQCONV_ERR_INVALID_ARG;
+    *out = nullptr;
+    const int lin = parse_natural_prefix(irreps_in);
+    const int lout = parse_natural_prefix(irreps_out);
+    if (lin == -1 || lout == -1 || L_sh < 0 || C <= 0) return EQCONV_ERR_INVALID_ARG;
+    if (lin == -2 || lout == -2) return EQCONV_ERR_UNSUPPORTED;
+    if (lin > eqc::kMaxL || lout > eqc::kMaxL || L_sh > eqc::kMaxL) return EQCONV_ERR_UNSUPPORTED;
+    if (C % 4 != 0 || C < 4 || C > 4096) return EQCONV_ERR_UNSUPPORTED;
+    const eqc::PathList PL = eqc::make_paths(lin, L_sh, lout);
+    if (PL.n == 0) return EQCONV_ERR_UNSUPPORTED;
+    eqconv_plan_s* p = new (std::nothrow) eqconv_plan_s();
+    if (!p) return EQCONV_ERR_CUDA;
+    p->lin = lin;
+    p->lsh = L_sh;
+    p->lout = lout;
+    p->C = C;
+    p->P = PL.n;
+    p->D_in = (lin + 1) * (lin + 1);
+    p->D_sh = (L_sh + 1) * (L_sh + 1);
+    p->D_out = (lout + 1) * (lout + 1);
+    for (int i = 0; i < PL.n; ++i) {
+        p->paths[i][0] = PL.l1[i];
+        p->paths[i][1] = PL.l2[i];
+        p->paths[i][2] = PL.l3[i];
+    }
+    p->fwd_vec = p->bwd_vec = default_vec(C);
+    p->fwd_ks = eqc::find_instance(lin, L_sh, lout, p->fwd_vec);
+    p->bwd_ks = eqc::find_instance(lin, L_sh, lout, p->bwd_vec);
+    if (!p->fwd_ks || !p->bwd_ks) {
+        delete p;
+        return EQCONV_ERR_UNSUPPORTED;
+    }
+    if (cudaGetDevice(&p->device) != cudaSuccess || cudaMalloc(&p->d_status, sizeof(unsigned)) != cudaSuccess) {
+        delete p;
+        return EQCONV_ERR_CUDA;
+    }
+    if (cudaMemset(p->d_status, 0, sizeof(unsigned)) != cudaSuccess) {
+        cudaFree(p->d_status);
+        delete p;
+        return EQCONV_ERR_CUDA;
+    }
+    *out = p;
+    return EQCONV_OK;
+}
+
+int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec) {
+    if (!plan) return EQCONV_ERR_INVALID_ARG;
+    if ((fwd_vec != 2 && fwd_vec != 4) || (bwd_vec != 2 && bwd_vec != 4)) return EQCONV_ERR_UNSUPPORTED;
+    const eqc::KernelSet* f = eqc::find_instance(plan->lin, plan->lsh, plan->lout, fwd_vec);
+    const eqc::KernelSet* b = eqc::find_instance(plan->lin, plan->lsh, plan->lout, bwd_vec);
+    if (!f || !b) return EQCONV_ERR_UNSUPPORTED;
+    plan->fwd_vec = fwd_vec;
+    plan->bwd_vec = bwd_vec;
+    plan->fwd_ks = f;
+    plan->bwd_ks = b;
+    return EQCONV_OK;
+}
+
+int eqconv_plan_info(eqconv_plan_t plan, int* P, int* D_in, int* D_sh, int* D_out, int* paths_l1l2l3) {
+    if (!plan) return EQCONV_ERR_INVALID_ARG;
+    if (P) *P = plan->P;
+    if (D_in) *D_in = plan->D_in;
+    if (D_sh) *D_sh = plan->D_sh;
+    if (D_out) *D_out = plan->D_out;
+    if (paths_l1l2l3)
+        for (int i = 0; i < plan->P; ++i)
+            for (int k = 0; k < 3; ++k) paths_l1l2l3[3 * i + k] = plan->paths[i][k];
+    return EQCONV_OK;
+}
+
+int eqconv_enumerate_paths(const char* irreps_in, int L_sh, const char* irreps_out, int* P, int* paths_l1l2l3,
+                           int max_paths) {
+    if (!P) return EQCONV_ERR_INVALID_ARG;
+    const int lin = parse_natural_prefix(irreps_in);
+    const int lout = parse_natural_prefix(irreps_out);
+    if (lin == -1 || lout == -1 || L_sh < 0) return EQCONV_ERR_INVALID_ARG;
+    if (lin == -2 || lout == -2 || lin > eqc::kMaxL || lout > eqc::kMaxL || L_sh > eqc::kMaxL)
+        return EQCONV_ERR_UNSUPPORTED;
+    const eqc::PathList PL = eqc::make_paths(lin, L_sh, lout);
+    *P = PL.n;
+    if (paths_l1l2l3) {
+        if (max_paths < PL.n) return EQCONV_ERR_INVALID_ARG;
+        for (int i = 0; i < PL.n; ++i) {
+            paths_l1l2l3[3 * i] = PL.l1[i];
+            paths_l1l2l3[3 * i + 1] = PL.l2[i];
+            paths_l1l2l3[3 * i + 2] = PL.l3[i];
+        }
+    }
+    return EQCONV_OK;
+}
+
+int eqconv_cg_table(int l1, int l2, int l3, double* out, int out_len) {
+    if (!out) return EQCONV_ERR_INVALID_ARG;
+    if (l1 < 0 || l2 < 0 || l3 < 0 || l1 > eqc::kMaxL || l2 > eqc::kMaxL || l3 > eqc::kMaxL)
+        return EQCONV_ERR_UNSUPPORTED;
+    if (l3 < eqc::iabs(l1 - l2) || l3 > l1 + l2 || ((l1 + l2 + l3) & 1)) return EQCONV_ERR_UNSUPPORTED;
+    const int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
+    if (out_len < d1 * d2 * d3) return EQCONV_ERR_INVALID_ARG;
+    const eqc::CG3 t = eqc::make_real_cg(l1, l2, l3);
+    for (int a = 0; a < d1; ++a)
+        for (int b = 0; b < d2; ++b)
+            for (int c = 0; c < d3; ++c) out[(a * d2 + b) * d3 + c] = t.v[a][b][c];
+    return EQCONV_OK;
+}
+
+size_t eqconv_graph_workspace_bytes(int N, int E) {
+    if (N < 0 || E < 0) return 0;
+    return eqc::graph_workspace_bytes(N, E);
+}
+
+int eqconv_graph_build(eqconv_plan_t plan, const eqconv_graph_t* g, void* workspace, size_t workspace_bytes,
+                       eqconv_stream_t stream) {
+    if (!plan) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_graph(g);
+    if (rc != EQCONV_OK) return rc;
+    if ((rc = check_device(plan)) != EQCONV_OK) return rc;
+    const size_t need = eqc::graph_workspace_bytes(g->N, g->E);
+    if (!workspace || workspace_bytes < need) return EQCONV_ERR_WORKSPACE;
+    return cuda_status(eqc::graph_build(g->N, g->E, g->senders, g->receivers, g->recv_ptr, g->recv_perm, g->send_ptr,
+                                        g->send_perm, workspace, plan->d_status, (cudaStream_t)stream));
+}
+
+int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r, const float* w,
+                   float* y, unsigned flags, eqconv_stream_t stream) {
+    (void)flags;
+    if (!plan) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_graph(g);
+    if (rc != EQCONV_OK) return rc;
+    if ((rc = check_device(plan)) != EQCONV_OK) return rc;
+    if (g->N == 0) return EQCONV_OK;
+    if (!x || !y || (g->E > 0 && (!r || !w))) return EQCONV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(w)) return EQCONV_ERR_INVALID_ARG;
+    eqc::FwdParams prm{x, r, w, y, g->recv_ptr, g->recv_perm, g->senders, g->N, plan->C, plan->d_status};
+    const int T = tiles_for(plan->C, plan->fwd_vec);
+    return cuda_status(plan->fwd_ks->fwd(prm, T, (cudaStream_t)stream));
+}
+
+size_t eqconv_backward_workspace_bytes(eqconv_plan_t plan, int E) {
+    if (!plan || E < 0) return 0;
+    const int T = tiles_for(plan->C, plan->bwd_vec);
+    const int G = plan->D_sh - 1;
+    if (T == 1 || G == 0) return 0;
+    return (size_t)E * T * G * sizeof(float);
+}
+
+int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r, const float* w,
+                    const float* gy, float* dx, float* dw, float* dr, void* workspace, size_t workspace_bytes,
+                    unsigned flags, eqconv_stream_t stream) {
+    if (!plan) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_graph(g);
+    if (rc != EQCONV_OK) return rc;
+    if ((rc = check_device(plan)) != EQCONV_OK) return rc;
+    if (g->N == 0) return EQCONV_OK;
+    if (!x || !gy || !dx || (g->E > 0 && (!r || !w || !dw || !dr))) return EQCONV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gy) || !aligned16(dx) || !aligned16(w) || !aligned16(dw))
+        return EQCONV_ERR_INVALID_ARG;
+    const cudaStream_t st = (cudaStream_t)stream;
+    const bool det = (flags & EQCONV_DETERMINISTIC) != 0;
+    const int T = tiles_for(plan->C, plan->bwd_vec);
+    const int G = plan->D_sh - 1;
+    const bool fused = (T == 1) || (G == 0);
+    const size_t need = eqconv_backward_workspace_bytes(plan, g->E);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return EQCONV_ERR_WORKSPACE;
+    if (!det) {
+        const int64_t n4 = (int64_t)g->N * plan->D_in * plan->C / 4;
+        eqc::k_zero_f4<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(reinterpret_cast<float4*>(dx), n4);
+        eqc::count_launch();
+        if (cudaGetLastError() != cudaSuccess) return EQCONV_ERR_CUDA;
+    }
+    if (g->E == 0) {
+        if (det) {
+            const int64_t n4 = (int64_t)g->N * plan->D_in * plan->C / 4;
+            eqc::k_zero_f4<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(reinterpret_cast<float4*>(dx), n4);
+            eqc::count_launch();
+            if (cudaGetLastError() != cudaSuccess) return EQCONV_ERR_CUDA;
+        }
+        return EQCONV_OK;
+    }
+    eqc::BwdParams prm{};
+    prm.x = x;
+    prm.r = r;
+    prm.w = w;
+    prm.gy = gy;
+    prm.dx = dx;
+    prm.dw = dw;
+    prm.dr = dr;
+    prm.gy_part = static_cast<float*>(workspace);
+    prm.ptr = det ? g->send_ptr : g->recv_ptr;
+    prm.perm = det ? g->send_perm : g->recv_perm;
+    prm.other = det ? g->receivers : g->senders;
+    prm.N = g->N;
+    prm.C = plan->C;
+    prm.T = T;
+    prm.status = plan->d_status;
+    cudaError_t err = plan->bwd_ks->bwd(prm, det, fused, st);
+    if (err != cudaSuccess) return EQCONV_ERR_CUDA;
+    if (!fused) err = eqc::launch_dr_epilogue(plan->lsh, prm.gy_part, T, r, dr, g->E, st);
+    return cuda_status(err);
+}
+
+int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y, eqconv_stream_t stream) {
+    if (!plan || E < 0 || (E > 0 && (!r || !Y))) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_device(plan);
+    if (rc != EQCONV_OK) return rc;
+    return cuda_status(eqc::launch_sh(plan->lsh, r, Y, E, (cudaStream_t)stream));
+}
+
+int eqconv_get_device_error(eqconv_plan_t plan, eqconv_stream_t stream, int* status) {
+    if (!plan || !status) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_device(plan);
+    if (rc != EQCONV_OK) return rc;
+    unsigned h = 0;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return EQCONV_ERR_CUDA;
+    if (cudaMemcpy(&h, plan->d_status, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return EQCONV_ERR_CUDA;
+    if (h != 0 && cudaMemset(plan->d_status, 0, sizeof(unsigned)) != cudaSuccess) return EQCONV_ERR_CUDA;
+    *status = h ? EQCONV_ERR_DEVICE_CHECK : EQCONV_OK;
+    return EQCONV_OK;
+}
+
+void eqconv_plan_destroy(eqconv_plan_t plan) {
+    if (!plan) return;
+    int cur = -1;
+    const bool switch_dev = cudaGetDevice(&cur) == cudaSuccess && cur != plan->device;
+    if (switch_dev) cudaSetDevice(plan->device);
+    cudaFree(plan->d_status);
+    if (switch_dev) cudaSetDevice(cur);
+    delete plan;
+}
+
+const char* eqconv_status_string(int status) {
+    switch (status) {
+        case EQCONV_OK: return "EQCONV_OK";
+        case EQCONV_ERR_INVALID_ARG: return "EQCONV_ERR_INVALID_ARG: null/misaligned pointer, bad size or bad irreps";
+        case EQCONV_ERR_UNSUPPORTED: return "EQCONV_ERR_UNSUPPORTED: L > 3, C % 4 != 0, non-prefix irreps or no path";
+        case EQCONV_ERR_CUDA: return "EQCONV_ERR_CUDA: a CUDA call or kernel launch failed";
+        case EQCONV_ERR_WORKSPACE: return "EQCONV_ERR_WORKSPACE: workspace missing or too small";
+        case EQCONV_ERR_DEVICE_CHECK: return "EQCONV_ERR_DEVICE_CHECK: a kernel saw an out-of-range index";
+        default: return "unknown eqconv status";
+    }
+}
+
+unsigned long long eqconv_launch_count(void) { return eqc::g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Dispatch table of kernel instances (host side, no device code).
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace eqc {
+
+struct FwdParams;
+struct BwdParams;
+
+struct KernelSet {
+    int lin, lsh, lout, vec, tile_c, g;
+    cudaError_t (*fwd)(const FwdParams&, int tiles, cudaStream_t);
+    cudaError_t (*bwd)(const BwdParams&, bool det, bool fused, cudaStream_t);
+};
+
+// Instances for one (L_in, L_sh); defined in eqc_inst_l<L_in>s<L_sh>.cu.
+const KernelSet* instances_l0_s0(int lout, int vec);
+const KernelSet* instances_l0_s1(int lout, int vec);
+const KernelSet* instances_l0_s2(int lout, int vec);
+const KernelSet* instances_l0_s3(int lout, int vec);
+const KernelSet* instances_l1_s0(int lout, int vec);
+const KernelSet* instances_l1_s1(int lout, int vec);
+const KernelSet* instances_l1_s2(int lout, int vec);
+const KernelSet* instances_l1_s3(int lout, int vec);
+const KernelSet* instances_l2_s0(int lout, int vec);
+const KernelSet* instances_l2_s1(int lout, int vec);
+const KernelSet* instances_l2_s2(int lout, int vec);
+const KernelSet* instances_l2_s3(int lout, int vec);
+const KernelSet* instances_l3_s0(int lout, int vec);
+const KernelSet* instances_l3_s1(int lout, int vec);
+const KernelSet* instances_l3_s2(int lout, int vec);
+const KernelSet* instances_l3_s3(int lout, int vec);
+
+inline const KernelSet* find_instance(int lin, int lsh, int lout, int vec) {
+    using Fn = const KernelSet* (*)(int, int);
+    static const Fn fns[4][4] = {
+        {instances_l0_s0, instances_l0_s1, instances_l0_s2, instances_l0_s3},
+        {instances_l1_s0, instances_l1_s1, instances_l1_s2, instances_l1_s3},
+        {instances_l2_s0, instances_l2_s1, instances_l2_s2, instances_l2_s3},
+        {instances_l3_s0, instances_l3_s1, instances_l3_s2, instances_l3_s3},
+    };
+    if (lin < 0 || lin > 3 || lsh < 0 || lsh > 3) return nullptr;
+    return fns[lin][lsh](lout, vec);
+}
+
+// Harmonics-only kernels (depend on L_sh only); defined in eqc_api.cu.
+cudaError_t launch_dr_epilogue(int lsh, const float* gy_part, int T, const float* r, float* dr, int E,
+                               cudaStream_t st);
+cudaError_t launch_sh(int lsh, const float* r, float* Y, int E, cudaStream_t st);
+
+}  // namespace eqc

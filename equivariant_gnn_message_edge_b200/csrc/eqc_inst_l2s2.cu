@@ -1,0 +1,4 @@
+// Kernel instances for L_in = 2, L_sh = 2.
+#define EQC_LIN 2
+#define EQC_LSH 2
+#include "eqc_inst.cuh"

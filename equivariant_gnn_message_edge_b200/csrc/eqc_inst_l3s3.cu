@@ -1,0 +1,4 @@
+// Kernel instances for L_in = 3, L_sh = 3.
+#define EQC_LIN 3
+#define EQC_LSH 3
+#include "eqc_inst.cuh"

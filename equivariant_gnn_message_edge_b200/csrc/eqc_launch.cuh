@@ -1,0 +1,60 @@
+// Host-side launchers for one kernel instance (irreps L_in, L_sh, L_out and
+// channel vector width VEC), collected into a KernelSet that the C ABI
+// dispatches through.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "eqc_conv.cuh"
+#include "eqc_dispatch.h"
+
+namespace eqc {
+
+void count_launch();
+
+// One-time (per kernel, per device) opt-in above the 48 KB shared-memory default;
+// `done` must be distinct for every kernel.
+template <class Kern>
+static cudaError_t ensure_smem(Kern kern, int bytes, bool (&done)[64]) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (bytes <= 48 * 1024 || dev >= 64 || done[dev]) return cudaSuccess;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err == cudaSuccess) done[dev] = true;
+    return err;
+}
+
+template <class K>
+struct Launch {
+    static cudaError_t fwd(const FwdParams& prm, int tiles, cudaStream_t st) {
+        auto kern = eqconv_fwd_kernel<K>;
+        static bool done[64] = {};
+        cudaError_t err = ensure_smem(kern, K::FWD_SMEM, done);
+        if (err != cudaSuccess) return err;
+        dim3 grid((prm.N + K::WARPS - 1) / K::WARPS, tiles);
+        kern<<<grid, K::WARPS * 32, K::FWD_SMEM, st>>>(prm);
+        count_launch();
+        return cudaGetLastError();
+    }
+    template <bool DET, bool FUSED>
+    static cudaError_t bwd_one(const BwdParams& prm, cudaStream_t st) {
+        auto kern = eqconv_bwd_kernel<K, DET, FUSED>;
+        static bool done[64] = {};
+        cudaError_t err = ensure_smem(kern, K::BWD_SMEM, done);
+        if (err != cudaSuccess) return err;
+        dim3 grid((prm.N + K::WARPS - 1) / K::WARPS, prm.T);
+        kern<<<grid, K::WARPS * 32, K::BWD_SMEM, st>>>(prm);
+        count_launch();
+        return cudaGetLastError();
+    }
+    static cudaError_t bwd(const BwdParams& prm, bool det, bool fused, cudaStream_t st) {
+        if (det) return fused ? bwd_one<true, true>(prm, st) : bwd_one<true, false>(prm, st);
+        return fused ? bwd_one<false, true>(prm, st) : bwd_one<false, false>(prm, st);
+    }
+    static constexpr KernelSet make() {
+        return KernelSet{K::LIN, K::LSH, K::LOUT, K::VEC, K::TILE_C, K::G, &fwd, &bwd};
+    }
+};
+
+}  // namespace eqc

@@ -114,6 +114,19 @@ def weights(E: int, P: int, C: int, seed: int = SEED_W, chunk_edges: int = 1 << 
     return out
 
 
+def weights_into(out: np.ndarray, seed: int = SEED_W, chunk_edges: int = 1 << 16) -> np.ndarray:
+    """Fill a preallocated fp32 array [E, P, C] (e.g. pinned host memory) with
+    the same values as ``weights(E, P, C, seed)``."""
+    E, P, C = out.shape
+    rng = np.random.default_rng(seed)
+    scale = np.float32(1.0 / np.sqrt(P))
+    for a in range(0, E, chunk_edges):
+        blk = out[min(E, a):min(E, a + chunk_edges)]
+        rng.standard_normal(blk.shape, dtype=np.float32, out=blk)
+        blk *= scale
+    return out
+
+
 def make_graph(wl: Workload):
     """(senders, receivers, r) for a workload."""
     if wl.kind == "box":

@@ -1,0 +1,168 @@
+/*
+ * eqconv.h - C ABI of libeqconv, the sm_100a (NVIDIA B200) implementation of
+ * the E(3)-equivariant message-passing convolution of MACE-style interatomic
+ * potentials.
+ *
+ * The operation (e3j: an Efficient and Open-Source Backend for Euclidean
+ * Equivariant Operations on GPU and TPU, abstract and Table 1; FlashCart: Fast
+ * Cartesian Tensor Products for Equivariant Interatomic Potentials, App. B,
+ * §4 and App. D):
+ *
+ *   y[i, l3 m3, c] = sum_{e: recv(e) = i} sum_{p = (l1, l2, l3)} w[e, p, c]
+ *                    sum_{m1, m2} C_p[m1, m2, m3] x[send(e), l1 m1, c] Y_{l2 m2}(r_e / |r_e|)
+ *
+ * with C_p the orthonormal real-basis Clebsch-Gordan coupling of path p
+ * (Condon-Shortley phase, first nonzero entry positive) and Y the real
+ * spherical harmonics, component-normalised (sum_m Y_lm^2 = 2l+1), z polar,
+ * m > 0 ~ cos(m phi), m < 0 ~ sin(|m| phi).  Paths are the admissible
+ * (l1, l2, l3): |l1 - l2| <= l3 <= l1 + l2 and natural parity, ordered by
+ * (l1, l2, l3); paths that land on the same l3 are summed.
+ *
+ * Layout (FlashCart App. D, Figure D1: rank blocks, then components, then
+ * channels): every tensor is fp32, row-major, channels innermost.
+ *   x      [N][D_in][C]      D_in  = (L_in + 1)^2
+ *   y, gy  [N][D_out][C]     D_out = (L_out + 1)^2
+ *   w, dw  [E][P][C]
+ *   r, dr  [E][3]            edge vectors (the op depends on r / |r| only)
+ *   senders, receivers [E]   int32
+ *
+ * Supported: irreps_in / irreps_out are natural-parity prefixes "0e+1o+2e+3o"
+ * cut at L_in / L_out; L_in, L_sh, L_out <= 3; 4 <= C <= 4096, C % 4 == 0;
+ * N, E < 2^31.  All device pointers must be 16-byte aligned.
+ *
+ * Memory and streams: every tensor and workspace is caller-owned device
+ * memory (e.g. PyTorch tensors).  The plan owns its coupling tables and one
+ * device status word (allocated at plan creation on the current device).  All
+ * device work is enqueued on the given stream; no call synchronises the host
+ * except eqconv_get_device_error.  Outputs are fully overwritten.
+ *
+ * Errors: every call returns an eqconv status; nothing throws across the ABI.
+ * Out-of-range sender/receiver indices never cause out-of-bounds accesses:
+ * the kernels skip such edges and set the plan's device status word, which
+ * eqconv_get_device_error reports as EQCONV_ERR_DEVICE_CHECK.
+ */
+#ifndef EQCONV_H
+#define EQCONV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define EQCONV_API __attribute__((visibility("default")))
+#else
+#define EQCONV_API
+#endif
+
+/* ABI-identical to cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* eqconv_stream_t;
+
+enum {
+    EQCONV_OK = 0,
+    EQCONV_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, bad irreps */
+    EQCONV_ERR_UNSUPPORTED = 2,   /* L > 3, C % 4 != 0, non-prefix irreps, no paths */
+    EQCONV_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+    EQCONV_ERR_WORKSPACE = 4,     /* workspace null or smaller than required */
+    EQCONV_ERR_DEVICE_CHECK = 5   /* a kernel saw an out-of-range index (see above) */
+};
+
+/* flags for eqconv_backward */
+#define EQCONV_DETERMINISTIC 1u   /* sender-ordered pass, no atomics: bitwise run-to-run identical */
+
+typedef struct eqconv_plan_s* eqconv_plan_t;
+
+/* Edge layout.  The caller fills N, E, senders and receivers and provides the
+ * four output arrays; eqconv_graph_build fills them (FlashCart §4: receiver
+ * sorted edges; sender order for deterministic sender gradients):
+ *   recv_ptr[N+1]  = [0, cumsum(in-degree)]    recv_perm[E] = stable argsort(receivers)
+ *   send_ptr[N+1]  = [0, cumsum(out-degree)]   send_perm[E] = stable argsort(senders)
+ * All device pointers, caller-owned; the struct itself is read on the host. */
+typedef struct eqconv_graph_s {
+    int32_t N, E;
+    const int32_t* senders;
+    const int32_t* receivers;
+    int32_t* recv_ptr;
+    int32_t* recv_perm;
+    int32_t* send_ptr;
+    int32_t* send_perm;
+} eqconv_graph_t;
+
+/* Plan: parses the irreps, enumerates the paths, builds the real CG tables
+ * (Racah formula, evaluated at compile time of the library) and selects the
+ * kernel instance.  Host only, not hot.  *out receives the handle. */
+EQCONV_API int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh,
+                       const char* irreps_out, int C);
+
+/* Channel vector width of the forward / backward kernels (2 or 4 channels per
+ * lane, i.e. channel tiles of 64 or 128).  The default is 4 when C >= 128,
+ * else 2.  A tuning knob; results agree within rounding across widths. */
+EQCONV_API int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec);
+
+/* Sizes of the plan; paths_l1l2l3 (3*P ints, may be NULL) receives the paths. */
+EQCONV_API int eqconv_plan_info(eqconv_plan_t plan, int* P, int* D_in, int* D_sh, int* D_out,
+                     int* paths_l1l2l3);
+
+/* Host only, no device needed.  The natural-parity paths of (irreps_in, L_sh,
+ * irreps_out) in kernel order: *P receives the count and paths_l1l2l3 (room
+ * for max_paths triples, may be NULL) the (l1, l2, l3) triples. */
+EQCONV_API int eqconv_enumerate_paths(const char* irreps_in, int L_sh, const char* irreps_out,
+                                      int* P, int* paths_l1l2l3, int max_paths);
+
+/* Host only, no device needed.  The real-basis CG tensor the kernels use for
+ * the natural-parity path (l1, l2, l3), fp64 row-major [2l1+1][2l2+1][2l3+1];
+ * out_len must be at least that size.  EQCONV_ERR_UNSUPPORTED for odd or
+ * inadmissible triples or l > 3. */
+EQCONV_API int eqconv_cg_table(int l1, int l2, int l3, double* out, int out_len);
+
+/* Device workspace bytes needed by eqconv_graph_build for (N, E). */
+EQCONV_API size_t eqconv_graph_workspace_bytes(int N, int E);
+
+/* Builds recv_ptr/recv_perm/send_ptr/send_perm on `stream` (stable LSD radix
+ * sort + histogram + exclusive scan; bit-exact with a stable argsort).
+ * Out-of-range senders/receivers set the device status word and are counted
+ * nowhere (the outputs are then unspecified but in-bounds). */
+EQCONV_API int eqconv_graph_build(eqconv_plan_t plan, const eqconv_graph_t* g, void* workspace,
+                       size_t workspace_bytes, eqconv_stream_t stream);
+
+/* Forward (one fused kernel; receiver-sorted, atomic-free, no per-edge
+ * messages in memory; deterministic): writes y [N][D_out][C]. */
+EQCONV_API int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
+                   const float* r, const float* w, float* y, unsigned flags,
+                   eqconv_stream_t stream);
+
+/* Device workspace bytes needed by eqconv_backward (0 when C fits one
+ * channel tile: the dr reduction is then done in-kernel). */
+EQCONV_API size_t eqconv_backward_workspace_bytes(eqconv_plan_t plan, int E);
+
+/* Backward given gy: writes dx [N][D_in][C], dw [E][P][C], dr [E][3].
+ * flags & EQCONV_DETERMINISTIC: one pass over the sender CSR, dx summed in
+ * registers, no atomics; otherwise one pass over the receiver CSR with dx
+ * accumulated by atomic adds (dx is zeroed by the library first). */
+EQCONV_API int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
+                    const float* r, const float* w, const float* gy, float* dx, float* dw,
+                    float* dr, void* workspace, size_t workspace_bytes, unsigned flags,
+                    eqconv_stream_t stream);
+
+/* The spherical harmonics the kernels use, Y [E][(L_sh+1)^2] (a test hook
+ * for the in-kernel harmonics; not on the hot path). */
+EQCONV_API int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y,
+                               eqconv_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the plan's device status word;
+ * *status receives EQCONV_OK or EQCONV_ERR_DEVICE_CHECK. */
+EQCONV_API int eqconv_get_device_error(eqconv_plan_t plan, eqconv_stream_t stream, int* status);
+
+EQCONV_API void eqconv_plan_destroy(eqconv_plan_t plan);
+
+EQCONV_API const char* eqconv_status_string(int status);
+
+/* Number of kernels this library has launched in this process (all devices). */
+EQCONV_API unsigned long long eqconv_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EQCONV_H */

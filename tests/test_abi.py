@@ -1,0 +1,131 @@
+"""The C-ABI library on the CPU: it loads, exports every declared symbol, its
+host-side planner agrees with the oracle, and bad arguments are rejected
+before any device work.  No kernel runs here."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from equivariant_gnn_message_edge_b200 import binding as B
+from equivariant_gnn_message_edge_b200.workloads import natural_irreps
+from oracle.cg import real_cg
+from oracle.irreps import enumerate_paths
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "eqconv.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    if not os.path.exists(B.LIB_PATH):
+        from equivariant_gnn_message_edge_b200 import build_lib
+        build_lib.build()
+    return B.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"EQCONV_API\s+[\w\s\*]+?\b(eqconv_\w+)\s*\(", text)))
+
+
+def exported_symbols():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    return {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+
+
+def test_every_declared_function_is_exported():
+    decl = declared_functions()
+    assert len(decl) >= 15
+    exported = exported_symbols()
+    missing = [f for f in decl if f not in exported]
+    assert not missing, missing
+    for f in decl:
+        getattr(B.lib(), f)
+
+
+def test_binding_covers_the_header():
+    assert sorted(B.ABI_FUNCTIONS) == declared_functions()
+
+
+def test_only_the_abi_is_exported():
+    extra = [s for s in exported_symbols() if not s.startswith("eqconv_") and not s.startswith("_")]
+    # the static CUDA runtime may export nothing else of ours
+    assert all(not s.startswith("eqc") for s in extra)
+
+
+@pytest.mark.parametrize("l1,l2,l3", [(a, b, c) for a in range(4) for b in range(4) for c in range(4)
+                                      if abs(a - b) <= c <= a + b and (a + b + c) % 2 == 0])
+def test_library_cg_matches_oracle(l1, l2, l3):
+    """The library's compile-time Racah evaluation vs the oracle's exact
+    rationals: same real basis, phase and sign convention."""
+    assert np.max(np.abs(B.eqconv_cg_table(l1, l2, l3) - real_cg(l1, l2, l3))) < 1e-12
+
+
+def test_library_rejects_odd_or_inadmissible_cg():
+    for t in [(1, 1, 1), (1, 1, 3), (4, 0, 4)]:
+        with pytest.raises(B.EqconvError) as e:
+            B.eqconv_cg_table(*t)
+        assert e.value.status == B.EQCONV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("lin,lsh,lout", [(a, b, c) for a in range(4) for b in range(4) for c in range(4)])
+def test_library_paths_match_oracle(lin, lsh, lout):
+    ins, outs = natural_irreps(lin), natural_irreps(lout)
+    lib_paths = B.eqconv_enumerate_paths(ins, lsh, outs)
+    ref = [(q["l1"], q["l2"], q["l3"]) for q in enumerate_paths(ins, lsh, outs)]
+    assert lib_paths == ref
+
+
+def test_irreps_parsing():
+    assert len(B.eqconv_enumerate_paths(" 1x0e + 1x1o ", 2, "0e+1o+2e")) == 7
+    for bad in ["", "0x", "0e++1o", "2q", "abc"]:
+        with pytest.raises(B.EqconvError) as e:
+            B.eqconv_enumerate_paths(bad, 2, "0e")
+        assert e.value.status == B.EQCONV_ERR_INVALID_ARG
+    for unsupported in ["1o", "0e+2e", "0o", "0e+1e", "0e+1o+2e+3o+4e"]:
+        with pytest.raises(B.EqconvError) as e:
+            B.eqconv_enumerate_paths(unsupported, 2, "0e")
+        assert e.value.status == B.EQCONV_ERR_UNSUPPORTED
+
+
+def test_plan_create_validates_before_device_work():
+    cases = [("0e+1o", 2, "0e", 30, B.EQCONV_ERR_UNSUPPORTED),     # C % 4
+             ("0e+1o", 2, "0e", 0, B.EQCONV_ERR_INVALID_ARG),
+             ("0e+1o", 4, "0e", 32, B.EQCONV_ERR_UNSUPPORTED),     # L_sh > 3
+             ("0e+2e", 2, "0e", 32, B.EQCONV_ERR_UNSUPPORTED),     # not a natural prefix
+             ("0e+1o", 2, "bad", 32, B.EQCONV_ERR_INVALID_ARG)]
+    for ins, lsh, outs, C, status in cases:
+        with pytest.raises(B.EqconvError) as e:
+            B.eqconv_plan_create(ins, lsh, outs, C)
+        assert e.value.status == status
+
+
+def test_plan_create_without_a_gpu_fails_loudly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(B.EqconvError) as e:
+        B.eqconv_plan_create("0e+1o", 2, "0e+1o+2e", 32)
+    assert e.value.status == B.EQCONV_ERR_CUDA
+
+
+def test_workspace_sizes():
+    assert B.eqconv_graph_workspace_bytes(10, 0) > 0
+    a = B.eqconv_graph_workspace_bytes(1000, 10000)
+    b = B.eqconv_graph_workspace_bytes(1000, 20000)
+    assert b > a >= 4 * 4 * 10000
+    assert B.eqconv_graph_workspace_bytes(-1, 5) == 0
+
+
+def test_status_strings():
+    for s in range(6):
+        assert B.eqconv_status_string(s).startswith("EQCONV_")
+    assert "unknown" in B.eqconv_status_string(99)
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        B._ptr(torch.zeros(4))

@@ -37,3 +37,9 @@ def test_edge_vector_lengths():
     v = wl.random_edge_vectors(10000)
     n = np.linalg.norm(v, axis=1)
     assert n.min() >= 0.5 - 1e-5 and n.max() <= 5.0 + 1e-5
+
+
+def test_weights_into_matches_weights():
+    out = np.empty((500, 7, 12), dtype=np.float32)
+    wl.weights_into(out, chunk_edges=64)
+    assert np.array_equal(out, wl.weights(500, 7, 12, chunk_edges=200))
