@@ -57,7 +57,8 @@ def byte_counts(N, E, C, D_in, D_out, P):
     step = sum(t.values())
     h2d = sum(t[k] for k in ("senders", "receivers", "x", "r", "w", "gy"))
     d2h = sum(t[k] for k in ("y", "dx", "dw", "dr"))
-    return dict(fwd=fwd, bwd=bwd, graph=graph, step=step, h2d=h2d, d2h=d2h)
+    # headline bytes: each kernel's own inputs and outputs, each counted once
+    return dict(fwd=fwd, bwd=bwd, graph=graph, step=step, h2d=h2d, d2h=d2h, kernels=graph + fwd + bwd)
 
 
 def measured_peak():
@@ -112,7 +113,7 @@ class ClockSampler:
         self.lines = []
 
     def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
         if self.gpu_id:
             cmd += ["-i", self.gpu_id]
         try:
@@ -125,7 +126,7 @@ class ClockSampler:
 
     def _read(self):
         for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+            self.lines.append((time.monotonic(), ln.strip()))
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -136,10 +137,18 @@ class ClockSampler:
                 self.proc.kill()
             self.thread.join(timeout=2)
 
-    def summary(self):
+    def summary(self, window=None):
+        """Median SM clock and the throttle reasons seen; restricted to the
+        timed window when it holds at least 2 samples (else warm-up + timed)."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        scope = "warmup+timed"
+        if window is not None:
+            inside = [(t, ln) for t, ln in lines if window[0] <= t <= window[1]]
+            if len(inside) >= 2:
+                lines, scope = inside, "timed"
+        for _, ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -153,7 +162,26 @@ class ClockSampler:
                     reasons.add(nm)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "scope": scope}
+
+
+# --------------------------------------------------------------------- ranks
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(bytes_per_step: int, steps: int, world: int, t_max_ms: float) -> float:
+    """Whole-job throughput: every rank's bytes over the slowest rank's time."""
+    return bytes_per_step * steps * world / (t_max_ms * 1e-3) / 1e9
 
 
 # --------------------------------------------------------------------- native
@@ -214,13 +242,6 @@ def run_native(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        step()
-    stream.synchronize()
-    assert B.eqconv_get_device_error(conv.plan, sh) == B.EQCONV_OK
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     gpu_id = None
     try:
         gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
@@ -228,26 +249,31 @@ def run_native(args, rank, world, local_rank):
             gpu_id = "GPU-" + gpu_id
     except Exception:
         gpu_id = None
-    barrier()
-    torch.cuda.synchronize(dev)
-    launches0 = B.eqconv_launch_count()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id) as clk:
+        time.sleep(0.3)                      # let the sampler start
+        for _ in range(args.warmup):
+            step()
+        stream.synchronize()
+        assert B.eqconv_get_device_error(conv.plan, sh) == B.EQCONV_OK
+        barrier()
+        torch.cuda.synchronize(dev)
+        launches0 = B.eqconv_launch_count()
+        w0 = time.monotonic()
         t0.record(stream)
         for k in range(args.steps):
             step(evs[k])
         t1.record(stream)
         torch.cuda.synchronize(dev)
+        w1 = time.monotonic()
+        launches = B.eqconv_launch_count() - launches0
         barrier()
-    launches = B.eqconv_launch_count() - launches0
     total_ms = t0.elapsed_time(t1)
     graph_ms = [e[0].elapsed_time(e[1]) for e in evs]
     fwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
     bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    t_max = total_ms
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
+    t_max = reduce_max(total_ms, world, dev)
 
     # non-deterministic backward, timed separately (not part of the step)
     nd_ms = []
@@ -288,19 +314,16 @@ def run_native(args, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         stream.synchronize()
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        e2e = {"value": bc["step"] * e2e_steps * world / (e_ms * 1e-3) / 1e9, "unit": UNIT,
+        e_ms = reduce_max(a.elapsed_time(b), world, dev)
+        e2e = {"value": round(aggregate_gbs(bc["kernels"], e2e_steps, world, e_ms), 2), "unit": UNIT,
                "h2d_bytes_per_step": bc["h2d"], "d2h_bytes_per_step": bc["d2h"],
                "ms_per_step": e_ms / e2e_steps}
 
     peak, peak_kind = measured_peak()
     ms_step = t_max / args.steps
     med = statistics.median
-    value = bc["step"] * args.steps * world / (t_max * 1e-3) / 1e9
+    value = aggregate_gbs(bc["kernels"], args.steps, world, t_max)
+    unique_gbs = aggregate_gbs(bc["step"], args.steps, world, t_max)
     fwd_gbs = bc["fwd"] / (med(fwd_ms) * 1e-3) / 1e9
     bwd_gbs = bc["bwd"] / (med(bwd_ms) * 1e-3) / 1e9
     fb_gbs = (bc["fwd"] + bc["bwd"]) / ((med(fwd_ms) + med(bwd_ms)) * 1e-3) / 1e9
@@ -317,8 +340,11 @@ def run_native(args, rank, world, local_rank):
             "step": "graph build (recv+send CSR) + fused forward + fused deterministic backward",
             "l2": "inputs larger than L2 (w alone is %.1f GB)" % (bc["step"] and 4 * E * P * C / 1e9),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "unique_bytes_per_step": bc["step"],
+            "bytes_per_step": bc["kernels"],
+            "bytes": "per kernel: every tensor it reads or writes, counted once (graph build + forward + "
+                     "backward); GB/s = bytes / device time",
         },
+        "unique_bytes_step_gbps": round(unique_gbs, 1),
         "fwd_gbps": round(fwd_gbs, 1), "bwd_gbps": round(bwd_gbs, 1), "fwd_bwd_gbps": round(fb_gbs, 1),
         "hbm_frac_fwd_bwd": round(fb_gbs / peak, 4),
         "edges_per_s_fwd": round(E / (med(fwd_ms) * 1e-3), 1),
@@ -334,7 +360,7 @@ def run_native(args, rank, world, local_rank):
                          "frac": round(bc["fwd"] / (fwd_avg * 1e-3) / 1e9 / peak, 4), "traffic": traffic.get("fwd"),
                          "algorithmic_bytes": bc["fwd"]},
         "gpu_launches": int(launches),
-        "clocks": clk.summary(),
+        "clocks": clk.summary((w0, w1)),
     }
     if e2e:
         result["e2e"] = e2e
@@ -386,8 +412,13 @@ def cpu_baseline(name, D_in, D_out, P, target_s, bytes_step, E_full):
     W = wl.WORKLOADS[name]
     x = wl.features(W.N, D_in, W.C, wl.SEED_X)
     gy = wl.features(W.N, D_out, W.C, wl.SEED_GY)
-    t0, k0 = oracle_sample_step(name, 16, D_in, D_out, P, x, gy)
-    n_recv = int(min(W.N, max(16, 16 * target_s / max(t0, 1e-3))))
+    n_recv, t = 16, 0.0
+    while n_recv < W.N:                       # grow the sample until it is long enough to scale
+        t, k = oracle_sample_step(name, n_recv, D_in, D_out, P, x, gy)
+        if t >= target_s / 8:
+            break
+        n_recv = min(W.N, n_recv * 4)
+    n_recv = int(min(W.N, max(16, n_recv * target_s / max(t, 1e-3))))
     t, k = oracle_sample_step(name, n_recv, D_in, D_out, P, x, gy)
     frac = k / E_full
     return {"value": round(bytes_step * frac / t / 1e9, 4), "unit": UNIT, "cores": oconv.max_threads(),
@@ -418,7 +449,7 @@ def run_reference(args, rank, world):
         t, k = oracle_sample_step(args.workload, n_recv, prob.D_in, prob.D_out, prob.P, x, gy)
         tot += t
     frac = k / E
-    value = bc["step"] * frac * args.steps / tot / 1e9
+    value = bc["kernels"] * frac * args.steps / tot / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot / args.steps, 2),
@@ -449,7 +480,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
+    ap.add_argument("--nodes", type=int, default=None,
+                    help="override the workload's node count (smaller profiling captures)")
     args = ap.parse_args()
+    if args.nodes:
+        import dataclasses
+        base = wl.WORKLOADS[args.workload]
+        name = f"{base.name}_N{args.nodes}"
+        wl.WORKLOADS[name] = dataclasses.replace(base, name=name, N=args.nodes)
+        args.workload = name
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
 
@@ -476,7 +515,7 @@ def main():
             obuild.build()
             N, E, C, D_in, D_out, P = dims
             result["cpu_baseline"] = cpu_baseline(args.workload, D_in, D_out, P, args.cpu_seconds,
-                                                  byte_counts(N, E, C, D_in, D_out, P)["step"], E)
+                                                  byte_counts(N, E, C, D_in, D_out, P)["kernels"], E)
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:

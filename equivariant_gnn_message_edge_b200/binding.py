@@ -30,12 +30,16 @@ ABI_FUNCTIONS = (
     "eqconv_graph_workspace_bytes", "eqconv_graph_build", "eqconv_forward",
     "eqconv_backward_workspace_bytes", "eqconv_backward", "eqconv_spherical_harmonics",
     "eqconv_get_device_error", "eqconv_plan_destroy", "eqconv_status_string", "eqconv_launch_count",
+    "eqconv_last_error",
 )
 
 
 class EqconvError(RuntimeError):
     def __init__(self, what: str, status: int):
-        super().__init__(f"{what}: {eqconv_status_string(status)} (status {status})")
+        msg = f"{what}: {eqconv_status_string(status)} (status {status})"
+        if status == EQCONV_ERR_CUDA:
+            msg += f" [{eqconv_last_error()}]"
+        super().__init__(msg)
         self.status = status
 
 
@@ -69,6 +73,7 @@ _SIGS = {
     "eqconv_plan_destroy": (None, [_vp]),
     "eqconv_status_string": (ctypes.c_char_p, [_ci]),
     "eqconv_launch_count": (ctypes.c_ulonglong, []),
+    "eqconv_last_error": (ctypes.c_char_p, []),
 }
 
 
@@ -134,6 +139,10 @@ def _i32():
 
 def eqconv_status_string(status: int) -> str:
     return lib().eqconv_status_string(int(status)).decode()
+
+
+def eqconv_last_error() -> str:
+    return lib().eqconv_last_error().decode()
 
 
 def eqconv_launch_count() -> int:

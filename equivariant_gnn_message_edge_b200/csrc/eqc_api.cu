@@ -10,6 +10,7 @@
 #include <atomic>
 #include <cctype>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <new>
 #include <string>
@@ -23,6 +24,12 @@ namespace eqc {
 
 static std::atomic<unsigned long long> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// Last CUDA failure seen by an entry point of this thread (for diagnostics).
+static thread_local char g_last_error[256] = "no error";
+static void note_error(const char* where, cudaError_t e) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
 
 template <int LSH>
 static cudaError_t dr_epi(const float* gy_part, int T, const float* r, float* dr, int E, cudaStream_t st) {
@@ -134,7 +141,11 @@ int check_graph(const eqconv_graph_t* g) {
     return EQCONV_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? EQCONV_OK : EQCONV_ERR_CUDA; }
+int cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return EQCONV_OK;
+    eqc::note_error(where, e);
+    return EQCONV_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -260,7 +271,8 @@ int eqconv_graph_build(eqconv_plan_t plan, const eqconv_graph_t* g, void* worksp
     const size_t need = eqc::graph_workspace_bytes(g->N, g->E);
     if (!workspace || workspace_bytes < need) return EQCONV_ERR_WORKSPACE;
     return cuda_status(eqc::graph_build(g->N, g->E, g->senders, g->receivers, g->recv_ptr, g->recv_perm, g->send_ptr,
-                                        g->send_perm, workspace, plan->d_status, (cudaStream_t)stream));
+                                        g->send_perm, workspace, plan->d_status, (cudaStream_t)stream),
+                       "graph_build");
 }
 
 int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r, const float* w,
@@ -275,7 +287,7 @@ int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, 
     if (!aligned16(x) || !aligned16(y) || !aligned16(w)) return EQCONV_ERR_INVALID_ARG;
     eqc::FwdParams prm{x, r, w, y, g->recv_ptr, g->recv_perm, g->senders, g->N, plan->C, plan->d_status};
     const int T = tiles_for(plan->C, plan->fwd_vec);
-    return cuda_status(plan->fwd_ks->fwd(prm, T, (cudaStream_t)stream));
+    return cuda_status(plan->fwd_ks->fwd(prm, T, (cudaStream_t)stream), "forward");
 }
 
 size_t eqconv_backward_workspace_bytes(eqconv_plan_t plan, int E) {
@@ -308,14 +320,16 @@ int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
         const int64_t n4 = (int64_t)g->N * plan->D_in * plan->C / 4;
         eqc::k_zero_f4<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(reinterpret_cast<float4*>(dx), n4);
         eqc::count_launch();
-        if (cudaGetLastError() != cudaSuccess) return EQCONV_ERR_CUDA;
+        const cudaError_t ze = cudaGetLastError();
+        if (ze != cudaSuccess) return cuda_status(ze, "backward zero dx");
     }
     if (g->E == 0) {
         if (det) {
             const int64_t n4 = (int64_t)g->N * plan->D_in * plan->C / 4;
             eqc::k_zero_f4<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(reinterpret_cast<float4*>(dx), n4);
             eqc::count_launch();
-            if (cudaGetLastError() != cudaSuccess) return EQCONV_ERR_CUDA;
+            const cudaError_t ze = cudaGetLastError();
+            if (ze != cudaSuccess) return cuda_status(ze, "backward zero dx");
         }
         return EQCONV_OK;
     }
@@ -336,16 +350,16 @@ int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
     prm.T = T;
     prm.status = plan->d_status;
     cudaError_t err = plan->bwd_ks->bwd(prm, det, fused, st);
-    if (err != cudaSuccess) return EQCONV_ERR_CUDA;
+    if (err != cudaSuccess) return cuda_status(err, det ? "backward (deterministic)" : "backward (atomic)");
     if (!fused) err = eqc::launch_dr_epilogue(plan->lsh, prm.gy_part, T, r, dr, g->E, st);
-    return cuda_status(err);
+    return cuda_status(err, "dr epilogue");
 }
 
 int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y, eqconv_stream_t stream) {
     if (!plan || E < 0 || (E > 0 && (!r || !Y))) return EQCONV_ERR_INVALID_ARG;
     int rc = check_device(plan);
     if (rc != EQCONV_OK) return rc;
-    return cuda_status(eqc::launch_sh(plan->lsh, r, Y, E, (cudaStream_t)stream));
+    return cuda_status(eqc::launch_sh(plan->lsh, r, Y, E, (cudaStream_t)stream), "spherical harmonics");
 }
 
 int eqconv_get_device_error(eqconv_plan_t plan, eqconv_stream_t stream, int* status) {
@@ -353,7 +367,8 @@ int eqconv_get_device_error(eqconv_plan_t plan, eqconv_stream_t stream, int* sta
     int rc = check_device(plan);
     if (rc != EQCONV_OK) return rc;
     unsigned h = 0;
-    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return EQCONV_ERR_CUDA;
+    const cudaError_t se = cudaStreamSynchronize((cudaStream_t)stream);
+    if (se != cudaSuccess) return cuda_status(se, "get_device_error sync");
     if (cudaMemcpy(&h, plan->d_status, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
         return EQCONV_ERR_CUDA;
     if (h != 0 && cudaMemset(plan->d_status, 0, sizeof(unsigned)) != cudaSuccess) return EQCONV_ERR_CUDA;
@@ -384,5 +399,7 @@ const char* eqconv_status_string(int status) {
 }
 
 unsigned long long eqconv_launch_count(void) { return eqc::g_launches.load(std::memory_order_relaxed); }
+
+const char* eqconv_last_error(void) { return eqc::g_last_error; }
 
 }  // extern "C"

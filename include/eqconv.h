@@ -159,6 +159,11 @@ EQCONV_API void eqconv_plan_destroy(eqconv_plan_t plan);
 
 EQCONV_API const char* eqconv_status_string(int status);
 
+/* Text of the last CUDA failure an entry point of the calling thread
+ * reported as EQCONV_ERR_CUDA (where, error name, description).  Owned by the
+ * library; valid until the thread's next failing call. */
+EQCONV_API const char* eqconv_last_error(void);
+
 /* Number of kernels this library has launched in this process (all devices). */
 EQCONV_API unsigned long long eqconv_launch_count(void);
 
