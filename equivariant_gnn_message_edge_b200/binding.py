@@ -30,7 +30,7 @@ ABI_FUNCTIONS = (
     "eqconv_graph_workspace_bytes", "eqconv_graph_build", "eqconv_forward",
     "eqconv_backward_workspace_bytes", "eqconv_backward", "eqconv_spherical_harmonics",
     "eqconv_get_device_error", "eqconv_plan_destroy", "eqconv_status_string", "eqconv_launch_count",
-    "eqconv_last_error",
+    "eqconv_last_error", "eqconv_graph_build_noalloc",
 )
 
 
@@ -65,6 +65,7 @@ _SIGS = {
     "eqconv_cg_table": (_ci, [_ci, _ci, _ci, _pd, _ci]),
     "eqconv_graph_workspace_bytes": (_sz, [_ci, _ci]),
     "eqconv_graph_build": (_ci, [_vp, _pg, _vp, _sz, _vp]),
+    "eqconv_graph_build_noalloc": (_ci, [_vp, _pg, _vp]),
     "eqconv_forward": (_ci, [_vp, _pg, _vp, _vp, _vp, _vp, _cu, _vp]),
     "eqconv_backward_workspace_bytes": (_sz, [_vp, _ci]),
     "eqconv_backward": (_ci, [_vp, _pg, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _cu, _vp]),
@@ -193,6 +194,13 @@ def eqconv_graph_workspace_bytes(N: int, E: int) -> int:
 def eqconv_graph_build(plan: int, graph: eqconv_graph_t, workspace, workspace_bytes: int, stream=None) -> None:
     _check(lib().eqconv_graph_build(plan, ctypes.byref(graph), _ptr(workspace), int(workspace_bytes),
                                     _stream(stream)), "eqconv_graph_build")
+
+
+def eqconv_graph_build_noalloc(plan: int, graph: eqconv_graph_t, stream=None) -> None:
+    """eqconv_graph_build without workspace or allocation (scratch in the
+    library's fixed 8 MiB device array; see include/eqconv.h)."""
+    _check(lib().eqconv_graph_build_noalloc(plan, ctypes.byref(graph), _stream(stream)),
+           "eqconv_graph_build_noalloc")
 
 
 def eqconv_forward(plan: int, graph: eqconv_graph_t, x, r, w, y, flags: int = 0, stream=None) -> None:

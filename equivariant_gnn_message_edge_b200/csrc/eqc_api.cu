@@ -275,6 +275,24 @@ int eqconv_graph_build(eqconv_plan_t plan, const eqconv_graph_t* g, void* worksp
                        "graph_build");
 }
 
+int eqconv_graph_build_noalloc(eqconv_plan_t plan, const eqconv_graph_t* g, eqconv_stream_t stream) {
+    if (!plan) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_graph(g);
+    if (rc != EQCONV_OK) return rc;
+    if ((rc = check_device(plan)) != EQCONV_OK) return rc;
+    bool too_large = false;
+    const cudaError_t err =
+        eqc::graph_build_noalloc(g->N, g->E, g->senders, g->receivers, g->recv_ptr, g->recv_perm, g->send_ptr,
+                                 g->send_perm, plan->d_status, (cudaStream_t)stream, &too_large);
+    if (too_large) {
+        snprintf(eqc::g_last_error, sizeof(eqc::g_last_error),
+                 "graph_build_noalloc: N=%d, E=%d needs %zu bytes of scratch; the fixed scratch holds %zu",
+                 g->N, g->E, eqc::graph_workspace_bytes(g->N, g->E), eqc::kGraphScratchBytes);
+        return EQCONV_ERR_WORKSPACE;
+    }
+    return cuda_status(err, "graph_build_noalloc");
+}
+
 int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r, const float* w,
                    float* y, unsigned flags, eqconv_stream_t stream) {
     (void)flags;

@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "eqc_graph.h"
 
@@ -271,6 +272,51 @@ cudaError_t graph_build(int N, int E, const int* senders, const int* receivers, 
     cudaError_t err = build_csr(receivers, N, E, recv_ptr, recv_perm, static_cast<char*>(ws), status, st);
     if (err != cudaSuccess) return err;
     return build_csr(senders, N, E, send_ptr, send_perm, static_cast<char*>(ws), status, st);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of graph_build.
+//
+// Some callers cannot allocate device memory: for example a plugin called
+// inside another program's simulation step, where the host program owns all
+// device memory, or code that must not call cudaMalloc because it blocks the
+// device.  For them the radix-sort scratch lives in this fixed array, which
+// every GPU that loads the library holds until the process exits.  Host code
+// must not pass `g_graph_scratch` itself to a kernel: on the host it is only
+// a stand-in symbol, not a device address.  Its device address is looked up
+// once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_graph_scratch[kGraphScratchBytes];
+
+cudaError_t graph_build_noalloc(int N, int E, const int* senders, const int* receivers, int* recv_ptr,
+                                int* recv_perm, int* send_ptr, int* send_perm, unsigned* status, cudaStream_t st,
+                                bool* too_large) {
+    *too_large = false;
+    if (graph_workspace_bytes(N, E) > kGraphScratchBytes) {
+        *too_large = true;
+        return cudaSuccess;
+    }
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!addr[dev]) {
+            err = cudaGetSymbolAddress(&addr[dev], g_graph_scratch);
+            if (err != cudaSuccess) {
+                addr[dev] = nullptr;
+                return err;
+            }
+        }
+        scratch = addr[dev];
+    }
+    // Every word of scratch that must start at zero (the key counts) is
+    // zeroed inside build_csr on each call; histograms and sort buffers are
+    // fully overwritten before they are read.
+    return graph_build(N, E, senders, receivers, recv_ptr, recv_perm, send_ptr, send_perm, scratch, status, st);
 }
 
 }  // namespace eqc

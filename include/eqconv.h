@@ -127,6 +127,27 @@ EQCONV_API size_t eqconv_graph_workspace_bytes(int N, int E);
 EQCONV_API int eqconv_graph_build(eqconv_plan_t plan, const eqconv_graph_t* g, void* workspace,
                        size_t workspace_bytes, eqconv_stream_t stream);
 
+/* Same result as eqconv_graph_build, for callers that cannot allocate device
+ * memory: a plugin running inside another program's simulation step where
+ * the host program owns every device allocation, or code that must not call
+ * cudaMalloc because cudaMalloc can block the device.  It takes no workspace
+ * and allocates nothing.  Its scratch is a fixed 8 MiB device array inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits.  (The pages have no counterpart to this entry point.)
+ *   - Limit: eqconv_graph_workspace_bytes(N, E) must be <= 8 MiB (about
+ *     16.5 B per edge + 4 B per node; e.g. E <= 480k edges at N <= 100k).
+ *     Larger graphs return EQCONV_ERR_WORKSPACE and launch nothing;
+ *     eqconv_last_error then states the bytes needed.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU (on two
+ *     streams, or from two threads) race and corrupt each other's result.
+ *     The scratch keeps the last call's contents; each call clears what it
+ *     needs zeroed itself. */
+EQCONV_API int eqconv_graph_build_noalloc(eqconv_plan_t plan, const eqconv_graph_t* g,
+                                          eqconv_stream_t stream);
+
 /* Forward (one fused kernel; receiver-sorted, atomic-free, no per-edge
  * messages in memory; deterministic): writes y [N][D_out][C]. */
 EQCONV_API int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
