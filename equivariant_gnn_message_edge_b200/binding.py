@@ -15,7 +15,8 @@ import threading
 
 import numpy as np
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libeqconv.so")
+LIB_PATH = os.environ.get("EQCONV_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                             "libeqconv.so")
 
 EQCONV_OK = 0
 EQCONV_ERR_INVALID_ARG = 1

@@ -7,7 +7,10 @@
 // stream.  Nothing here allocates per call.
 #include <cuda_runtime.h>
 
+#include <cudaTypedefs.h>
+
 #include <atomic>
+#include <mutex>
 #include <cctype>
 #include <cstdint>
 #include <cstdio>
@@ -68,6 +71,38 @@ cudaError_t launch_sh(int lsh, const float* r, float* Y, int E, cudaStream_t st)
     }
 }
 
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t count, int rows, int C, int tile_c) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc || !base || count == 0 || rows <= 0 || rows > 256 || tile_c > 256) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)rows, (cuuint64_t)count};
+    const cuuint64_t strides[2] = {(cuuint64_t)C * 4u, (cuuint64_t)rows * (cuuint64_t)C * 4u};
+    const cuuint32_t box[3] = {(cuuint32_t)tile_c, (cuuint32_t)rows, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    // promote L2 fills to the box row width at most: a wider promotion would
+    // fetch the neighbouring channel tile, which is not read until much later
+    const int row_bytes = tile_c * 4;
+    const CUtensorMapL2promotion promo = row_bytes >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                         : row_bytes >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                            : CU_TENSOR_MAP_L2_PROMOTION_NONE;
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, promo,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 __global__ void k_zero_f4(float4* p, int64_t n4) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n4) p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -77,13 +112,14 @@ __global__ void k_zero_f4(float4* p, int64_t n4) {
 
 struct eqconv_plan_s {
     int lin, lsh, lout, C;
-    int fwd_vec, bwd_vec;
+    int fwd_vec, det_vec, atomic_vec;
     int P, D_in, D_sh, D_out;
     int paths[eqc::kMaxPaths][3];
     int device;
     unsigned* d_status;
     const eqc::KernelSet* fwd_ks;
-    const eqc::KernelSet* bwd_ks;
+    const eqc::KernelSet* det_ks;      // deterministic backward
+    const eqc::KernelSet* atomic_ks;   // atomic backward
 };
 
 namespace {
@@ -122,9 +158,15 @@ int parse_natural_prefix(const char* s) {
     return expect - 1;
 }
 
-int default_vec(int C) { return C >= 128 ? 4 : 2; }
+// Channel vector widths measured best on B200 at C = 128 (lmax 2 and 3):
+// 64-channel tiles for the forward and the atomic backward (their gathered
+// rows stay in L2 and more warps fit), 128-channel tiles for the
+// deterministic backward (fewer coupling-matrix builds per edge).
+int default_fwd_vec(int) { return 2; }
+int default_det_vec(int C) { return C >= 128 ? 4 : 2; }
+int default_atomic_vec(int) { return 2; }
 
-int tiles_for(int C, int vec) { return (C + 32 * vec - 1) / (32 * vec); }
+int tiles_for(int C, int tile_c) { return (C + tile_c - 1) / tile_c; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -177,10 +219,13 @@ int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh, cons
         p->paths[i][1] = PL.l2[i];
         p->paths[i][2] = PL.l3[i];
     }
-    p->fwd_vec = p->bwd_vec = default_vec(C);
+    p->fwd_vec = default_fwd_vec(C);
+    p->det_vec = default_det_vec(C);
+    p->atomic_vec = default_atomic_vec(C);
     p->fwd_ks = eqc::find_instance(lin, L_sh, lout, p->fwd_vec);
-    p->bwd_ks = eqc::find_instance(lin, L_sh, lout, p->bwd_vec);
-    if (!p->fwd_ks || !p->bwd_ks) {
+    p->det_ks = eqc::find_instance(lin, L_sh, lout, p->det_vec);
+    p->atomic_ks = eqc::find_instance(lin, L_sh, lout, p->atomic_vec);
+    if (!p->fwd_ks || !p->det_ks || !p->atomic_ks) {
         delete p;
         return EQCONV_ERR_UNSUPPORTED;
     }
@@ -204,9 +249,9 @@ int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec) {
     const eqc::KernelSet* b = eqc::find_instance(plan->lin, plan->lsh, plan->lout, bwd_vec);
     if (!f || !b) return EQCONV_ERR_UNSUPPORTED;
     plan->fwd_vec = fwd_vec;
-    plan->bwd_vec = bwd_vec;
+    plan->det_vec = plan->atomic_vec = bwd_vec;
     plan->fwd_ks = f;
-    plan->bwd_ks = b;
+    plan->det_ks = plan->atomic_ks = b;
     return EQCONV_OK;
 }
 
@@ -303,17 +348,22 @@ int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, 
     if (g->N == 0) return EQCONV_OK;
     if (!x || !y || (g->E > 0 && (!r || !w))) return EQCONV_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(y) || !aligned16(w)) return EQCONV_ERR_INVALID_ARG;
-    eqc::FwdParams prm{x, r, w, y, g->recv_ptr, g->recv_perm, g->senders, g->N, plan->C, plan->d_status};
-    const int T = tiles_for(plan->C, plan->fwd_vec);
+    eqc::FwdParams prm{x, r, w, y, g->recv_ptr, g->recv_perm, g->senders, g->N, plan->C, g->E, plan->d_status};
+    const int T = tiles_for(plan->C, plan->fwd_ks->tile_c);
     return cuda_status(plan->fwd_ks->fwd(prm, T, (cudaStream_t)stream), "forward");
+}
+
+static size_t bwd_ws_bytes(eqconv_plan_t plan, const eqc::KernelSet* ks, int E) {
+    const int T = tiles_for(plan->C, ks->tile_c);
+    const int G = plan->D_sh - 1;
+    if (T == 1 || G == 0) return 0;
+    return (size_t)E * T * G * sizeof(float);
 }
 
 size_t eqconv_backward_workspace_bytes(eqconv_plan_t plan, int E) {
     if (!plan || E < 0) return 0;
-    const int T = tiles_for(plan->C, plan->bwd_vec);
-    const int G = plan->D_sh - 1;
-    if (T == 1 || G == 0) return 0;
-    return (size_t)E * T * G * sizeof(float);
+    const size_t a = bwd_ws_bytes(plan, plan->det_ks, E), b = bwd_ws_bytes(plan, plan->atomic_ks, E);
+    return a > b ? a : b;
 }
 
 int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r, const float* w,
@@ -329,10 +379,11 @@ int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
         return EQCONV_ERR_INVALID_ARG;
     const cudaStream_t st = (cudaStream_t)stream;
     const bool det = (flags & EQCONV_DETERMINISTIC) != 0;
-    const int T = tiles_for(plan->C, plan->bwd_vec);
+    const eqc::KernelSet* ks = det ? plan->det_ks : plan->atomic_ks;
+    const int T = tiles_for(plan->C, ks->tile_c);
     const int G = plan->D_sh - 1;
     const bool fused = (T == 1) || (G == 0);
-    const size_t need = eqconv_backward_workspace_bytes(plan, g->E);
+    const size_t need = bwd_ws_bytes(plan, ks, g->E);
     if (need > 0 && (!workspace || workspace_bytes < need)) return EQCONV_ERR_WORKSPACE;
     if (!det) {
         const int64_t n4 = (int64_t)g->N * plan->D_in * plan->C / 4;
@@ -366,8 +417,9 @@ int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
     prm.N = g->N;
     prm.C = plan->C;
     prm.T = T;
+    prm.E = g->E;
     prm.status = plan->d_status;
-    cudaError_t err = plan->bwd_ks->bwd(prm, det, fused, st);
+    cudaError_t err = ks->bwd(prm, det, fused, st);
     if (err != cudaSuccess) return cuda_status(err, det ? "backward (deterministic)" : "backward (atomic)");
     if (!fused) err = eqc::launch_dr_epilogue(plan->lsh, prm.gy_part, T, r, dr, g->E, st);
     return cuda_status(err, "dr epilogue");

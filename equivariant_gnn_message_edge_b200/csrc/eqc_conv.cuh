@@ -28,12 +28,22 @@
 // (x or gy, reused ~45 times) carry evict-last hints.
 #pragma once
 
+#include <cuda.h>
+
 #include <cstdint>
 #include <type_traits>
 #include <utility>
 
 #include "eqc_sh.cuh"
 #include "eqc_tables.h"
+
+// Build-time tuning knobs (defaults are the tuned values).
+#ifndef EQC_STAGES
+#define EQC_STAGES 2
+#endif
+#ifndef EQC_CHUNK_SMALL
+#define EQC_CHUNK_SMALL 0   // 0: 16 edges at VEC=4, 8 at narrower tiles
+#endif
 
 namespace eqc {
 
@@ -66,16 +76,18 @@ struct Cfg {
     static constexpr AOffsets AO = make_aoffsets(PL);
     static constexpr int NA = AO.total;
     static constexpr int NA_PAD = pad_odd4(NA);     // row stride; NA_PAD/4 odd: conflict-free STS.128
-    static constexpr int CHUNK = NA_PAD <= 128 ? 32 : (NA_PAD <= 256 ? 16 : 8);
+    // edges whose coupling matrices A sit in shared memory at a time
+    static constexpr int CHUNK = NA_PAD > 128 ? 8 : (EQC_CHUNK_SMALL > 0 ? EQC_CHUNK_SMALL : (VEC >= 4 ? 16 : 8));
     static constexpr int GS = G | 1;                // gY row stride in shared memory (odd)
-    static constexpr int WARPS = 4;
     static constexpr int TILE_C = 32 * VEC;
-    // register estimate of the double-buffered edge rows
-    static constexpr int FWD_ROWS = (D_IN + NP) * VEC;
-    static constexpr bool FWD_PREFETCH = 2 * FWD_ROWS + D_OUT * VEC <= 160;
-    static constexpr bool BWD_PREFETCH = 2 * (D_OUT + NP) * VEC + 2 * D_IN * VEC <= 160;
-    static constexpr int FWD_SMEM = WARPS * CHUNK * NA_PAD * 4;
-    static constexpr int BWD_SMEM = WARPS * CHUNK * (NA_PAD + GS) * 4;
+    static constexpr int STAGES = EQC_STAGES;       // edges staged ahead per warp (ring depth)
+    // per-warp shared memory (bytes) of the largest kernel of this instance,
+    // used to size the CTA so that two CTAs fit on one SM (<= 113 KB each)
+    static constexpr int WARP_BYTES_EST =
+        4 * (32 + ((CHUNK * NA_PAD + 31) & ~31) + ((CHUNK * GS + 31) & ~31) +
+             STAGES * (NP + (D_IN > D_OUT ? D_IN : D_OUT)) * TILE_C);
+    static constexpr int WARPS_FIT = (113 * 1024) / WARP_BYTES_EST;
+    static constexpr int WARPS = WARPS_FIT < 1 ? 1 : (WARPS_FIT > 4 ? 4 : WARPS_FIT);
     static_assert(NP > 0, "no admissible path");
 };
 
@@ -94,7 +106,9 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 
 template <int VEC>
 __device__ __forceinline__ void ld_stream(float* d, const float* p, uint64_t pol) {
-    if constexpr (VEC == 4) {
+    if constexpr (VEC == 1) {
+        asm("ld.global.nc.L1::no_allocate.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(d[0]) : "l"(p), "l"(pol));
+    } else if constexpr (VEC == 4) {
         asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0,%1,%2,%3}, [%4], %5;"
             : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
             : "l"(p), "l"(pol));
@@ -106,7 +120,9 @@ __device__ __forceinline__ void ld_stream(float* d, const float* p, uint64_t pol
 }
 template <int VEC>
 __device__ __forceinline__ void ld_keep(float* d, const float* p, uint64_t pol) {
-    if constexpr (VEC == 4) {
+    if constexpr (VEC == 1) {
+        asm("ld.global.nc.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(d[0]) : "l"(p), "l"(pol));
+    } else if constexpr (VEC == 4) {
         asm("ld.global.nc.L2::cache_hint.v4.f32 {%0,%1,%2,%3}, [%4], %5;"
             : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
             : "l"(p), "l"(pol));
@@ -118,24 +134,47 @@ __device__ __forceinline__ void ld_keep(float* d, const float* p, uint64_t pol) 
 }
 template <int VEC>
 __device__ __forceinline__ void st_plain(float* p, const float* v) {
-    if constexpr (VEC == 4)
+    if constexpr (VEC == 1)
+        *p = v[0];
+    else if constexpr (VEC == 4)
         *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
     else
         *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
 }
 template <int VEC>
 __device__ __forceinline__ void st_stream(float* p, const float* v) {
-    if constexpr (VEC == 4)
+    if constexpr (VEC == 1)
+        __stcs(p, v[0]);
+    else if constexpr (VEC == 4)
         __stcs(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
     else
         __stcs(reinterpret_cast<float2*>(p), make_float2(v[0], v[1]));
 }
 template <int VEC>
 __device__ __forceinline__ void red_add(float* p, const float* v) {
-    if constexpr (VEC == 4)
+    if constexpr (VEC == 1)
+        atomicAdd(p, v[0]);
+    else if constexpr (VEC == 4)
         atomicAdd(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
     else
         atomicAdd(reinterpret_cast<float2*>(p), make_float2(v[0], v[1]));
+}
+
+template <int V>
+__device__ __forceinline__ void lds_vec(float* d, const float* p) {
+    if constexpr (V == 1) {
+        d[0] = *p;
+    } else if constexpr (V == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(p);
+        d[0] = t.x;
+        d[1] = t.y;
+        d[2] = t.z;
+        d[3] = t.w;
+    } else {
+        const float2 t = *reinterpret_cast<const float2*>(p);
+        d[0] = t.x;
+        d[1] = t.y;
+    }
 }
 
 // ------------------------------------------------------- per-edge coupling A
@@ -245,24 +284,72 @@ __device__ __forceinline__ void fwd_edge(const float* As, const float (&xv)[K::D
 
 // ----------------------------------------------------------- backward math
 
-// Given x (sender rows), g (receiver output-gradient rows) and w for one edge:
-// dw[p] (stored through `dwp`), dx += w_p A_p^T g, gyl += per-lane partial of gY.
-template <class K, class StoreDw>
-__device__ __forceinline__ void bwd_edge(const float* As, const float (&xv)[K::D_IN][K::VEC],
-                                         const float (&gv)[K::D_OUT][K::VEC], const float (&wv)[K::NP][K::VEC],
-                                         float (&dxv)[K::D_IN][K::VEC], float (&gyl)[K::G > 0 ? K::G : 1],
-                                         StoreDw&& store_dw) {
+// Row accessors for the per-edge math: a row block lives either in registers
+// (the warp's resident node) or in the shared-memory stage of the edge; the
+// math asks for one row (component) at a time so that only the rows of the
+// current path are live in registers.
+template <int V, int D>
+struct RegRows {
+    const float (&r)[D][V];
+    __device__ __forceinline__ void get(int d, float* out) const {
+#pragma unroll
+        for (int v = 0; v < V; ++v) out[v] = r[d][v];
+    }
+};
+template <int V>
+struct SmemRows {
+    const float* base;  // row 0 of this lane's channels
+    int stride;         // floats between rows
+    bool on;            // false: rows read as zero (inactive lane or invalid edge)
+    __device__ __forceinline__ void get(int d, float* out) const {
+        if (on) {
+            lds_vec<V>(out, base + d * stride);
+        } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) out[v] = 0.f;
+        }
+    }
+};
+
+// One edge of the backward: with x (sender rows), g (receiver output-gradient
+// rows) and w (weight rows) given by accessors,
+//   t_p = A_p^T g_l3,  dw_p = x_l1 . t_p (stored through store_dw),
+//   dx_l1 += w_p t_p,  gyl[l2 m2] += w_p sum_{m1,m3} C_p[m1,m2,m3] x[m1] g[m3]
+// (gyl is this lane's partial over its channels).
+// DIRECT: dx accumulates straight into dx_full (the deterministic pass keeps
+// its sender's dx in registers).  Otherwise the dx of one input block (paths
+// are ordered by l1) is summed in a small block and handed to
+// dx_sink(o1, d1, block) after the block's last path (atomic pass).
+template <class K, bool DIRECT, class XR, class GR, class WR, class StoreDw, class DxSink>
+__device__ __forceinline__ void bwd_edge(const float* As, const XR& X, const GR& Gr, const WR& Wr,
+                                         float (&dx_full)[DIRECT ? K::D_IN : 1][K::VEC], DxSink&& dx_sink,
+                                         float (&gyl)[K::G > 0 ? K::G : 1], StoreDw&& store_dw) {
     constexpr int V = K::VEC;
+    float dxg[DIRECT ? 1 : 2 * kMaxL + 1][V];
     static_for<K::NP>([&](auto pc) {
         constexpr int p = EQC_CV(pc);
         constexpr int l1 = K::PL.l1[p], l2 = K::PL.l2[p], l3 = K::PL.l3[p];
         constexpr int d1 = 2 * l1 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o3 = l3 * l3;
+        [[maybe_unused]] constexpr bool first_of_block = (p == 0) || (K::PL.l1[p == 0 ? 0 : p - 1] != l1);
+        [[maybe_unused]] constexpr bool last_of_block = (p == K::NP - 1) || (K::PL.l1[p + 1 < K::NP ? p + 1 : p] != l1);
+        if constexpr (!DIRECT && first_of_block) {
+#pragma unroll
+            for (int m = 0; m < d1; ++m)
+#pragma unroll
+                for (int v = 0; v < V; ++v) dxg[m][v] = 0.f;
+        }
+        float gv[d3][V], xv[d1][V], wp[V];
+#pragma unroll
+        for (int m = 0; m < d3; ++m) Gr.get(o3 + m, gv[m]);
+#pragma unroll
+        for (int m = 0; m < d1; ++m) X.get(o1 + m, xv[m]);
+        Wr.get(p, wp);
         float t[d1][V];
         if constexpr (l2 == 0) {
 #pragma unroll
             for (int m = 0; m < d1; ++m)
 #pragma unroll
-                for (int v = 0; v < V; ++v) t[m][v] = gv[o3 + m][v];
+                for (int v = 0; v < V; ++v) t[m][v] = gv[m][v];
         } else {
             constexpr int n4 = (d1 * d3 + 3) / 4;
             constexpr int aoff = K::AO.off[p];
@@ -271,26 +358,34 @@ __device__ __forceinline__ void bwd_edge(const float* As, const float (&xv)[K::D
 #pragma unroll
             for (int m1 = 0; m1 < d1; ++m1) {
 #pragma unroll
-                for (int v = 0; v < V; ++v) t[m1][v] = a[m1] * gv[o3][v];
+                for (int v = 0; v < V; ++v) t[m1][v] = a[m1] * gv[0][v];
 #pragma unroll
                 for (int m3 = 1; m3 < d3; ++m3)
 #pragma unroll
-                    for (int v = 0; v < V; ++v) t[m1][v] = fmaf(a[m3 * d1 + m1], gv[o3 + m3][v], t[m1][v]);
+                    for (int v = 0; v < V; ++v) t[m1][v] = fmaf(a[m3 * d1 + m1], gv[m3][v], t[m1][v]);
             }
         }
         float dw[V];
 #pragma unroll
         for (int v = 0; v < V; ++v) {
-            float s = xv[o1][v] * t[0][v];
+            float s = xv[0][v] * t[0][v];
 #pragma unroll
-            for (int m1 = 1; m1 < d1; ++m1) s = fmaf(xv[o1 + m1][v], t[m1][v], s);
+            for (int m1 = 1; m1 < d1; ++m1) s = fmaf(xv[m1][v], t[m1][v], s);
             dw[v] = s;
         }
         store_dw(p, dw);
+        if constexpr (DIRECT) {
 #pragma unroll
-        for (int m1 = 0; m1 < d1; ++m1)
+            for (int m1 = 0; m1 < d1; ++m1)
 #pragma unroll
-            for (int v = 0; v < V; ++v) dxv[o1 + m1][v] = fmaf(wv[p][v], t[m1][v], dxv[o1 + m1][v]);
+                for (int v = 0; v < V; ++v) dx_full[o1 + m1][v] = fmaf(wp[v], t[m1][v], dx_full[o1 + m1][v]);
+        } else {
+#pragma unroll
+            for (int m1 = 0; m1 < d1; ++m1)
+#pragma unroll
+                for (int v = 0; v < V; ++v) dxg[m1][v] = fmaf(wp[v], t[m1][v], dxg[m1][v]);
+            if constexpr (last_of_block) dx_sink(o1, d1, dxg);
+        }
         if constexpr (l2 > 0) {
             constexpr int d2 = 2 * l2 + 1, o2 = l2 * l2;
             static_for<d2>([&](auto m2c) {
@@ -306,12 +401,12 @@ __device__ __forceinline__ void bwd_edge(const float* As, const float (&xv)[K::D
                             static_for<d3>([&](auto m3c) {
                                 constexpr int m3 = EQC_CV(m3c);
                                 constexpr double c = RealCG<l1, l2, l3>::t.v[m1][m2][m3];
-                                if constexpr (c != 0.0) s = fmaf((float)c, gv[o3 + m3][v], s);
+                                if constexpr (c != 0.0) s = fmaf((float)c, gv[m3][v], s);
                             });
-                            g = fmaf(xv[o1 + m1][v], s, g);
+                            g = fmaf(xv[m1][v], s, g);
                         }
                     });
-                    gsum = fmaf(wv[p][v], g, gsum);
+                    gsum = fmaf(wp[v], g, gsum);
                 }
                 gyl[o2 + m2 - 1] += gsum;
             });
@@ -329,7 +424,7 @@ struct FwdParams {
     const int* ptr;    // recv_ptr
     const int* perm;   // recv_perm
     const int* other;  // senders
-    int N, C;
+    int N, C, E;
     unsigned* status;
 };
 
@@ -345,26 +440,139 @@ struct BwdParams {
     const int* ptr;    // DET: send_ptr   ATOMIC: recv_ptr
     const int* perm;   // DET: send_perm  ATOMIC: recv_perm
     const int* other;  // DET: receivers  ATOMIC: senders
-    int N, C, T;
+    int N, C, T, E;
     unsigned* status;
+};
+
+// ------------------------------------------------------ async row staging
+//
+// Each warp owns a ring of S stages in shared memory.  A stage holds one
+// edge's rows for the warp's channel tile: the weight row w[e, 0..P) and the
+// gathered row (x[s] in the forward and the atomic backward, gy[i] in the
+// deterministic backward), each component a run of TILE_C channels.  One
+// mbarrier per stage counts the bytes of the bulk copies (cp.async.bulk, no
+// multicast) that fill it; the warp waits on the stage's phase before reading
+// it, and refills it S edges later.  Every wait is bounded: after
+// kWaitLimit polls the kernel sets status bit 4 and stops processing.
+
+constexpr uint32_t kWaitLimit = 1u << 24;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Returns false if the phase did not complete within the poll limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_addr(bar);
+    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// One tensor-map box [rows][TILE_C] at (c0, 0, idx) of a [count][rows][C] tensor.
+__device__ __forceinline__ void tma_rows(void* dst, const CUtensorMap* map, int c0, int idx, uint64_t* bar,
+                                         uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(0), "r"(idx),
+        "r"(smem_addr(bar)), "l"(pol)
+        : "memory");
+}
+
+// Stage geometry: NP weight rows then NG gathered rows, TILE_C floats each.
+template <class K, int NG>
+struct Stage {
+    static constexpr int ROWS = K::NP + NG;
+    static constexpr int FLOATS = ROWS * K::TILE_C;   // per stage (a multiple of 64 floats)
+    static constexpr uint32_t BYTES = FLOATS * 4;
+};
+
+// Fill stage `st` with w[e, :, tile] and g[o, :, tile] (o >= 0): two tensor-map
+// copies issued by lane 0.  The caller has __syncwarp()ed after the stage's
+// previous readers; the proxy fence orders those reads before the async writes.
+template <class K, int NG>
+__device__ __forceinline__ void stage_fill(float* st, uint64_t* bar, const CUtensorMap* tw, const CUtensorMap* tg,
+                                           int e, int o, int c0, uint64_t pol_w, uint64_t pol_g, int lane) {
+    if (lane == 0) {
+        fence_proxy_async();
+        mbar_expect_tx(bar, Stage<K, NG>::BYTES);
+        tma_rows(st, tw, c0, e, bar, pol_w);
+        tma_rows(st + K::NP * K::TILE_C, tg, c0, o, bar, pol_g);
+    }
+}
+
+
+// Per-warp shared-memory layout (floats), every region 128-byte aligned:
+// [stages: S x FLOATS] [mbarriers: 16 B each] [A: CHUNK x NA_PAD] [gY: CHUNK x GS]
+template <class K, int NG, bool WITH_GY>
+struct WarpSmem {
+    static constexpr int S = K::STAGES;
+    static constexpr int up32(int f) { return (f + 31) & ~31; }
+    static constexpr int ST_F = S * Stage<K, NG>::FLOATS;
+    static constexpr int BAR_F = up32(4 * S);
+    static constexpr int A_F = up32(K::CHUNK * K::NA_PAD);
+    static constexpr int GY_F = WITH_GY ? up32(K::CHUNK * K::GS) : 0;
+    static constexpr int TOTAL_F = ST_F + BAR_F + A_F + GY_F;
+    static constexpr int BYTES = TOTAL_F * 4;
 };
 
 // ---------------------------------------------------------------- forward
 
 template <class K>
-__global__ void __launch_bounds__(K::WARPS * 32) eqconv_fwd_kernel(const FwdParams prm) {
+__global__ void __launch_bounds__(K::WARPS * 32)
+    eqconv_fwd_kernel(const FwdParams prm, const __grid_constant__ CUtensorMap tmap_w,
+                      const __grid_constant__ CUtensorMap tmap_x) {
     constexpr int V = K::VEC;
-    extern __shared__ float4 smem4[];
-    float* smem = reinterpret_cast<float*>(smem4);
+    constexpr int S = K::STAGES;
+    using L = WarpSmem<K, K::D_IN, false>;
+    constexpr int SF = Stage<K, K::D_IN>::FLOATS;
+    extern __shared__ __align__(128) float4 smem4[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int node = blockIdx.x * K::WARPS + warp;
     if (node >= prm.N) return;
-    float* As = smem + warp * (K::CHUNK * K::NA_PAD);
-    const int c0 = blockIdx.y * K::TILE_C + lane * V;
-    const bool active = c0 < prm.C;
-    const size_t C = (size_t)prm.C;
+    float* stages = reinterpret_cast<float*>(smem4) + warp * L::TOTAL_F;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + L::ST_F);
+    float* As = stages + L::ST_F + L::BAR_F;
+    const int tile = blockIdx.y;
+    const int C = prm.C;
+    const int c0 = tile * K::TILE_C;
+    const int ct_len = min(K::TILE_C, C - c0);
+    const int cl = lane * V;                 // lane's channel offset inside the tile
+    const bool active = cl < ct_len;
     const uint64_t pol_stream = policy_evict_first();
     const uint64_t pol_keep = policy_evict_last();
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&bars[2 * s], 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
 
     float acc[K::D_OUT][V];
 #pragma unroll
@@ -372,33 +580,13 @@ __global__ void __launch_bounds__(K::WARPS * 32) eqconv_fwd_kernel(const FwdPara
 #pragma unroll
         for (int v = 0; v < V; ++v) acc[d][v] = 0.f;
 
-    auto load_edge = [&](int e, int s, float (&xv)[K::D_IN][V], float (&wv)[K::NP][V]) {
-        if (active && s >= 0) {
-            const float* xs = prm.x + (size_t)s * K::D_IN * C + c0;
-#pragma unroll
-            for (int d = 0; d < K::D_IN; ++d) ld_keep<V>(xv[d], xs + d * C, pol_keep);
-        } else {
-#pragma unroll
-            for (int d = 0; d < K::D_IN; ++d)
-#pragma unroll
-                for (int v = 0; v < V; ++v) xv[d][v] = 0.f;
-        }
-        if (active) {
-            const float* we = prm.w + (size_t)e * K::NP * C + c0;
-#pragma unroll
-            for (int p = 0; p < K::NP; ++p) ld_stream<V>(wv[p], we + p * C, pol_stream);
-        } else {
-#pragma unroll
-            for (int p = 0; p < K::NP; ++p)
-#pragma unroll
-                for (int v = 0; v < V; ++v) wv[p][v] = 0.f;
-        }
-    };
-
+    uint32_t g = 0;        // edges staged so far by this warp (stage = g % S, phase = (g / S) & 1)
+    bool ok_all = true;
     const int kb = prm.ptr[node], ke = prm.ptr[node + 1];
-    for (int k0 = kb; k0 < ke; k0 += K::CHUNK) {
+    for (int k0 = kb; k0 < ke && ok_all; k0 += K::CHUNK) {
         const int n = min(K::CHUNK, ke - k0);
         int my_e = 0, my_s = -1;
+        float rx = 0.f, ry = 0.f, rz = 0.f;
         if (lane < n) {
             my_e = prm.perm[k0 + lane];
             const int s = prm.other[my_e];
@@ -407,42 +595,72 @@ __global__ void __launch_bounds__(K::WARPS * 32) eqconv_fwd_kernel(const FwdPara
             else
                 atomicOr(prm.status, 1u);
             const float* re = prm.r + (size_t)my_e * 3;
+            rx = re[0];
+            ry = re[1];
+            rz = re[2];
+        }
+        // start the first S edges' copies, then build A while they fly
+        const int pre = min(S, n);
+        for (int t = 0; t < pre; ++t) {
+            const int e = __shfl_sync(0xffffffffu, my_e, t), s = __shfl_sync(0xffffffffu, my_s, t);
+            const uint32_t gi = g + t;
+            stage_fill<K, K::D_IN>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_x, e, s < 0 ? 0 : s,
+                                   c0, pol_stream, pol_keep, lane);
+        }
+        if (lane < n) {
             float ux, uy, uz, il;
-            const bool ok = unit_dir(re[0], re[1], re[2], ux, uy, uz, il);
+            const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
             float Y[K::D_SH];
             sh_eval<K::LSH>(ok, ux, uy, uz, Y);
             compute_A<K>(Y, As + lane * K::NA_PAD);
         }
         __syncwarp();
-        if constexpr (K::FWD_PREFETCH) {
-            float xc[K::D_IN][V], wc[K::NP][V], xn[K::D_IN][V], wn[K::NP][V];
-            load_edge(__shfl_sync(0xffffffffu, my_e, 0), __shfl_sync(0xffffffffu, my_s, 0), xc, wc);
-            for (int t = 0; t < n; ++t) {
-                if (t + 1 < n)
-                    load_edge(__shfl_sync(0xffffffffu, my_e, t + 1), __shfl_sync(0xffffffffu, my_s, t + 1), xn, wn);
-                fwd_edge<K>(As + t * K::NA_PAD, xc, wc, acc);
-#pragma unroll
-                for (int d = 0; d < K::D_IN; ++d)
-#pragma unroll
-                    for (int v = 0; v < V; ++v) xc[d][v] = xn[d][v];
-#pragma unroll
-                for (int p = 0; p < K::NP; ++p)
-#pragma unroll
-                    for (int v = 0; v < V; ++v) wc[p][v] = wn[p][v];
+        for (int t = 0; t < n; ++t) {
+            const uint32_t gi = g + t;
+            float* st = stages + (gi % S) * SF;
+            if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
+                if (lane == 0) atomicOr(prm.status, 4u);
+                ok_all = false;
+                break;
             }
-        } else {
-            for (int t = 0; t < n; ++t) {
-                float xc[K::D_IN][V], wc[K::NP][V];
-                load_edge(__shfl_sync(0xffffffffu, my_e, t), __shfl_sync(0xffffffffu, my_s, t), xc, wc);
-                fwd_edge<K>(As + t * K::NA_PAD, xc, wc, acc);
+            const bool valid = __shfl_sync(0xffffffffu, my_s, t) >= 0;
+            float xv[K::D_IN][V], wv[K::NP][V];
+#pragma unroll
+            for (int p = 0; p < K::NP; ++p) {
+                if (active)
+                    lds_vec<V>(wv[p], st + p * K::TILE_C + cl);
+                else
+#pragma unroll
+                    for (int v = 0; v < V; ++v) wv[p][v] = 0.f;
+            }
+#pragma unroll
+            for (int d = 0; d < K::D_IN; ++d) {
+                if (active && valid)
+                    lds_vec<V>(xv[d], st + (K::NP + d) * K::TILE_C + cl);
+                else
+#pragma unroll
+                    for (int v = 0; v < V; ++v) xv[d][v] = 0.f;
+            }
+            fwd_edge<K>(As + t * K::NA_PAD, xv, wv, acc);
+            __syncwarp();
+            if (t + S < n) {
+                const int e = __shfl_sync(0xffffffffu, my_e, t + S), s = __shfl_sync(0xffffffffu, my_s, t + S);
+                stage_fill<K, K::D_IN>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_x, e, s < 0 ? 0 : s, c0, pol_stream,
+                                       pol_keep, lane);
             }
         }
+        g += n;
         __syncwarp();
     }
+    if (!ok_all) {
+        // drain: wait (bounded) for copies still in flight before the warp exits
+        for (int s = 0; s < S; ++s) mbar_wait(&bars[2 * s], 0), mbar_wait(&bars[2 * s], 1);
+        return;
+    }
     if (active) {
-        float* yi = prm.y + (size_t)node * K::D_OUT * C + c0;
+        float* yi = prm.y + (size_t)node * K::D_OUT * C + c0 + cl;
 #pragma unroll
-        for (int d = 0; d < K::D_OUT; ++d) st_plain<V>(yi + d * C, acc[d]);
+        for (int d = 0; d < K::D_OUT; ++d) st_stream<V>(yi + (size_t)d * C, acc[d]);
     }
 }
 
@@ -461,33 +679,48 @@ __device__ __forceinline__ void warp_sum(float (&v)[G]) {
 // !DET: node = receiver i, resident gy_i, dx scattered with atomic adds.
 // FUSED: the tile covers every channel (T == 1): dr is finished in-kernel.
 template <class K, bool DET, bool FUSED>
-__global__ void __launch_bounds__(K::WARPS * 32) eqconv_bwd_kernel(const BwdParams prm) {
+__global__ void __launch_bounds__(K::WARPS * 32)
+    eqconv_bwd_kernel(const BwdParams prm, const __grid_constant__ CUtensorMap tmap_w,
+                      const __grid_constant__ CUtensorMap tmap_g) {
     constexpr int V = K::VEC;
+    constexpr int S = K::STAGES;
     constexpr int GG = K::G > 0 ? K::G : 1;
-    extern __shared__ float4 smem4[];
-    float* smem = reinterpret_cast<float*>(smem4);
+    constexpr int DL = DET ? K::D_OUT : K::D_IN;     // rows gathered per edge
+    using L = WarpSmem<K, DL, true>;
+    constexpr int SF = Stage<K, DL>::FLOATS;
+    extern __shared__ __align__(128) float4 smem4[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int node = blockIdx.x * K::WARPS + warp;
     if (node >= prm.N) return;
-    float* As = smem + warp * (K::CHUNK * (K::NA_PAD + K::GS));
-    float* gYs = As + K::CHUNK * K::NA_PAD;
+    float* stages = reinterpret_cast<float*>(smem4) + warp * L::TOTAL_F;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + L::ST_F);
+    float* As = stages + L::ST_F + L::BAR_F;
+    float* gYs = As + L::A_F;
     const int tile = blockIdx.y;
-    const int c0 = tile * K::TILE_C + lane * V;
-    const bool active = c0 < prm.C;
-    const size_t C = (size_t)prm.C;
+    const int C = prm.C;
+    const int c0 = tile * K::TILE_C;
+    const int ct_len = min(K::TILE_C, C - c0);
+    const int cl = lane * V;
+    const bool active = cl < ct_len;
+    const size_t c_off = (size_t)c0 + cl;
     const uint64_t pol_stream = policy_evict_first();
     const uint64_t pol_keep = policy_evict_last();
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&bars[2 * s], 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
 
     // resident rows: x_j (DET) or gy_i (!DET)
     float xres[DET ? K::D_IN : 1][V];
     float gres[DET ? 1 : K::D_OUT][V];
     float dxacc[DET ? K::D_IN : 1][V];
     if constexpr (DET) {
-        const float* xj = prm.x + (size_t)node * K::D_IN * C + c0;
+        const float* xj = prm.x + (size_t)node * K::D_IN * C + c_off;
 #pragma unroll
         for (int d = 0; d < K::D_IN; ++d) {
             if (active)
-                ld_keep<V>(xres[d], xj + d * C, pol_keep);
+                ld_keep<V>(xres[d], xj + (size_t)d * C, pol_keep);
             else
 #pragma unroll
                 for (int v = 0; v < V; ++v) xres[d][v] = 0.f;
@@ -495,82 +728,21 @@ __global__ void __launch_bounds__(K::WARPS * 32) eqconv_bwd_kernel(const BwdPara
             for (int v = 0; v < V; ++v) dxacc[d][v] = 0.f;
         }
     } else {
-        const float* gi = prm.gy + (size_t)node * K::D_OUT * C + c0;
+        const float* gi = prm.gy + (size_t)node * K::D_OUT * C + c_off;
 #pragma unroll
         for (int d = 0; d < K::D_OUT; ++d) {
             if (active)
-                ld_keep<V>(gres[d], gi + d * C, pol_keep);
+                ld_keep<V>(gres[d], gi + (size_t)d * C, pol_keep);
             else
 #pragma unroll
                 for (int v = 0; v < V; ++v) gres[d][v] = 0.f;
         }
     }
 
-    // rows loaded per edge: gy_i and w_e (DET) or x_s and w_e (!DET)
-    constexpr int DL = DET ? K::D_OUT : K::D_IN;
-    auto load_edge = [&](int e, int o, float (&lv)[DL][V], float (&wv)[K::NP][V]) {
-        if (active && o >= 0) {
-            const float* src = DET ? prm.gy + (size_t)o * K::D_OUT * C + c0 : prm.x + (size_t)o * K::D_IN * C + c0;
-#pragma unroll
-            for (int d = 0; d < DL; ++d) ld_keep<V>(lv[d], src + d * C, pol_keep);
-        } else {
-#pragma unroll
-            for (int d = 0; d < DL; ++d)
-#pragma unroll
-                for (int v = 0; v < V; ++v) lv[d][v] = 0.f;
-        }
-        if (active) {
-            const float* we = prm.w + (size_t)e * K::NP * C + c0;
-#pragma unroll
-            for (int p = 0; p < K::NP; ++p) ld_stream<V>(wv[p], we + p * C, pol_stream);
-        } else {
-#pragma unroll
-            for (int p = 0; p < K::NP; ++p)
-#pragma unroll
-                for (int v = 0; v < V; ++v) wv[p][v] = 0.f;
-        }
-    };
-
-    auto do_edge = [&](int t, int e, int o, const float (&lv)[DL][V], const float (&wv)[K::NP][V]) {
-        float gyl[GG];
-#pragma unroll
-        for (int k = 0; k < GG; ++k) gyl[k] = 0.f;
-        float* dwe = prm.dw + (size_t)e * K::NP * C + c0;
-        auto store_dw = [&](int p, const float* dwv) {
-            if (active) st_stream<V>(dwe + p * C, dwv);
-        };
-        if constexpr (DET) {
-            bwd_edge<K>(As + t * K::NA_PAD, xres, lv, wv, dxacc, gyl, store_dw);
-        } else {
-            float dxe[K::D_IN][V];
-#pragma unroll
-            for (int d = 0; d < K::D_IN; ++d)
-#pragma unroll
-                for (int v = 0; v < V; ++v) dxe[d][v] = 0.f;
-            bwd_edge<K>(As + t * K::NA_PAD, lv, gres, wv, dxe, gyl, store_dw);
-            if (active && o >= 0) {
-                float* dxs = prm.dx + (size_t)o * K::D_IN * C + c0;
-#pragma unroll
-                for (int d = 0; d < K::D_IN; ++d) red_add<V>(dxs + d * C, dxe[d]);
-            }
-        }
-        if constexpr (K::G > 0) {
-            warp_sum<K::G>(gyl);
-            if (lane == 0) {
-                if constexpr (FUSED) {
-#pragma unroll
-                    for (int k = 0; k < K::G; ++k) gYs[t * K::GS + k] = gyl[k];
-                } else {
-                    float* gp = prm.gy_part + ((size_t)e * prm.T + tile) * K::G;
-#pragma unroll
-                    for (int k = 0; k < K::G; ++k) gp[k] = gyl[k];
-                }
-            }
-        }
-    };
-
+    uint32_t g = 0;
+    bool ok_all = true;
     const int kb = prm.ptr[node], ke = prm.ptr[node + 1];
-    for (int k0 = kb; k0 < ke; k0 += K::CHUNK) {
+    for (int k0 = kb; k0 < ke && ok_all; k0 += K::CHUNK) {
         const int n = min(K::CHUNK, ke - k0);
         int my_e = 0, my_o = -1;
         float rx = 0.f, ry = 0.f, rz = 0.f;
@@ -585,6 +757,15 @@ __global__ void __launch_bounds__(K::WARPS * 32) eqconv_bwd_kernel(const BwdPara
             rx = re[0];
             ry = re[1];
             rz = re[2];
+        }
+        const int pre = min(S, n);
+        for (int t = 0; t < pre; ++t) {
+            const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_o, t);
+            const uint32_t gi = g + t;
+            stage_fill<K, DL>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e, o < 0 ? 0 : o, c0,
+                              pol_stream, pol_keep, lane);
+        }
+        if (lane < n) {
             float ux, uy, uz, il;
             const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
             float Y[K::D_SH];
@@ -592,40 +773,63 @@ __global__ void __launch_bounds__(K::WARPS * 32) eqconv_bwd_kernel(const BwdPara
             compute_A<K>(Y, As + lane * K::NA_PAD);
         }
         __syncwarp();
-        if constexpr (K::BWD_PREFETCH) {
-            float lc[DL][V], wc[K::NP][V], ln[DL][V], wn[K::NP][V];
-            int e_c = __shfl_sync(0xffffffffu, my_e, 0), o_c = __shfl_sync(0xffffffffu, my_o, 0);
-            load_edge(e_c, o_c, lc, wc);
-            for (int t = 0; t < n; ++t) {
-                int e_n = 0, o_n = -1;
-                if (t + 1 < n) {
-                    e_n = __shfl_sync(0xffffffffu, my_e, t + 1);
-                    o_n = __shfl_sync(0xffffffffu, my_o, t + 1);
-                    load_edge(e_n, o_n, ln, wn);
-                }
-                do_edge(t, e_c, o_c, lc, wc);
-#pragma unroll
-                for (int d = 0; d < DL; ++d)
-#pragma unroll
-                    for (int v = 0; v < V; ++v) lc[d][v] = ln[d][v];
-#pragma unroll
-                for (int p = 0; p < K::NP; ++p)
-#pragma unroll
-                    for (int v = 0; v < V; ++v) wc[p][v] = wn[p][v];
-                e_c = e_n;
-                o_c = o_n;
+        for (int t = 0; t < n; ++t) {
+            const uint32_t gi = g + t;
+            float* st = stages + (gi % S) * SF;
+            if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
+                if (lane == 0) atomicOr(prm.status, 4u);
+                ok_all = false;
+                break;
             }
-        } else {
-            for (int t = 0; t < n; ++t) {
-                float lc[DL][V], wc[K::NP][V];
-                const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_o, t);
-                load_edge(e, o, lc, wc);
-                do_edge(t, e, o, lc, wc);
+            const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_o, t);
+            const SmemRows<V> Wr{st + cl, K::TILE_C, active};
+            const SmemRows<V> Lr{st + K::NP * K::TILE_C + cl, K::TILE_C, active && o >= 0};
+            float gyl[GG];
+#pragma unroll
+            for (int k = 0; k < GG; ++k) gyl[k] = 0.f;
+            float* dwe = prm.dw + (size_t)e * K::NP * C + c_off;
+            auto store_dw = [&](int p, const float* dwv) {
+                if (active) st_stream<V>(dwe + (size_t)p * C, dwv);
+            };
+            if constexpr (DET) {
+                auto no_sink = [](int, int, const float (&)[1][V]) {};
+                bwd_edge<K, true>(As + t * K::NA_PAD, RegRows<V, K::D_IN>{xres}, Lr, Wr, dxacc, no_sink, gyl,
+                                  store_dw);
+            } else {
+                float* dxs = prm.dx + (size_t)(o < 0 ? 0 : o) * K::D_IN * C + c_off;
+                const bool add = active && o >= 0;
+                auto sink = [&](int o1, int d1, const float (&blk)[2 * kMaxL + 1][V]) {
+                    if (add)
+#pragma unroll
+                        for (int m = 0; m < d1; ++m) red_add<V>(dxs + (size_t)(o1 + m) * C, blk[m]);
+                };
+                bwd_edge<K, false>(As + t * K::NA_PAD, Lr, RegRows<V, K::D_OUT>{gres}, Wr, dxacc, sink, gyl,
+                                   store_dw);
+            }
+            if constexpr (K::G > 0) {
+                warp_sum<K::G>(gyl);
+                if (lane == 0) {
+                    if constexpr (FUSED) {
+#pragma unroll
+                        for (int k = 0; k < K::G; ++k) gYs[t * K::GS + k] = gyl[k];
+                    } else {
+                        float* gp = prm.gy_part + ((size_t)e * prm.T + tile) * K::G;
+#pragma unroll
+                        for (int k = 0; k < K::G; ++k) gp[k] = gyl[k];
+                    }
+                }
+            }
+            __syncwarp();
+            if (t + S < n) {
+                const int e2 = __shfl_sync(0xffffffffu, my_e, t + S), o2 = __shfl_sync(0xffffffffu, my_o, t + S);
+                stage_fill<K, DL>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e2, o2 < 0 ? 0 : o2, c0, pol_stream,
+                                  pol_keep, lane);
             }
         }
+        g += n;
         __syncwarp();
         if constexpr (FUSED) {
-            if (lane < n) {
+            if (ok_all && lane < n) {
                 float ux, uy, uz, il;
                 const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
                 float d0 = 0.f, d1 = 0.f, d2 = 0.f;
@@ -638,11 +842,15 @@ __global__ void __launch_bounds__(K::WARPS * 32) eqconv_bwd_kernel(const BwdPara
             __syncwarp();
         }
     }
+    if (!ok_all) {
+        for (int s = 0; s < S; ++s) mbar_wait(&bars[2 * s], 0), mbar_wait(&bars[2 * s], 1);
+        return;
+    }
     if constexpr (DET) {
         if (active) {
-            float* dxj = prm.dx + (size_t)node * K::D_IN * C + c0;
+            float* dxj = prm.dx + (size_t)node * K::D_IN * C + c_off;
 #pragma unroll
-            for (int d = 0; d < K::D_IN; ++d) st_plain<V>(dxj + d * C, dxacc[d]);
+            for (int d = 0; d < K::D_IN; ++d) st_stream<V>(dxj + (size_t)d * C, dxacc[d]);
         }
     }
 }

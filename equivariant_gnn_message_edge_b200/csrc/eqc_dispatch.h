@@ -1,9 +1,17 @@
 // Dispatch table of kernel instances (host side, no device code).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstdint>
+
 namespace eqc {
+
+// Tensor map of a row-major fp32 tensor [count][rows][C] read in boxes of
+// [rows][tile_c] (one box per node or edge and channel tile).  False if the
+// driver entry point is unavailable or rejects the layout.
+bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t count, int rows, int C, int tile_c);
 
 struct FwdParams;
 struct BwdParams;

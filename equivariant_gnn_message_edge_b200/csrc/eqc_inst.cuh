@@ -8,7 +8,10 @@
 
 namespace eqc {
 
-#define EQC_PAIR(LOUT) {Launch<Cfg<EQC_LIN, EQC_LSH, LOUT, 2>>::make(), Launch<Cfg<EQC_LIN, EQC_LSH, LOUT, 4>>::make()}
+#ifndef EQC_VEC_SMALL
+#define EQC_VEC_SMALL 2
+#endif
+#define EQC_PAIR(LOUT) {Launch<Cfg<EQC_LIN, EQC_LSH, LOUT, EQC_VEC_SMALL>>::make(), Launch<Cfg<EQC_LIN, EQC_LSH, LOUT, 4>>::make()}
 #define EQC_NAME2(a, b) instances_l##a##_s##b
 #define EQC_NAME(a, b) EQC_NAME2(a, b)
 

@@ -30,10 +30,18 @@ struct Launch {
     static cudaError_t fwd(const FwdParams& prm, int tiles, cudaStream_t st) {
         auto kern = eqconv_fwd_kernel<K>;
         static bool done[64] = {};
-        cudaError_t err = ensure_smem(kern, K::FWD_SMEM, done);
+        constexpr int smem = K::WARPS * WarpSmem<K, K::D_IN, false>::BYTES;
+        cudaError_t err = ensure_smem(kern, smem, done);
         if (err != cudaSuccess) return err;
+        // with no edges the weight map is never read: give it a valid stand-in
+        CUtensorMap tw, tx;
+        if (!encode_rows_map(&tw, prm.E > 0 ? (const void*)prm.w : (const void*)prm.x,
+                             prm.E > 0 ? (uint64_t)prm.E : (uint64_t)prm.N, prm.E > 0 ? K::NP : K::D_IN, prm.C,
+                             K::TILE_C) ||
+            !encode_rows_map(&tx, prm.x, (uint64_t)prm.N, K::D_IN, prm.C, K::TILE_C))
+            return cudaErrorInvalidValue;
         dim3 grid((prm.N + K::WARPS - 1) / K::WARPS, tiles);
-        kern<<<grid, K::WARPS * 32, K::FWD_SMEM, st>>>(prm);
+        kern<<<grid, K::WARPS * 32, smem, st>>>(prm, tw, tx);
         count_launch();
         return cudaGetLastError();
     }
@@ -41,10 +49,16 @@ struct Launch {
     static cudaError_t bwd_one(const BwdParams& prm, cudaStream_t st) {
         auto kern = eqconv_bwd_kernel<K, DET, FUSED>;
         static bool done[64] = {};
-        cudaError_t err = ensure_smem(kern, K::BWD_SMEM, done);
+        constexpr int smem = K::WARPS * WarpSmem<K, DET ? K::D_OUT : K::D_IN, true>::BYTES;
+        cudaError_t err = ensure_smem(kern, smem, done);
         if (err != cudaSuccess) return err;
+        CUtensorMap tw, tg;
+        const float* g = DET ? prm.gy : prm.x;
+        if (!encode_rows_map(&tw, prm.w, (uint64_t)prm.E, K::NP, prm.C, K::TILE_C) ||
+            !encode_rows_map(&tg, g, (uint64_t)prm.N, DET ? K::D_OUT : K::D_IN, prm.C, K::TILE_C))
+            return cudaErrorInvalidValue;
         dim3 grid((prm.N + K::WARPS - 1) / K::WARPS, prm.T);
-        kern<<<grid, K::WARPS * 32, K::BWD_SMEM, st>>>(prm);
+        kern<<<grid, K::WARPS * 32, smem, st>>>(prm, tw, tg);
         count_launch();
         return cudaGetLastError();
     }

@@ -97,8 +97,11 @@ EQCONV_API int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int
                        const char* irreps_out, int C);
 
 /* Channel vector width of the forward / backward kernels (2 or 4 channels per
- * lane, i.e. channel tiles of 64 or 128).  The default is 4 when C >= 128,
- * else 2.  A tuning knob; results agree within rounding across widths. */
+ * lane, i.e. channel tiles of 64 or 128 channels).  Defaults (measured best on
+ * B200 at C = 128): 2 for the forward and the atomic backward, 4 for the
+ * deterministic backward when C >= 128.  bwd_vec sets both backward modes.  A
+ * tuning knob; results agree within rounding across widths (deterministic
+ * mode stays bitwise reproducible for a fixed width). */
 EQCONV_API int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec);
 
 /* Sizes of the plan; paths_l1l2l3 (3*P ints, may be NULL) receives the paths. */
@@ -154,8 +157,9 @@ EQCONV_API int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const
                    const float* r, const float* w, float* y, unsigned flags,
                    eqconv_stream_t stream);
 
-/* Device workspace bytes needed by eqconv_backward (0 when C fits one
- * channel tile: the dr reduction is then done in-kernel). */
+/* Device workspace bytes needed by eqconv_backward in either mode (0 when C
+ * fits one channel tile of both modes: the dr reduction is then done
+ * in-kernel; otherwise per-tile partials of dr's harmonic gradient). */
 EQCONV_API size_t eqconv_backward_workspace_bytes(eqconv_plan_t plan, int E);
 
 /* Backward given gy: writes dx [N][D_in][C], dw [E][P][C], dr [E][3].
