@@ -205,38 +205,46 @@ def run_native(args, rank, world, local_rank):
     bc = byte_counts(N, E, C, D_in, D_out, P)
 
     stream = torch.cuda.Stream(device=dev)
-    with torch.cuda.stream(stream):
-        s_d = inp.senders.to(dev, non_blocking=True)
-        r_d = inp.receivers.to(dev, non_blocking=True)
-        x_d = inp.x.to(dev, non_blocking=True)
-        rv_d = inp.r.to(dev, non_blocking=True)
-        w_d = inp.w.to(dev, non_blocking=True)
-        gy_d = inp.gy.to(dev, non_blocking=True)
-        g = conv.graph(s_d, r_d, N, stream=stream)
-        y_d = torch.empty((N, D_out, C), dtype=torch.float32, device=dev)
-        dx_d = torch.empty_like(x_d)
-        dw_d = torch.empty_like(w_d)
-        dr_d = torch.empty_like(rv_d)
-        gws_n = B.eqconv_graph_workspace_bytes(N, E)
-        gws = torch.empty(max(gws_n, 1), dtype=torch.uint8, device=dev)
-        bws_n = B.eqconv_backward_workspace_bytes(conv.plan, E)
-        bws = torch.empty(max(bws_n, 1), dtype=torch.uint8, device=dev)
-    stream.synchronize()
+
+    class DeviceSet:
+        """Device copies of one step's inputs, its edge layout and outputs."""
+
+        def __init__(self):
+            with torch.cuda.stream(stream):
+                self.s = inp.senders.to(dev, non_blocking=True)
+                self.r = inp.receivers.to(dev, non_blocking=True)
+                self.x = inp.x.to(dev, non_blocking=True)
+                self.rv = inp.r.to(dev, non_blocking=True)
+                self.w = inp.w.to(dev, non_blocking=True)
+                self.gy = inp.gy.to(dev, non_blocking=True)
+                self.g = conv.graph(self.s, self.r, N, stream=stream)
+                self.y = torch.empty((N, D_out, C), dtype=torch.float32, device=dev)
+                self.dx = torch.empty_like(self.x)
+                self.dw = torch.empty_like(self.w)
+                self.dr = torch.empty_like(self.rv)
+            stream.synchronize()
+
+    ds0 = DeviceSet()
+    gws_n = B.eqconv_graph_workspace_bytes(N, E)
+    gws = torch.empty(max(gws_n, 1), dtype=torch.uint8, device=dev)
+    bws_n = B.eqconv_backward_workspace_bytes(conv.plan, E)
+    bws = torch.empty(max(bws_n, 1), dtype=torch.uint8, device=dev)
     sh = stream.cuda_stream
 
-    def step(ev=None):
+    def step(ev=None, ds=ds0, st=stream):
+        h = st.cuda_stream
         if ev is not None:
-            ev[0].record(stream)
-        B.eqconv_graph_build(conv.plan, g.c, gws, gws_n, sh)
+            ev[0].record(st)
+        B.eqconv_graph_build(conv.plan, ds.g.c, gws, gws_n, h)
         if ev is not None:
-            ev[1].record(stream)
-        B.eqconv_forward(conv.plan, g.c, x_d, rv_d, w_d, y_d, 0, sh)
+            ev[1].record(st)
+        B.eqconv_forward(conv.plan, ds.g.c, ds.x, ds.rv, ds.w, ds.y, 0, h)
         if ev is not None:
-            ev[2].record(stream)
-        B.eqconv_backward(conv.plan, g.c, x_d, rv_d, w_d, gy_d, dx_d, dw_d, dr_d, bws, bws_n,
-                          B.EQCONV_DETERMINISTIC, sh)
+            ev[2].record(st)
+        B.eqconv_backward(conv.plan, ds.g.c, ds.x, ds.rv, ds.w, ds.gy, ds.dx, ds.dw, ds.dr, bws, bws_n,
+                          B.EQCONV_DETERMINISTIC, h)
         if ev is not None:
-            ev[3].record(stream)
+            ev[3].record(st)
 
     def barrier():
         if world > 1:
@@ -280,44 +288,67 @@ def run_native(args, rank, world, local_rank):
     for _ in range(max(2, args.steps // 2)):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        B.eqconv_backward(conv.plan, g.c, x_d, rv_d, w_d, gy_d, dx_d, dw_d, dr_d, bws, bws_n, 0, sh)
+        B.eqconv_backward(conv.plan, ds0.g.c, ds0.x, ds0.rv, ds0.w, ds0.gy, ds0.dx, ds0.dw, ds0.dr, bws, bws_n,
+                          0, sh)
         b.record(stream)
         nd_ms.append((a, b))
     stream.synchronize()
     nd_ms = [a.elapsed_time(b) for a, b in nd_ms[1:]]
 
-    # end-to-end through the public API with host buffers (pinned), copies timed
+    # End to end through the public API with host buffers (pinned), copies
+    # timed: every step uploads its inputs and downloads its results.  Steps
+    # are pipelined over two device sets and three streams, so step k's
+    # upload, step k-1's compute and step k-2's download overlap.
     e2e = None
     if not args.no_e2e:
-        y_h = torch.empty((N, D_out, C), dtype=torch.float32, pin_memory=True)
-        dx_h = torch.empty((N, D_in, C), dtype=torch.float32, pin_memory=True)
-        dw_h = torch.empty((E, P, C), dtype=torch.float32, pin_memory=True)
-        dr_h = torch.empty((E, 3), dtype=torch.float32, pin_memory=True)
+        sets = [ds0, DeviceSet()]
+        outs_h = [(torch.empty((N, D_out, C), dtype=torch.float32, pin_memory=True),
+                   torch.empty((N, D_in, C), dtype=torch.float32, pin_memory=True),
+                   torch.empty((E, P, C), dtype=torch.float32, pin_memory=True),
+                   torch.empty((E, 3), dtype=torch.float32, pin_memory=True)) for _ in range(2)]
+        up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        free = [None, None]     # event: the set's previous download has finished
 
-        def e2e_step():
-            with torch.cuda.stream(stream):
-                for dst, src in ((s_d, inp.senders), (r_d, inp.receivers), (x_d, inp.x), (rv_d, inp.r),
-                                 (w_d, inp.w), (gy_d, inp.gy)):
+        def e2e_step(k):
+            ds, oh = sets[k % 2], outs_h[k % 2]
+            if free[k % 2] is not None:
+                up.wait_event(free[k % 2])
+            with torch.cuda.stream(up):
+                for dst, src in ((ds.s, inp.senders), (ds.r, inp.receivers), (ds.x, inp.x), (ds.rv, inp.r),
+                                 (ds.w, inp.w), (ds.gy, inp.gy)):
                     dst.copy_(src, non_blocking=True)
-                step()
-                for dst, src in ((y_h, y_d), (dx_h, dx_d), (dw_h, dw_d), (dr_h, dr_d)):
+                loaded = torch.cuda.Event()
+                loaded.record(up)
+            stream.wait_event(loaded)
+            step(ds=ds, st=stream)
+            done = torch.cuda.Event()
+            done.record(stream)
+            down.wait_event(done)
+            with torch.cuda.stream(down):
+                for dst, src in zip(oh, (ds.y, ds.dx, ds.dw, ds.dr)):
                     dst.copy_(src, non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(down)
+            free[k % 2] = ev
 
-        e2e_steps = max(2, min(args.steps, 5))
-        for _ in range(2):
-            e2e_step()
-        stream.synchronize()
+        e2e_steps = max(3, min(args.steps, 6))
+        for k in range(2):
+            e2e_step(k)
+        torch.cuda.synchronize(dev)
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        b.record(stream)
-        stream.synchronize()
+        a.record(up)
+        for k in range(e2e_steps):
+            e2e_step(k)
+        down.wait_event(free[(e2e_steps - 1) % 2])
+        b.record(down)
+        torch.cuda.synchronize(dev)
         e_ms = reduce_max(a.elapsed_time(b), world, dev)
         e2e = {"value": round(aggregate_gbs(bc["kernels"], e2e_steps, world, e_ms), 2), "unit": UNIT,
                "h2d_bytes_per_step": bc["h2d"], "d2h_bytes_per_step": bc["d2h"],
-               "ms_per_step": e_ms / e2e_steps}
+               "ms_per_step": round(e_ms / e2e_steps, 3),
+               "pipeline": "2 device sets; upload / compute / download streams overlap across steps"}
+        del sets[1]
 
     peak, peak_kind = measured_peak()
     ms_step = t_max / args.steps
@@ -368,11 +399,19 @@ def run_native(args, rank, world, local_rank):
 
 
 def load_traffic():
-    """DRAM bytes per launch from the committed ncu summary (None if absent)."""
+    """DRAM bytes per launch from the committed ncu summary; empty (so the
+    roofline's traffic is null) when absent or when the kernel sources have
+    changed since the counters were taken."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            return json.load(f)
+            d = json.load(f)
+        h = hashlib.sha256()
+        for rel in d["kernel_sources"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        return d if h.hexdigest() == d["kernel_sources_sha256"] else {}
     except Exception:
         return {}
 
