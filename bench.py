@@ -199,6 +199,8 @@ def run_native(args, rank, world, local_rank):
     conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C)
     if args.vec:
         conv.set_vec(*[int(v) for v in args.vec.split(",")])
+    if args.gather_budget_mib is not None:
+        conv.set_gather_budget(int(args.gather_budget_mib * (1 << 20)))
     P, D_in, D_out = conv.P, conv.D_in, conv.D_out
     inp = Inputs(args.workload, P, D_in, D_out, pinned=True)
     N, E, C = inp.N, inp.E, inp.C
@@ -515,6 +517,8 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="lmax2", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--vec", default=None, help="fwd,bwd channel vector widths (2 or 4)")
+    ap.add_argument("--gather-budget-mib", type=float, default=None,
+                    help="L2 budget of one gather band in MiB (0: no banding)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -31,7 +31,7 @@ ABI_FUNCTIONS = (
     "eqconv_graph_workspace_bytes", "eqconv_graph_build", "eqconv_forward",
     "eqconv_backward_workspace_bytes", "eqconv_backward", "eqconv_spherical_harmonics",
     "eqconv_get_device_error", "eqconv_plan_destroy", "eqconv_status_string", "eqconv_launch_count",
-    "eqconv_last_error", "eqconv_graph_build_noalloc",
+    "eqconv_last_error", "eqconv_graph_build_noalloc", "eqconv_plan_set_gather_budget",
 )
 
 
@@ -61,6 +61,7 @@ _pg = ctypes.POINTER(eqconv_graph_t)
 _SIGS = {
     "eqconv_plan_create": (_ci, [ctypes.POINTER(_vp), ctypes.c_char_p, _ci, ctypes.c_char_p, _ci]),
     "eqconv_plan_set_vec": (_ci, [_vp, _ci, _ci]),
+    "eqconv_plan_set_gather_budget": (_ci, [_vp, _sz]),
     "eqconv_plan_info": (_ci, [_vp, _pi, _pi, _pi, _pi, _pi]),
     "eqconv_enumerate_paths": (_ci, [ctypes.c_char_p, _ci, ctypes.c_char_p, _pi, _pi, _ci]),
     "eqconv_cg_table": (_ci, [_ci, _ci, _ci, _pd, _ci]),
@@ -160,6 +161,10 @@ def eqconv_plan_create(irreps_in: str, L_sh: int, irreps_out: str, C: int) -> in
 
 def eqconv_plan_set_vec(plan: int, fwd_vec: int, bwd_vec: int) -> None:
     _check(lib().eqconv_plan_set_vec(plan, int(fwd_vec), int(bwd_vec)), "eqconv_plan_set_vec")
+
+
+def eqconv_plan_set_gather_budget(plan: int, nbytes: int) -> None:
+    _check(lib().eqconv_plan_set_gather_budget(plan, int(nbytes)), "eqconv_plan_set_gather_budget")
 
 
 def eqconv_plan_info(plan: int) -> dict:

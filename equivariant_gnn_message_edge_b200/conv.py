@@ -59,6 +59,10 @@ class EqConv:
     def set_vec(self, fwd_vec: int, bwd_vec: int):
         B.eqconv_plan_set_vec(self.plan, fwd_vec, bwd_vec)
 
+    def set_gather_budget(self, nbytes: int):
+        """L2 budget of one gather band (0: no banding); see include/eqconv.h."""
+        B.eqconv_plan_set_gather_budget(self.plan, nbytes)
+
     def graph(self, senders: torch.Tensor, receivers: torch.Tensor, N: int, stream=None) -> Graph:
         return Graph(self.plan, senders, receivers, N, stream)
 

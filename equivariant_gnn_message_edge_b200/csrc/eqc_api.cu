@@ -113,6 +113,8 @@ __global__ void k_zero_f4(float4* p, int64_t n4) {
 struct eqconv_plan_s {
     int lin, lsh, lout, C;
     int fwd_vec, det_vec, atomic_vec;
+    size_t gather_budget;   // bytes of gathered rows one band may touch (0: one band)
+    bool budget_set;        // false: per-mode defaults (bands for the atomic backward only)
     int P, D_in, D_sh, D_out;
     int paths[eqc::kMaxPaths][3];
     int device;
@@ -168,6 +170,28 @@ int default_atomic_vec(int) { return 2; }
 
 int tiles_for(int C, int tile_c) { return (C + tile_c - 1) / tile_c; }
 
+// L2 budget of one gather band.  Rows gathered by every SM stay in L2 on B200
+// while their set is about 40 MB (151 MB of x at lmax 2, C = 128 missed on
+// about half the gathers).  Measured on B200 (lmax 2, C = 128): bands cut the
+// DRAM bytes of every pass, but only the atomic backward gets faster (its dx
+// atomics stay in L2); the forward breaks even and the deterministic backward
+// slows down (each band gives a warp few edges to pipeline and dx is re-read),
+// so by default only the atomic backward is banded.
+constexpr size_t kDefaultGatherBudget = size_t(40) << 20;
+
+// Number of bands so that one band's gathered slice (rows of D components x
+// the channel tile) fits the budget.
+int bands_for(eqconv_plan_t plan, int N, int D, int tile_c, bool atomic_bwd) {
+    const size_t budget = plan->budget_set ? plan->gather_budget : (atomic_bwd ? kDefaultGatherBudget : 0);
+    if (budget == 0 || N <= 1) return 1;
+    const size_t slice = (size_t)N * (size_t)D * (size_t)(tile_c < plan->C ? tile_c : plan->C) * sizeof(float);
+    size_t b = (slice + budget - 1) / budget;
+    if (b < 1) b = 1;
+    if (b > 64) b = 64;
+    if (b > (size_t)N) b = (size_t)N;
+    return (int)b;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_device(eqconv_plan_t plan) {
@@ -219,6 +243,8 @@ int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh, cons
         p->paths[i][1] = PL.l2[i];
         p->paths[i][2] = PL.l3[i];
     }
+    p->gather_budget = 0;
+    p->budget_set = false;
     p->fwd_vec = default_fwd_vec(C);
     p->det_vec = default_det_vec(C);
     p->atomic_vec = default_atomic_vec(C);
@@ -252,6 +278,13 @@ int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec) {
     plan->det_vec = plan->atomic_vec = bwd_vec;
     plan->fwd_ks = f;
     plan->det_ks = plan->atomic_ks = b;
+    return EQCONV_OK;
+}
+
+int eqconv_plan_set_gather_budget(eqconv_plan_t plan, size_t bytes) {
+    if (!plan) return EQCONV_ERR_INVALID_ARG;
+    plan->gather_budget = bytes;
+    plan->budget_set = true;
     return EQCONV_OK;
 }
 
@@ -348,9 +381,11 @@ int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, 
     if (g->N == 0) return EQCONV_OK;
     if (!x || !y || (g->E > 0 && (!r || !w))) return EQCONV_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(y) || !aligned16(w)) return EQCONV_ERR_INVALID_ARG;
-    eqc::FwdParams prm{x, r, w, y, g->recv_ptr, g->recv_perm, g->senders, g->N, plan->C, g->E, plan->d_status};
+    eqc::FwdParams prm{x, r, w, y, g->recv_ptr, g->recv_perm, g->senders, g->N, plan->C, g->E, 0, g->N, 0,
+                       plan->d_status};
     const int T = tiles_for(plan->C, plan->fwd_ks->tile_c);
-    return cuda_status(plan->fwd_ks->fwd(prm, T, (cudaStream_t)stream), "forward");
+    const int bands = bands_for(plan, g->N, plan->D_in, plan->fwd_ks->tile_c, false);
+    return cuda_status(plan->fwd_ks->fwd(prm, T, bands, (cudaStream_t)stream), "forward");
 }
 
 static size_t bwd_ws_bytes(eqconv_plan_t plan, const eqc::KernelSet* ks, int E) {
@@ -419,7 +454,8 @@ int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
     prm.T = T;
     prm.E = g->E;
     prm.status = plan->d_status;
-    cudaError_t err = ks->bwd(prm, det, fused, st);
+    const int bands = bands_for(plan, g->N, det ? plan->D_out : plan->D_in, ks->tile_c, !det);
+    cudaError_t err = ks->bwd(prm, det, fused, bands, st);
     if (err != cudaSuccess) return cuda_status(err, det ? "backward (deterministic)" : "backward (atomic)");
     if (!fused) err = eqc::launch_dr_epilogue(plan->lsh, prm.gy_part, T, r, dr, g->E, st);
     return cuda_status(err, "dr epilogue");

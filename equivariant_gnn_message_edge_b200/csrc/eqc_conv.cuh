@@ -300,7 +300,7 @@ template <int V>
 struct SmemRows {
     const float* base;  // row 0 of this lane's channels
     int stride;         // floats between rows
-    bool on;            // false: rows read as zero (inactive lane or invalid edge)
+    bool on;            // false: rows read as zero (inactive lane)
     __device__ __forceinline__ void get(int d, float* out) const {
         if (on) {
             lds_vec<V>(out, base + d * stride);
@@ -425,6 +425,8 @@ struct FwdParams {
     const int* perm;   // recv_perm
     const int* other;  // senders
     int N, C, E;
+    int band_lo, band_hi;  // only edges whose sender is in [band_lo, band_hi)
+    int accumulate;        // 0: y = sum over the band; 1: y += sum over the band
     unsigned* status;
 };
 
@@ -441,6 +443,8 @@ struct BwdParams {
     const int* perm;   // DET: send_perm  ATOMIC: recv_perm
     const int* other;  // DET: receivers  ATOMIC: senders
     int N, C, T, E;
+    int band_lo, band_hi;  // only edges whose `other` node is in [band_lo, band_hi)
+    int accumulate;        // DET: 0: dx = band sum; 1: dx += band sum
     unsigned* status;
 };
 
@@ -543,6 +547,54 @@ struct WarpSmem {
     static constexpr int BYTES = TOTAL_F * 4;
 };
 
+// Collects the next window of up to 32 edges of a node's list whose gathered
+// node `other[e]` lies in [lo, hi), scanning 32 list positions at a time from
+// position k (advanced past the positions consumed) and keeping list order.
+// Out-of-range nodes set status bit 1 and are dropped.  Lanes < n receive
+// (e, o, r_e); returns n (0 only when the list is exhausted).
+__device__ __forceinline__ int gather_window(const int* perm, const int* other, const float* r, int N, int lo,
+                                             int hi, int& k, int ke, unsigned* status, int lane, int& my_e,
+                                             int& my_o, float& rx, float& ry, float& rz) {
+    int n = 0;
+    my_e = 0;
+    my_o = 0;
+    while (k < ke) {
+        const int n_all = min(32, ke - k);
+        int e_l = 0, o_l = 0;
+        bool in_band = false;
+        if (lane < n_all) {
+            e_l = perm[k + lane];
+            o_l = other[e_l];
+            if ((unsigned)o_l >= (unsigned)N)
+                atomicOr(status, 1u);
+            else
+                in_band = o_l >= lo && o_l < hi;
+        }
+        const unsigned mask = __ballot_sync(0xffffffffu, in_band);
+        const int cnt = __popc(mask);
+        if (n + cnt > 32) break;                      // the block goes to the next window
+        const int slot = lane - n;
+        const bool mine = slot >= 0 && slot < cnt;
+        const int src = mine ? (int)__fns(mask, 0u, slot + 1) : 0;
+        const int e2 = __shfl_sync(0xffffffffu, e_l, src), o2 = __shfl_sync(0xffffffffu, o_l, src);
+        if (mine) {
+            my_e = e2;
+            my_o = o2;
+        }
+        n += cnt;
+        k += n_all;
+        if (n == 32) break;
+    }
+    rx = ry = rz = 0.f;
+    if (lane < n) {
+        const float* re = r + (size_t)my_e * 3;
+        rx = re[0];
+        ry = re[1];
+        rz = re[2];
+    }
+    return n;
+}
+
 // ---------------------------------------------------------------- forward
 
 template <class K>
@@ -582,85 +634,89 @@ __global__ void __launch_bounds__(K::WARPS * 32)
 
     uint32_t g = 0;        // edges staged so far by this warp (stage = g % S, phase = (g / S) & 1)
     bool ok_all = true;
-    const int kb = prm.ptr[node], ke = prm.ptr[node + 1];
-    for (int k0 = kb; k0 < ke && ok_all; k0 += K::CHUNK) {
-        const int n = min(K::CHUNK, ke - k0);
-        int my_e = 0, my_s = -1;
-        float rx = 0.f, ry = 0.f, rz = 0.f;
-        if (lane < n) {
-            my_e = prm.perm[k0 + lane];
-            const int s = prm.other[my_e];
-            if ((unsigned)s < (unsigned)prm.N)
-                my_s = s;
-            else
-                atomicOr(prm.status, 1u);
-            const float* re = prm.r + (size_t)my_e * 3;
-            rx = re[0];
-            ry = re[1];
-            rz = re[2];
-        }
-        // start the first S edges' copies, then build A while they fly
+    int k = prm.ptr[node];
+    const int ke = prm.ptr[node + 1];
+    while (k < ke && ok_all) {
+        int my_e, my_s;
+        float rx, ry, rz;
+        const int n = gather_window(prm.perm, prm.other, prm.r, prm.N, prm.band_lo, prm.band_hi, k, ke, prm.status,
+                                    lane, my_e, my_s, rx, ry, rz);
+        if (n == 0) continue;
+        // the copy pipeline runs S edges ahead across the whole window
         const int pre = min(S, n);
         for (int t = 0; t < pre; ++t) {
             const int e = __shfl_sync(0xffffffffu, my_e, t), s = __shfl_sync(0xffffffffu, my_s, t);
             const uint32_t gi = g + t;
-            stage_fill<K, K::D_IN>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_x, e, s < 0 ? 0 : s,
-                                   c0, pol_stream, pol_keep, lane);
+            stage_fill<K, K::D_IN>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_x, e, s, c0,
+                                   pol_stream, pol_keep, lane);
         }
-        if (lane < n) {
-            float ux, uy, uz, il;
-            const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
-            float Y[K::D_SH];
-            sh_eval<K::LSH>(ok, ux, uy, uz, Y);
-            compute_A<K>(Y, As + lane * K::NA_PAD);
-        }
-        __syncwarp();
-        for (int t = 0; t < n; ++t) {
-            const uint32_t gi = g + t;
-            float* st = stages + (gi % S) * SF;
-            if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
-                if (lane == 0) atomicOr(prm.status, 4u);
-                ok_all = false;
-                break;
+        for (int b0 = 0; b0 < n && ok_all; b0 += K::CHUNK) {
+            const int nb = min(K::CHUNK, n - b0);
+            if (lane >= b0 && lane < b0 + nb) {
+                float ux, uy, uz, il;
+                const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
+                float Y[K::D_SH];
+                sh_eval<K::LSH>(ok, ux, uy, uz, Y);
+                compute_A<K>(Y, As + (lane - b0) * K::NA_PAD);
             }
-            const bool valid = __shfl_sync(0xffffffffu, my_s, t) >= 0;
-            float xv[K::D_IN][V], wv[K::NP][V];
-#pragma unroll
-            for (int p = 0; p < K::NP; ++p) {
-                if (active)
-                    lds_vec<V>(wv[p], st + p * K::TILE_C + cl);
-                else
-#pragma unroll
-                    for (int v = 0; v < V; ++v) wv[p][v] = 0.f;
-            }
-#pragma unroll
-            for (int d = 0; d < K::D_IN; ++d) {
-                if (active && valid)
-                    lds_vec<V>(xv[d], st + (K::NP + d) * K::TILE_C + cl);
-                else
-#pragma unroll
-                    for (int v = 0; v < V; ++v) xv[d][v] = 0.f;
-            }
-            fwd_edge<K>(As + t * K::NA_PAD, xv, wv, acc);
             __syncwarp();
-            if (t + S < n) {
-                const int e = __shfl_sync(0xffffffffu, my_e, t + S), s = __shfl_sync(0xffffffffu, my_s, t + S);
-                stage_fill<K, K::D_IN>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_x, e, s < 0 ? 0 : s, c0, pol_stream,
-                                       pol_keep, lane);
+            for (int t = b0; t < b0 + nb; ++t) {
+                const uint32_t gi = g + t;
+                float* st = stages + (gi % S) * SF;
+                if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
+                    if (lane == 0) atomicOr(prm.status, 4u);
+                    ok_all = false;
+                    break;
+                }
+                // inactive lanes (past C in a ragged tile) compute on zeros; the
+                // predicate also keeps the compiler from hoisting every row load
+                float xv[K::D_IN][V], wv[K::NP][V];
+#pragma unroll
+                for (int p = 0; p < K::NP; ++p) {
+                    if (active)
+                        lds_vec<V>(wv[p], st + p * K::TILE_C + cl);
+                    else
+#pragma unroll
+                        for (int v = 0; v < V; ++v) wv[p][v] = 0.f;
+                }
+#pragma unroll
+                for (int d = 0; d < K::D_IN; ++d) {
+                    if (active)
+                        lds_vec<V>(xv[d], st + (K::NP + d) * K::TILE_C + cl);
+                    else
+#pragma unroll
+                        for (int v = 0; v < V; ++v) xv[d][v] = 0.f;
+                }
+                fwd_edge<K>(As + (t - b0) * K::NA_PAD, xv, wv, acc);
+                __syncwarp();
+                if (t + S < n) {
+                    const int e = __shfl_sync(0xffffffffu, my_e, t + S), s = __shfl_sync(0xffffffffu, my_s, t + S);
+                    stage_fill<K, K::D_IN>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_x, e, s, c0, pol_stream,
+                                           pol_keep, lane);
+                }
             }
+            __syncwarp();
         }
         g += n;
-        __syncwarp();
     }
     if (!ok_all) {
         // drain: wait (bounded) for copies still in flight before the warp exits
         for (int s = 0; s < S; ++s) mbar_wait(&bars[2 * s], 0), mbar_wait(&bars[2 * s], 1);
         return;
     }
-    if (active) {
+    // a later band adds its sum; a band without edges for this node leaves y as it is
+    if (active && (!prm.accumulate || g > 0)) {
         float* yi = prm.y + (size_t)node * K::D_OUT * C + c0 + cl;
 #pragma unroll
-        for (int d = 0; d < K::D_OUT; ++d) st_stream<V>(yi + (size_t)d * C, acc[d]);
+        for (int d = 0; d < K::D_OUT; ++d) {
+            if (prm.accumulate) {
+                float old[V];
+                ld_keep<V>(old, yi + (size_t)d * C, pol_stream);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[d][v] += old[v];
+            }
+            st_stream<V>(yi + (size_t)d * C, acc[d]);
+        }
     }
 }
 
@@ -741,116 +797,122 @@ __global__ void __launch_bounds__(K::WARPS * 32)
 
     uint32_t g = 0;
     bool ok_all = true;
-    const int kb = prm.ptr[node], ke = prm.ptr[node + 1];
-    for (int k0 = kb; k0 < ke && ok_all; k0 += K::CHUNK) {
-        const int n = min(K::CHUNK, ke - k0);
-        int my_e = 0, my_o = -1;
-        float rx = 0.f, ry = 0.f, rz = 0.f;
-        if (lane < n) {
-            my_e = prm.perm[k0 + lane];
-            const int o = prm.other[my_e];
-            if ((unsigned)o < (unsigned)prm.N)
-                my_o = o;
-            else
-                atomicOr(prm.status, 1u);
-            const float* re = prm.r + (size_t)my_e * 3;
-            rx = re[0];
-            ry = re[1];
-            rz = re[2];
-        }
+    int k = prm.ptr[node];
+    const int ke = prm.ptr[node + 1];
+    while (k < ke && ok_all) {
+        int my_e, my_o;
+        float rx, ry, rz;
+        const int n = gather_window(prm.perm, prm.other, prm.r, prm.N, prm.band_lo, prm.band_hi, k, ke, prm.status,
+                                    lane, my_e, my_o, rx, ry, rz);
+        if (n == 0) continue;
+        // the copy pipeline runs S edges ahead across the whole window
         const int pre = min(S, n);
         for (int t = 0; t < pre; ++t) {
             const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_o, t);
             const uint32_t gi = g + t;
-            stage_fill<K, DL>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e, o < 0 ? 0 : o, c0,
-                              pol_stream, pol_keep, lane);
+            stage_fill<K, DL>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e, o, c0, pol_stream,
+                              pol_keep, lane);
         }
-        if (lane < n) {
-            float ux, uy, uz, il;
-            const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
-            float Y[K::D_SH];
-            sh_eval<K::LSH>(ok, ux, uy, uz, Y);
-            compute_A<K>(Y, As + lane * K::NA_PAD);
-        }
-        __syncwarp();
-        for (int t = 0; t < n; ++t) {
-            const uint32_t gi = g + t;
-            float* st = stages + (gi % S) * SF;
-            if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
-                if (lane == 0) atomicOr(prm.status, 4u);
-                ok_all = false;
-                break;
+        for (int b0 = 0; b0 < n && ok_all; b0 += K::CHUNK) {
+            const int nb = min(K::CHUNK, n - b0);
+            if (lane >= b0 && lane < b0 + nb) {
+                float ux, uy, uz, il;
+                const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
+                float Y[K::D_SH];
+                sh_eval<K::LSH>(ok, ux, uy, uz, Y);
+                compute_A<K>(Y, As + (lane - b0) * K::NA_PAD);
             }
-            const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_o, t);
-            const SmemRows<V> Wr{st + cl, K::TILE_C, active};
-            const SmemRows<V> Lr{st + K::NP * K::TILE_C + cl, K::TILE_C, active && o >= 0};
-            float gyl[GG];
+            __syncwarp();
+            for (int t = b0; t < b0 + nb; ++t) {
+                const uint32_t gi = g + t;
+                float* st = stages + (gi % S) * SF;
+                if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
+                    if (lane == 0) atomicOr(prm.status, 4u);
+                    ok_all = false;
+                    break;
+                }
+                const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_o, t);
+                // inactive lanes (past C in a ragged tile) read zeros; the predicate
+                // also keeps the compiler from hoisting every row load
+                const SmemRows<V> Wr{st + cl, K::TILE_C, active};
+                const SmemRows<V> Lr{st + K::NP * K::TILE_C + cl, K::TILE_C, active};
+                float gyl[GG];
 #pragma unroll
-            for (int k = 0; k < GG; ++k) gyl[k] = 0.f;
-            float* dwe = prm.dw + (size_t)e * K::NP * C + c_off;
-            auto store_dw = [&](int p, const float* dwv) {
-                if (active) st_stream<V>(dwe + (size_t)p * C, dwv);
-            };
-            if constexpr (DET) {
-                auto no_sink = [](int, int, const float (&)[1][V]) {};
-                bwd_edge<K, true>(As + t * K::NA_PAD, RegRows<V, K::D_IN>{xres}, Lr, Wr, dxacc, no_sink, gyl,
-                                  store_dw);
-            } else {
-                float* dxs = prm.dx + (size_t)(o < 0 ? 0 : o) * K::D_IN * C + c_off;
-                const bool add = active && o >= 0;
-                auto sink = [&](int o1, int d1, const float (&blk)[2 * kMaxL + 1][V]) {
-                    if (add)
-#pragma unroll
-                        for (int m = 0; m < d1; ++m) red_add<V>(dxs + (size_t)(o1 + m) * C, blk[m]);
+                for (int q = 0; q < GG; ++q) gyl[q] = 0.f;
+                float* dwe = prm.dw + (size_t)e * K::NP * C + c_off;
+                auto store_dw = [&](int p, const float* dwv) {
+                    if (active) st_stream<V>(dwe + (size_t)p * C, dwv);
                 };
-                bwd_edge<K, false>(As + t * K::NA_PAD, Lr, RegRows<V, K::D_OUT>{gres}, Wr, dxacc, sink, gyl,
-                                   store_dw);
-            }
-            if constexpr (K::G > 0) {
-                warp_sum<K::G>(gyl);
-                if (lane == 0) {
-                    if constexpr (FUSED) {
+                if constexpr (DET) {
+                    auto no_sink = [](int, int, const float (&)[1][V]) {};
+                    bwd_edge<K, true>(As + (t - b0) * K::NA_PAD, RegRows<V, K::D_IN>{xres}, Lr, Wr, dxacc, no_sink,
+                                      gyl, store_dw);
+                } else {
+                    float* dxs = prm.dx + (size_t)o * K::D_IN * C + c_off;
+                    auto sink = [&](int o1, int d1, const float (&blk)[2 * kMaxL + 1][V]) {
+                        if (active)
 #pragma unroll
-                        for (int k = 0; k < K::G; ++k) gYs[t * K::GS + k] = gyl[k];
-                    } else {
-                        float* gp = prm.gy_part + ((size_t)e * prm.T + tile) * K::G;
+                            for (int m = 0; m < d1; ++m) red_add<V>(dxs + (size_t)(o1 + m) * C, blk[m]);
+                    };
+                    bwd_edge<K, false>(As + (t - b0) * K::NA_PAD, Lr, RegRows<V, K::D_OUT>{gres}, Wr, dxacc, sink,
+                                       gyl, store_dw);
+                }
+                if constexpr (K::G > 0) {
+                    warp_sum<K::G>(gyl);
+                    if (lane == 0) {
+                        if constexpr (FUSED) {
 #pragma unroll
-                        for (int k = 0; k < K::G; ++k) gp[k] = gyl[k];
+                            for (int q = 0; q < K::G; ++q) gYs[(t - b0) * K::GS + q] = gyl[q];
+                        } else {
+                            float* gp = prm.gy_part + ((size_t)e * prm.T + tile) * K::G;
+#pragma unroll
+                            for (int q = 0; q < K::G; ++q) gp[q] = gyl[q];
+                        }
                     }
+                }
+                __syncwarp();
+                if (t + S < n) {
+                    const int e2 = __shfl_sync(0xffffffffu, my_e, t + S), o2 = __shfl_sync(0xffffffffu, my_o, t + S);
+                    stage_fill<K, DL>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e2, o2, c0, pol_stream, pol_keep,
+                                      lane);
                 }
             }
             __syncwarp();
-            if (t + S < n) {
-                const int e2 = __shfl_sync(0xffffffffu, my_e, t + S), o2 = __shfl_sync(0xffffffffu, my_o, t + S);
-                stage_fill<K, DL>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e2, o2 < 0 ? 0 : o2, c0, pol_stream,
-                                  pol_keep, lane);
+            if constexpr (FUSED) {
+                if (ok_all && lane >= b0 && lane < b0 + nb) {
+                    float ux, uy, uz, il;
+                    const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
+                    float d0 = 0.f, d1 = 0.f, d2 = 0.f;
+                    if constexpr (K::G > 0)
+                        sh_grad_contract<K::LSH>(ok, ux, uy, uz, il, gYs + (lane - b0) * K::GS, d0, d1, d2);
+                    float* dre = prm.dr + (size_t)my_e * 3;
+                    dre[0] = d0;
+                    dre[1] = d1;
+                    dre[2] = d2;
+                }
+                __syncwarp();
             }
         }
         g += n;
-        __syncwarp();
-        if constexpr (FUSED) {
-            if (ok_all && lane < n) {
-                float ux, uy, uz, il;
-                const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
-                float d0 = 0.f, d1 = 0.f, d2 = 0.f;
-                if constexpr (K::G > 0) sh_grad_contract<K::LSH>(ok, ux, uy, uz, il, gYs + lane * K::GS, d0, d1, d2);
-                float* dre = prm.dr + (size_t)my_e * 3;
-                dre[0] = d0;
-                dre[1] = d1;
-                dre[2] = d2;
-            }
-            __syncwarp();
-        }
     }
     if (!ok_all) {
         for (int s = 0; s < S; ++s) mbar_wait(&bars[2 * s], 0), mbar_wait(&bars[2 * s], 1);
         return;
     }
     if constexpr (DET) {
-        if (active) {
+        // a later band adds its sum; a band without edges for this node leaves dx as it is
+        if (active && (!prm.accumulate || g > 0)) {
             float* dxj = prm.dx + (size_t)node * K::D_IN * C + c_off;
 #pragma unroll
-            for (int d = 0; d < K::D_IN; ++d) st_stream<V>(dxj + (size_t)d * C, dxacc[d]);
+            for (int d = 0; d < K::D_IN; ++d) {
+                if (prm.accumulate) {
+                    float old[V];
+                    ld_keep<V>(old, dxj + (size_t)d * C, pol_stream);
+#pragma unroll
+                    for (int v = 0; v < V; ++v) dxacc[d][v] += old[v];
+                }
+                st_stream<V>(dxj + (size_t)d * C, dxacc[d]);
+            }
         }
     }
 }

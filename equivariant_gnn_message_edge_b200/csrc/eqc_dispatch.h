@@ -18,8 +18,9 @@ struct BwdParams;
 
 struct KernelSet {
     int lin, lsh, lout, vec, tile_c, g;
-    cudaError_t (*fwd)(const FwdParams&, int tiles, cudaStream_t);
-    cudaError_t (*bwd)(const BwdParams&, bool det, bool fused, cudaStream_t);
+    // `bands` launches over consecutive ranges of the gathered node index
+    cudaError_t (*fwd)(const FwdParams&, int tiles, int bands, cudaStream_t);
+    cudaError_t (*bwd)(const BwdParams&, bool det, bool fused, int bands, cudaStream_t);
 };
 
 // Instances for one (L_in, L_sh); defined in eqc_inst_l<L_in>s<L_sh>.cu.

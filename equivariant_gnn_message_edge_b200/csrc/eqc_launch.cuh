@@ -27,7 +27,8 @@ static cudaError_t ensure_smem(Kern kern, int bytes, bool (&done)[64]) {
 
 template <class K>
 struct Launch {
-    static cudaError_t fwd(const FwdParams& prm, int tiles, cudaStream_t st) {
+    static cudaError_t fwd(const FwdParams& prm_in, int tiles, int bands, cudaStream_t st) {
+        FwdParams prm = prm_in;
         auto kern = eqconv_fwd_kernel<K>;
         static bool done[64] = {};
         constexpr int smem = K::WARPS * WarpSmem<K, K::D_IN, false>::BYTES;
@@ -41,12 +42,19 @@ struct Launch {
             !encode_rows_map(&tx, prm.x, (uint64_t)prm.N, K::D_IN, prm.C, K::TILE_C))
             return cudaErrorInvalidValue;
         dim3 grid((prm.N + K::WARPS - 1) / K::WARPS, tiles);
-        kern<<<grid, K::WARPS * 32, smem, st>>>(prm, tw, tx);
-        count_launch();
-        return cudaGetLastError();
+        for (int b = 0; b < bands; ++b) {
+            prm.band_lo = (int)((int64_t)prm.N * b / bands);
+            prm.band_hi = (int)((int64_t)prm.N * (b + 1) / bands);
+            prm.accumulate = b > 0;
+            kern<<<grid, K::WARPS * 32, smem, st>>>(prm, tw, tx);
+            count_launch();
+            if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        }
+        return cudaSuccess;
     }
     template <bool DET, bool FUSED>
-    static cudaError_t bwd_one(const BwdParams& prm, cudaStream_t st) {
+    static cudaError_t bwd_one(const BwdParams& prm_in, int bands, cudaStream_t st) {
+        BwdParams prm = prm_in;
         auto kern = eqconv_bwd_kernel<K, DET, FUSED>;
         static bool done[64] = {};
         constexpr int smem = K::WARPS * WarpSmem<K, DET ? K::D_OUT : K::D_IN, true>::BYTES;
@@ -58,13 +66,19 @@ struct Launch {
             !encode_rows_map(&tg, g, (uint64_t)prm.N, DET ? K::D_OUT : K::D_IN, prm.C, K::TILE_C))
             return cudaErrorInvalidValue;
         dim3 grid((prm.N + K::WARPS - 1) / K::WARPS, prm.T);
-        kern<<<grid, K::WARPS * 32, smem, st>>>(prm, tw, tg);
-        count_launch();
-        return cudaGetLastError();
+        for (int b = 0; b < bands; ++b) {
+            prm.band_lo = (int)((int64_t)prm.N * b / bands);
+            prm.band_hi = (int)((int64_t)prm.N * (b + 1) / bands);
+            prm.accumulate = b > 0;
+            kern<<<grid, K::WARPS * 32, smem, st>>>(prm, tw, tg);
+            count_launch();
+            if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        }
+        return cudaSuccess;
     }
-    static cudaError_t bwd(const BwdParams& prm, bool det, bool fused, cudaStream_t st) {
-        if (det) return fused ? bwd_one<true, true>(prm, st) : bwd_one<true, false>(prm, st);
-        return fused ? bwd_one<false, true>(prm, st) : bwd_one<false, false>(prm, st);
+    static cudaError_t bwd(const BwdParams& prm, bool det, bool fused, int bands, cudaStream_t st) {
+        if (det) return fused ? bwd_one<true, true>(prm, bands, st) : bwd_one<true, false>(prm, bands, st);
+        return fused ? bwd_one<false, true>(prm, bands, st) : bwd_one<false, false>(prm, bands, st);
     }
     static constexpr KernelSet make() {
         return KernelSet{K::LIN, K::LSH, K::LOUT, K::VEC, K::TILE_C, K::G, &fwd, &bwd};

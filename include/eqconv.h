@@ -104,6 +104,20 @@ EQCONV_API int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int
  * mode stays bitwise reproducible for a fixed width). */
 EQCONV_API int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec);
 
+/* L2 budget (bytes) of one gather band.  The forward and the atomic backward
+ * gather sender rows x[s], the deterministic backward gathers receiver rows
+ * gy[i], about 45 times per row.  When N x (rows gathered) x (channel tile)
+ * x 4 B exceeds the budget, the op runs as B launches over consecutive ranges
+ * of the gathered node index, each touching only that range's rows, so they
+ * stay in L2; y (or deterministic dx) is written by the first band and
+ * accumulated by the next ones in fixed order.  Default (no call): 40 MiB
+ * for the atomic backward (rows every SM reads stay in B200's L2 up to about
+ * that size) and no banding for the forward and the deterministic backward,
+ * which measured faster unbanded; a call sets the budget of all three, and 0
+ * disables banding.  A tuning knob: results agree within rounding for any
+ * budget, and deterministic mode is bitwise reproducible for a fixed budget. */
+EQCONV_API int eqconv_plan_set_gather_budget(eqconv_plan_t plan, size_t bytes);
+
 /* Sizes of the plan; paths_l1l2l3 (3*P ints, may be NULL) receives the paths. */
 EQCONV_API int eqconv_plan_info(eqconv_plan_t plan, int* P, int* D_in, int* D_sh, int* D_out,
                      int* paths_l1l2l3);

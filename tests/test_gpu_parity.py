@@ -118,6 +118,46 @@ def test_vector_widths_agree_with_oracle(vec):
         check_all(run_gpu(ins, L_sh, ins, C, N, s, rcv, r, x, w, gy, det=det, vec=vec), ref)
 
 
+@pytest.mark.parametrize("budget", [1, 150_000, 0])
+def test_gather_bands_agree_with_oracle(budget):
+    """Splitting the gathered node range into bands (budget 1 B: one band per
+    node up to 64 bands; 150 kB: a few bands; 0: none) changes only the
+    grouping of sums."""
+    L_in, L_sh, L_out, C, N, E = 2, 2, 2, 132, 150, 5000
+    s, rcv, r, x, w, gy = random_case(N, E, C, L_in, L_sh, L_out, seed=21)
+    ins = NAT(2)
+    ref = oracle_full(ins, L_sh, ins, C, N, s, rcv, r, x, w, gy)
+    for vec in ((2, 2), (4, 4)):
+        for det in (True, False):
+            conv = EqConv(ins, L_sh, ins, C)
+            conv.set_vec(*vec)
+            conv.set_gather_budget(budget)
+            g = conv.graph(to_dev(s), to_dev(rcv), N)
+            xd, rd, wd = to_dev(x), to_dev(r), to_dev(w)
+            y = conv.forward_raw(g, xd, rd, wd)
+            dx, dw, dr = conv.backward_raw(g, xd, rd, wd, to_dev(gy), deterministic=det)
+            torch.cuda.synchronize()
+            assert B.eqconv_get_device_error(conv.plan) == B.EQCONV_OK
+            check_all(dict(y=y.cpu().numpy(), dx=dx.cpu().numpy(), dw=dw.cpu().numpy(), dr=dr.cpu().numpy()), ref)
+
+
+def test_bands_deterministic_mode_reproducible():
+    L_in, L_sh, L_out, C, N, E = 2, 2, 2, 128, 300, 9000
+    s, rcv, r, x, w, gy = random_case(N, E, C, L_in, L_sh, L_out, seed=22)
+    ins = NAT(2)
+    conv = EqConv(ins, L_sh, ins, C)
+    conv.set_gather_budget(50_000)
+    g = conv.graph(to_dev(s), to_dev(rcv), N)
+    xd, rd, wd, gd = to_dev(x), to_dev(r), to_dev(w), to_dev(gy)
+    outs = []
+    for _ in range(2):
+        y = conv.forward_raw(g, xd, rd, wd)
+        dx, dw, dr = conv.backward_raw(g, xd, rd, wd, gd, deterministic=True)
+        torch.cuda.synchronize()
+        outs.append([t.cpu().numpy().tobytes() for t in (y, dx, dw, dr)])
+    assert outs[0] == outs[1]
+
+
 def test_tiny_workload_full():
     """The 256-atom periodic box (C=32, 0e+1o -> 0e+1o+2e, L_sh=2), checked in full."""
     W = wl.WORKLOADS["tiny"]
