@@ -160,13 +160,15 @@ int parse_natural_prefix(const char* s) {
     return expect - 1;
 }
 
-// Channel vector widths measured best on B200 at C = 128 (lmax 2 and 3):
-// 64-channel tiles for the forward and the atomic backward (their gathered
-// rows stay in L2 and more warps fit), 128-channel tiles for the
-// deterministic backward (fewer coupling-matrix builds per edge).
+// Channel vector widths measured best on B200 at C = 128: 64-channel tiles for
+// the forward and the atomic backward (their gathered rows stay in L2 and more
+// warps fit), 128-channel tiles for the deterministic backward (fewer
+// coupling-matrix builds per edge).  With an l = 3 block the backward's
+// unrolled per-edge code outgrows the instruction cache; 32-channel tiles
+// halve it and measured fastest for both backward modes.
 int default_fwd_vec(int) { return 2; }
-int default_det_vec(int C) { return C >= 128 ? 4 : 2; }
-int default_atomic_vec(int) { return 2; }
+int default_det_vec(int C, bool l3) { return l3 ? 1 : (C >= 128 ? 4 : 2); }
+int default_atomic_vec(bool l3) { return l3 ? 1 : 2; }
 
 int tiles_for(int C, int tile_c) { return (C + tile_c - 1) / tile_c; }
 
@@ -246,8 +248,9 @@ int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh, cons
     p->gather_budget = 0;
     p->budget_set = false;
     p->fwd_vec = default_fwd_vec(C);
-    p->det_vec = default_det_vec(C);
-    p->atomic_vec = default_atomic_vec(C);
+    const bool l3 = lin == 3 || L_sh == 3 || lout == 3;
+    p->det_vec = default_det_vec(C, l3);
+    p->atomic_vec = default_atomic_vec(l3);
     p->fwd_ks = eqc::find_instance(lin, L_sh, lout, p->fwd_vec);
     p->det_ks = eqc::find_instance(lin, L_sh, lout, p->det_vec);
     p->atomic_ks = eqc::find_instance(lin, L_sh, lout, p->atomic_vec);
@@ -270,7 +273,8 @@ int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh, cons
 
 int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec) {
     if (!plan) return EQCONV_ERR_INVALID_ARG;
-    if ((fwd_vec != 2 && fwd_vec != 4) || (bwd_vec != 2 && bwd_vec != 4)) return EQCONV_ERR_UNSUPPORTED;
+    const auto ok = [](int v) { return v == 1 || v == 2 || v == 4; };
+    if (!ok(fwd_vec) || !ok(bwd_vec)) return EQCONV_ERR_UNSUPPORTED;
     const eqc::KernelSet* f = eqc::find_instance(plan->lin, plan->lsh, plan->lout, fwd_vec);
     const eqc::KernelSet* b = eqc::find_instance(plan->lin, plan->lsh, plan->lout, bwd_vec);
     if (!f || !b) return EQCONV_ERR_UNSUPPORTED;

@@ -37,15 +37,18 @@ __global__ void k_iota(int* p, int n) {
     if (i < n) p[i] = i;
 }
 
-// counts[key]++ for keys in range; others set status bit 2.
+// counts[key]++ for keys in range; others set status bit 2.  Lanes of a warp
+// holding the same key add once (sorted keys would otherwise serialise on one
+// counter).
 __global__ void k_key_hist(const int* keys, int E, int N, int* counts, unsigned* status) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= E) return;
-    const int k = keys[i];
-    if ((unsigned)k < (unsigned)N)
-        atomicAdd(&counts[k], 1);
-    else
-        atomicOr(status, 2u);
+    const int lane = threadIdx.x & 31;
+    const bool inb = i < E;
+    const int k = inb ? keys[i] : 0;
+    const bool valid = inb && (unsigned)k < (unsigned)N;
+    if (inb && !valid) atomicOr(status, 2u);
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? k : -1 - lane);
+    if (valid && __ffs(peers) - 1 == lane) atomicAdd(&counts[k], __popc(peers));
 }
 
 // Block-level exclusive scan of kTile ints; writes block totals.

@@ -133,3 +133,85 @@ def make_graph(wl: Workload):
         return periodic_box_graph(wl.N, wl.box, wl.cutoff)
     s, rcv = poisson_graph(wl.N, wl.mean_degree)
     return s, rcv, random_edge_vectors(len(s))
+
+
+# ---------------------------------------------------------------- water box
+
+WATER_BOX = dict(n_atoms=1503, box=25.0, min_dist=0.9, cutoff=5.0, pad=0.10, C=128, L=3, hidden=64, n_bessel=8)
+
+
+def random_sequential_packing(n_atoms: int, box: float, min_dist: float, seed: int = SEED_GRAPH):
+    """Positions added one by one uniformly in a periodic cube, rejecting any
+    closer than min_dist (minimum image) to an accepted one."""
+    rng = np.random.default_rng(seed)
+    pos = np.empty((n_atoms, 3))
+    n = 0
+    while n < n_atoms:
+        cand = rng.uniform(0.0, box, size=(256, 3))
+        for c in cand:
+            if n:
+                d = pos[:n] - c
+                d -= box * np.round(d / box)
+                if np.min(np.einsum("ij,ij->i", d, d)) < min_dist * min_dist:
+                    continue
+            pos[n] = c
+            n += 1
+            if n == n_atoms:
+                break
+    return pos
+
+
+def padded_box_graph(pos: np.ndarray, box: float, cutoff: float, pad: float):
+    """Ordered pairs (receiver i, sender j != i) within the cutoff (minimum
+    image), r = pos[j] - pos[i], then int(E * pad) dummy edges i -> i
+    (round-robin over atoms, r = (cutoff, 0, 0)); everything sorted by receiver,
+    stable.  Returns (senders, receivers, r, is_dummy)."""
+    n = len(pos)
+    d = pos[None, :, :] - pos[:, None, :]
+    d -= box * np.round(d / box)
+    dist = np.linalg.norm(d, axis=-1)
+    mask = (dist < cutoff) & ~np.eye(n, dtype=bool)
+    recv, send = np.nonzero(mask)
+    r = d[recv, send]
+    n_pad = int(len(recv) * pad)
+    dummy_nodes = np.arange(n_pad) % n
+    recv = np.concatenate([recv, dummy_nodes])
+    send = np.concatenate([send, dummy_nodes])
+    r = np.concatenate([r, np.tile([[cutoff, 0.0, 0.0]], (n_pad, 1))])
+    is_dummy = np.concatenate([np.zeros(len(recv) - n_pad, bool), np.ones(n_pad, bool)])
+    order = np.argsort(recv, kind="stable")
+    return (send[order].astype(np.int32), recv[order].astype(np.int32), r[order].astype(np.float32),
+            is_dummy[order])
+
+
+def radial_mlp_params(P: int, C: int, hidden: int = 64, n_bessel: int = 8, seed: int = SEED_W):
+    """Seeded weights of the 2-hidden-layer radial MLP (n_bessel -> hidden ->
+    hidden -> P*C, SiLU), fp32, Kaiming-style scaling."""
+    rng = np.random.default_rng(seed)
+    dims = [n_bessel, hidden, hidden, P * C]
+    return [(rng.standard_normal((a, b)).astype(np.float32) / np.float32(np.sqrt(a))) for a, b in zip(dims[:-1], dims[1:])]
+
+
+def radial_weights(r: np.ndarray, cutoff: float, params, P: int, C: int, is_dummy=None,
+                   n_bessel: int = 8, p_env: int = 6) -> np.ndarray:
+    """w[E, P, C] = envelope(d) * MLP(bessel(d)) for d = |r| (fp32): Bessel
+    basis sqrt(2/rc) sin(n pi d / rc) / d, n = 1..n_bessel; polynomial envelope
+    of order p_env (1 at d = 0, zero with its first two derivatives at the
+    cutoff); dummy edges get w = 0."""
+    d = np.linalg.norm(r.astype(np.float64), axis=1)
+    u = np.clip(d / cutoff, 0.0, 1.0)
+    p = p_env
+    env = 1.0 - (p + 1) * (p + 2) / 2 * u ** p + p * (p + 2) * u ** (p + 1) - p * (p + 1) / 2 * u ** (p + 2)
+    n = np.arange(1, n_bessel + 1)
+    safe = np.maximum(d, 1e-9)
+    bes = np.sqrt(2.0 / cutoff) * np.sin(n[None, :] * np.pi * d[:, None] / cutoff) / safe[:, None]
+    silu = lambda z: z / (1.0 + np.exp(-z))
+    h = bes.astype(np.float32)
+    for i, W in enumerate(params):
+        h = h @ W
+        if i < len(params) - 1:
+            h = silu(h).astype(np.float32)
+    w = (h * env[:, None].astype(np.float32)).reshape(len(d), P, C).astype(np.float32)
+    if is_dummy is not None:
+        w[is_dummy] = 0.0
+    return w

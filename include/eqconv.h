@@ -96,12 +96,14 @@ typedef struct eqconv_graph_s {
 EQCONV_API int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh,
                        const char* irreps_out, int C);
 
-/* Channel vector width of the forward / backward kernels (2 or 4 channels per
- * lane, i.e. channel tiles of 64 or 128 channels).  Defaults (measured best on
- * B200 at C = 128): 2 for the forward and the atomic backward, 4 for the
- * deterministic backward when C >= 128.  bwd_vec sets both backward modes.  A
- * tuning knob; results agree within rounding across widths (deterministic
- * mode stays bitwise reproducible for a fixed width). */
+/* Channel vector width of the forward / backward kernels (1, 2 or 4 channels
+ * per lane, i.e. channel tiles of 32, 64 or 128 channels; width 1 exists only
+ * for plans with an l = 3 block and falls back to 2 otherwise).  Defaults
+ * (measured best on B200 at C = 128): 2 for the forward; for the backward 4
+ * (deterministic, C >= 128) or 2 (atomic), and 1 for both modes when the plan
+ * has an l = 3 block.  bwd_vec sets both backward modes.  A tuning knob;
+ * results agree within rounding across widths (deterministic mode stays
+ * bitwise reproducible for a fixed width). */
 EQCONV_API int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec);
 
 /* L2 budget (bytes) of one gather band.  The forward and the atomic backward

@@ -108,11 +108,13 @@ def test_conv_parity(case, det):
     check_all(res, oracle_full(ins, L_sh, outs, C, N, s, rcv, r, x, w, gy))
 
 
-@pytest.mark.parametrize("vec", [(2, 2), (4, 4), (2, 4), (4, 2)])
-def test_vector_widths_agree_with_oracle(vec):
-    L_in, L_sh, L_out, C, N, E = 2, 2, 2, 128, 200, 6000
+@pytest.mark.parametrize("lmax", [2, 3])
+@pytest.mark.parametrize("vec", [(2, 2), (4, 4), (2, 4), (4, 2), (1, 1), (2, 1)])
+def test_vector_widths_agree_with_oracle(vec, lmax):
+    """Width 1 exists for plans with an l = 3 block and falls back to 2 else."""
+    L_in, L_sh, L_out, C, N, E = lmax, lmax, lmax, 128, 120, 3000
     s, rcv, r, x, w, gy = random_case(N, E, C, L_in, L_sh, L_out, seed=5)
-    ins = NAT(2)
+    ins = NAT(lmax)
     ref = oracle_full(ins, L_sh, ins, C, N, s, rcv, r, x, w, gy)
     for det in (True, False):
         check_all(run_gpu(ins, L_sh, ins, C, N, s, rcv, r, x, w, gy, det=det, vec=vec), ref)
