@@ -196,7 +196,7 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     W = wl.WORKLOADS[args.workload]
-    conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C, all_parity=W.all_parity, per_path=W.per_path)
     if args.vec:
         conv.set_vec(*[int(v) for v in args.vec.split(",")])
     if args.gather_budget_mib is not None:
@@ -362,13 +362,15 @@ def run_native(args, rank, world, local_rank):
     fb_gbs = (bc["fwd"] + bc["bwd"]) / ((med(fwd_ms) + med(bwd_ms)) * 1e-3) / 1e9
     bwd_avg = sum(bwd_ms) / len(bwd_ms)
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
-    traffic = load_traffic()
+    layout = f" (per-path blocks, D_out={D_out})" if W.per_path else ""
+    # ncu counters hold for the default launch configuration only
+    traffic = load_traffic(W.name) if not (args.vec or args.gather_budget_mib is not None) else {}
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded NumPy PCG64)",
         "config": {
-            "workload": f"{W.name}: N={N}, C={C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}, L_sh={W.L_sh}, "
+            "workload": f"{W.name}: N={N}, C={C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}{layout}, L_sh={W.L_sh}, "
                         f"P={P}, in-degree Poisson({W.mean_degree:g}), uniform senders",
             "step": "graph build (recv+send CSR) + fused forward + fused deterministic backward",
             "l2": "inputs larger than L2 (w alone is %.1f GB)" % (bc["step"] and 4 * E * P * C / 1e9),
@@ -400,10 +402,11 @@ def run_native(args, rank, world, local_rank):
     return result, inp, (N, E, C, D_in, D_out, P)
 
 
-def load_traffic():
-    """DRAM bytes per launch from the committed ncu summary; empty (so the
-    roofline's traffic is null) when absent or when the kernel sources have
-    changed since the counters were taken."""
+def load_traffic(workload):
+    """DRAM bytes per launch of the forward and the deterministic backward
+    for `workload` from the committed ncu summary; empty (so the roofline's
+    traffic is null) when absent, when that workload was not captured, or
+    when the kernel sources have changed since the counters were taken."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -413,7 +416,9 @@ def load_traffic():
         for rel in d["kernel_sources"]:
             with open(os.path.join(ROOT, rel), "rb") as f:
                 h.update(f.read())
-        return d if h.hexdigest() == d["kernel_sources_sha256"] else {}
+        if h.hexdigest() != d["kernel_sources_sha256"]:
+            return {}
+        return d["workloads"].get(workload, {})
     except Exception:
         return {}
 
@@ -436,7 +441,7 @@ def oracle_sample_step(name, n_recv, D_in, D_out, P, x=None, gy=None, nthreads=0
         x = wl.features(W.N, D_in, W.C, wl.SEED_X)
     if gy is None:
         gy = wl.features(W.N, D_out, W.C, wl.SEED_GY)
-    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C, per_path=W.per_path)
     t = time.perf_counter()
     rp, rperm = csr(r_s, W.N)
     sp, sperm = csr(s_s, W.N)
@@ -474,7 +479,7 @@ def run_reference(args, rank, world):
     from oracle import conv as oconv
     obuild.build()
     W = wl.WORKLOADS[args.workload]
-    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C, per_path=W.per_path)
     s, rcv, r = wl.make_graph(W)
     E = len(s)
     bc = byte_counts(W.N, E, W.C, prob.D_in, prob.D_out, prob.P)
@@ -496,7 +501,8 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded NumPy PCG64)",
-        "config": {"workload": f"{W.name}: N={W.N}, C={W.C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}, "
+        "config": {"workload": f"{W.name}: N={W.N}, C={W.C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}"
+                               f"{' (per-path blocks)' if W.per_path else ''}, "
                                f"L_sh={W.L_sh}, P={prob.P}",
                    "step": "graph build + forward + backward (dx, dw, dr), oracle on a bounded sample"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oconv.max_threads(), "kind": "oracle",

@@ -25,6 +25,8 @@ EQCONV_ERR_CUDA = 3
 EQCONV_ERR_WORKSPACE = 4
 EQCONV_ERR_DEVICE_CHECK = 5
 EQCONV_DETERMINISTIC = 1
+EQCONV_OUT_ALL_PARITY = 1
+EQCONV_OUT_PER_PATH = 2
 
 ABI_FUNCTIONS = (
     "eqconv_plan_create", "eqconv_plan_set_vec", "eqconv_plan_info", "eqconv_enumerate_paths", "eqconv_cg_table",
@@ -32,6 +34,7 @@ ABI_FUNCTIONS = (
     "eqconv_backward_workspace_bytes", "eqconv_backward", "eqconv_spherical_harmonics",
     "eqconv_get_device_error", "eqconv_plan_destroy", "eqconv_status_string", "eqconv_launch_count",
     "eqconv_last_error", "eqconv_graph_build_noalloc", "eqconv_plan_set_gather_budget",
+    "eqconv_plan_create_ex", "eqconv_plan_path_rows", "eqconv_enumerate_paths_ex",
 )
 
 
@@ -60,6 +63,9 @@ _pg = ctypes.POINTER(eqconv_graph_t)
 
 _SIGS = {
     "eqconv_plan_create": (_ci, [ctypes.POINTER(_vp), ctypes.c_char_p, _ci, ctypes.c_char_p, _ci]),
+    "eqconv_plan_create_ex": (_ci, [ctypes.POINTER(_vp), ctypes.c_char_p, _ci, ctypes.c_char_p, _ci, _cu]),
+    "eqconv_plan_path_rows": (_ci, [_vp, _pi]),
+    "eqconv_enumerate_paths_ex": (_ci, [ctypes.c_char_p, _ci, ctypes.c_char_p, _cu, _pi, _pi, _pi, _pi, _ci]),
     "eqconv_plan_set_vec": (_ci, [_vp, _ci, _ci]),
     "eqconv_plan_set_gather_budget": (_ci, [_vp, _sz]),
     "eqconv_plan_info": (_ci, [_vp, _pi, _pi, _pi, _pi, _pi]),
@@ -157,6 +163,34 @@ def eqconv_plan_create(irreps_in: str, L_sh: int, irreps_out: str, C: int) -> in
     _check(lib().eqconv_plan_create(ctypes.byref(h), irreps_in.encode(), int(L_sh), irreps_out.encode(), int(C)),
            "eqconv_plan_create")
     return h.value
+
+
+def eqconv_plan_create_ex(irreps_in: str, L_sh: int, irreps_out: str, C: int, out_mode: int) -> int:
+    h = _vp()
+    _check(lib().eqconv_plan_create_ex(ctypes.byref(h), irreps_in.encode(), int(L_sh), irreps_out.encode(), int(C),
+                                       int(out_mode)), "eqconv_plan_create_ex")
+    return h.value
+
+
+def eqconv_plan_path_rows(plan: int) -> list:
+    P = eqconv_plan_info(plan)["P"]
+    buf = (ctypes.c_int * max(1, P))()
+    _check(lib().eqconv_plan_path_rows(plan, buf), "eqconv_plan_path_rows")
+    return list(buf[:P])
+
+
+def eqconv_enumerate_paths_ex(irreps_in: str, L_sh: int, irreps_out: str, out_mode: int) -> dict:
+    """{'paths': [(l1, l2, l3)], 'rows': [first output row], 'D_out': n}."""
+    P, D = ctypes.c_int(), ctypes.c_int()
+    args = (irreps_in.encode(), int(L_sh), irreps_out.encode(), int(out_mode))
+    _check(lib().eqconv_enumerate_paths_ex(*args, ctypes.byref(P), None, None, ctypes.byref(D), 0),
+           "eqconv_enumerate_paths_ex")
+    paths = (ctypes.c_int * max(1, 3 * P.value))()
+    rows = (ctypes.c_int * max(1, P.value))()
+    _check(lib().eqconv_enumerate_paths_ex(*args, ctypes.byref(P), paths, rows, ctypes.byref(D), P.value),
+           "eqconv_enumerate_paths_ex")
+    return dict(paths=[tuple(paths[3 * i:3 * i + 3]) for i in range(P.value)], rows=list(rows[:P.value]),
+                D_out=D.value)
 
 
 def eqconv_plan_set_vec(plan: int, fwd_vec: int, bwd_vec: int) -> None:

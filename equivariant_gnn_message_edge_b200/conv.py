@@ -41,14 +41,22 @@ class Graph:
 
 
 class EqConv:
-    """One convolution configuration (irreps, L_sh, C) on the current device."""
+    """One convolution configuration (irreps, L_sh, C) on the current device.
 
-    def __init__(self, irreps_in: str, L_sh: int, irreps_out: str, C: int):
+    all_parity: outputs of both parities (irreps_out is then the both-parity
+    prefix "0e+1o+1e+2e+2o..."); per_path: one output block per path, in path
+    order, starting at row ``self.path_rows[p]`` (see include/eqconv.h)."""
+
+    def __init__(self, irreps_in: str, L_sh: int, irreps_out: str, C: int, all_parity: bool = False,
+                 per_path: bool = False):
         self.irreps_in, self.L_sh, self.irreps_out, self.C = irreps_in, L_sh, irreps_out, C
-        self.plan = B.eqconv_plan_create(irreps_in, L_sh, irreps_out, C)
+        mode = (B.EQCONV_OUT_ALL_PARITY if all_parity else 0) | (B.EQCONV_OUT_PER_PATH if per_path else 0)
+        self.out_mode = mode
+        self.plan = B.eqconv_plan_create_ex(irreps_in, L_sh, irreps_out, C, mode)
         info = B.eqconv_plan_info(self.plan)
         self.P, self.D_in, self.D_sh, self.D_out = info["P"], info["D_in"], info["D_sh"], info["D_out"]
         self.paths = info["paths"]
+        self.path_rows = B.eqconv_plan_path_rows(self.plan)
 
     def __del__(self):
         try:

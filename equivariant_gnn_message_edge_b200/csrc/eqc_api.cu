@@ -17,6 +17,8 @@
 #include <cstring>
 #include <new>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "eqc_conv.cuh"
 #include "eqc_dispatch.h"
@@ -115,8 +117,10 @@ struct eqconv_plan_s {
     int fwd_vec, det_vec, atomic_vec;
     size_t gather_budget;   // bytes of gathered rows one band may touch (0: one band)
     bool budget_set;        // false: per-mode defaults (bands for the atomic backward only)
+    int mode;               // output variant bits (eqc::kModeAllParity, eqc::kModePerPath)
     int P, D_in, D_sh, D_out;
     int paths[eqc::kMaxPaths][3];
+    int path_rows[eqc::kMaxPaths];
     int device;
     unsigned* d_status;
     const eqc::KernelSet* fwd_ks;
@@ -126,38 +130,71 @@ struct eqconv_plan_s {
 
 namespace {
 
-// "0e+1o+2e" (optionally "1x0e + 1x1o ...") -> L when it is the natural-parity
-// prefix 0..L; -1 if malformed, -2 if well formed but not such a prefix.
-int parse_natural_prefix(const char* s) {
-    if (!s) return -1;
+// Irreps string -> list of (l, parity +1/-1); "1x" multiplicities and spaces
+// are accepted.  False if malformed.
+bool parse_irreps(const char* s, std::vector<std::pair<int, int>>& out) {
+    out.clear();
+    if (!s) return false;
     std::string t;
     for (const char* c = s; *c; ++c)
         if (!std::isspace((unsigned char)*c)) t.push_back(*c);
-    if (t.empty()) return -1;
-    int expect = 0;
+    if (t.empty()) return false;
     size_t i = 0;
-    bool prefix = true;
-    while (i < t.size()) {
+    while (i <= t.size()) {
         size_t j = t.find('+', i);
         if (j == std::string::npos) j = t.size();
         std::string tok = t.substr(i, j - i);
         if (tok.size() >= 2 && tok[0] == '1' && tok[1] == 'x') tok = tok.substr(2);
-        if (tok.size() < 2) return -1;
+        if (tok.size() < 2) return false;
         const char par = tok.back();
-        if (par != 'e' && par != 'o') return -1;
+        if (par != 'e' && par != 'o') return false;
         const std::string num = tok.substr(0, tok.size() - 1);
-        if (num.empty() || num.size() > 2) return -1;
+        if (num.empty() || num.size() > 2) return false;
         for (char ch : num)
-            if (!std::isdigit((unsigned char)ch)) return -1;
-        const int l = std::stoi(num);
-        const char nat = (l % 2 == 0) ? 'e' : 'o';
-        if (l != expect || par != nat) prefix = false;
-        ++expect;
-        i = j + 1;
+            if (!std::isdigit((unsigned char)ch)) return false;
+        out.emplace_back(std::stoi(num), par == 'e' ? 1 : -1);
         if (j == t.size()) break;
+        i = j + 1;
     }
-    if (!prefix) return -2;
-    return expect - 1;
+    return true;
+}
+
+// The canonical irreps list of degree 0..L: natural parity (0e, 1o, 2e, ...)
+// or both parities (0e, 1o, 1e, 2e, 2o, 3o, 3e, ...).
+std::vector<std::pair<int, int>> prefix_irreps(int L, bool all_parity) {
+    std::vector<std::pair<int, int>> v;
+    for (int l = 0; l <= L; ++l) {
+        const int nat = (l % 2 == 0) ? 1 : -1;
+        v.emplace_back(l, nat);
+        if (all_parity && l > 0) v.emplace_back(l, -nat);
+    }
+    return v;
+}
+
+// L when `s` is the canonical prefix 0..L (natural or both parities); -1 if
+// malformed, -2 if well formed but not such a prefix (or L > 3).
+int parse_prefix(const char* s, bool all_parity) {
+    std::vector<std::pair<int, int>> v;
+    if (!parse_irreps(s, v)) return -1;
+    for (int L = 0; L <= eqc::kMaxL; ++L)
+        if (v == prefix_irreps(L, all_parity)) return L;
+    return -2;
+}
+
+int parse_natural_prefix(const char* s) { return parse_prefix(s, false); }
+
+// Validates (irreps_in, L_sh, irreps_out, out_mode) and enumerates the paths.
+int plan_paths(const char* irreps_in, int L_sh, const char* irreps_out, unsigned out_mode, int& lin, int& lout,
+               eqc::PathList& PL) {
+    if (out_mode & ~(EQCONV_OUT_ALL_PARITY | EQCONV_OUT_PER_PATH)) return EQCONV_ERR_INVALID_ARG;
+    const int mode = (int)out_mode;
+    lin = parse_natural_prefix(irreps_in);
+    lout = parse_prefix(irreps_out, (mode & eqc::kModeAllParity) != 0);
+    if (lin == -1 || lout == -1 || L_sh < 0) return EQCONV_ERR_INVALID_ARG;
+    if (lin == -2 || lout == -2 || L_sh > eqc::kMaxL) return EQCONV_ERR_UNSUPPORTED;
+    PL = eqc::make_paths(lin, L_sh, lout, mode);
+    if (PL.n == 0) return EQCONV_ERR_UNSUPPORTED;
+    return EQCONV_OK;
 }
 
 // Channel vector widths measured best on B200 at C = 128: 64-channel tiles for
@@ -220,40 +257,51 @@ int cuda_status(cudaError_t e, const char* where) {
 extern "C" {
 
 int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh, const char* irreps_out, int C) {
+    return eqconv_plan_create_ex(out, irreps_in, L_sh, irreps_out, C, 0u);
+}
+
+int eqconv_plan_create_ex(eqconv_plan_t* out, const char* irreps_in, int L_sh, const char* irreps_out, int C,
+                          unsigned out_mode) {
     if (!out) return EQCONV_ERR_INVALID_ARG;
     *out = nullptr;
-    const int lin = parse_natural_prefix(irreps_in);
-    const int lout = parse_natural_prefix(irreps_out);
-    if (lin == -1 || lout == -1 || L_sh < 0 || C <= 0) return EQCONV_ERR_INVALID_ARG;
-    if (lin == -2 || lout == -2) return EQCONV_ERR_UNSUPPORTED;
-    if (lin > eqc::kMaxL || lout > eqc::kMaxL || L_sh > eqc::kMaxL) return EQCONV_ERR_UNSUPPORTED;
+    int lin = 0, lout = 0;
+    eqc::PathList PL{};
+    const int rc = plan_paths(irreps_in, L_sh, irreps_out, out_mode, lin, lout, PL);
+    if (rc != EQCONV_OK) return rc;
+    if (C <= 0) return EQCONV_ERR_INVALID_ARG;
     if (C % 4 != 0 || C < 4 || C > 4096) return EQCONV_ERR_UNSUPPORTED;
-    const eqc::PathList PL = eqc::make_paths(lin, L_sh, lout);
-    if (PL.n == 0) return EQCONV_ERR_UNSUPPORTED;
+    const int mode = (int)out_mode;
     eqconv_plan_s* p = new (std::nothrow) eqconv_plan_s();
     if (!p) return EQCONV_ERR_CUDA;
     p->lin = lin;
     p->lsh = L_sh;
     p->lout = lout;
     p->C = C;
+    p->mode = mode;
     p->P = PL.n;
     p->D_in = (lin + 1) * (lin + 1);
     p->D_sh = (L_sh + 1) * (L_sh + 1);
-    p->D_out = (lout + 1) * (lout + 1);
+    p->D_out = PL.dout;
     for (int i = 0; i < PL.n; ++i) {
         p->paths[i][0] = PL.l1[i];
         p->paths[i][1] = PL.l2[i];
         p->paths[i][2] = PL.l3[i];
+        p->path_rows[i] = PL.o3[i];
     }
     p->gather_budget = 0;
     p->budget_set = false;
-    p->fwd_vec = default_fwd_vec(C);
-    const bool l3 = lin == 3 || L_sh == 3 || lout == 3;
-    p->det_vec = default_det_vec(C, l3);
-    p->atomic_vec = default_atomic_vec(l3);
-    p->fwd_ks = eqc::find_instance(lin, L_sh, lout, p->fwd_vec);
-    p->det_ks = eqc::find_instance(lin, L_sh, lout, p->det_vec);
-    p->atomic_ks = eqc::find_instance(lin, L_sh, lout, p->atomic_vec);
+    if (mode == 0) {
+        p->fwd_vec = default_fwd_vec(C);
+        const bool l3 = lin == 3 || L_sh == 3 || lout == 3;
+        p->det_vec = default_det_vec(C, l3);
+        p->atomic_vec = default_atomic_vec(l3);
+        p->fwd_ks = eqc::find_instance(lin, L_sh, lout, p->fwd_vec);
+        p->det_ks = eqc::find_instance(lin, L_sh, lout, p->det_vec);
+        p->atomic_ks = eqc::find_instance(lin, L_sh, lout, p->atomic_vec);
+    } else {
+        p->fwd_vec = p->det_vec = p->atomic_vec = eqc::mode_vec(lin, L_sh, lout);
+        p->fwd_ks = p->det_ks = p->atomic_ks = eqc::find_mode_instance(lin, L_sh, lout, mode);
+    }
     if (!p->fwd_ks || !p->det_ks || !p->atomic_ks) {
         delete p;
         return EQCONV_ERR_UNSUPPORTED;
@@ -275,6 +323,11 @@ int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec) {
     if (!plan) return EQCONV_ERR_INVALID_ARG;
     const auto ok = [](int v) { return v == 1 || v == 2 || v == 4; };
     if (!ok(fwd_vec) || !ok(bwd_vec)) return EQCONV_ERR_UNSUPPORTED;
+    if (plan->mode != 0) {
+        // output variants are compiled at one width
+        const int v = eqc::mode_vec(plan->lin, plan->lsh, plan->lout);
+        return (fwd_vec == v && bwd_vec == v) ? EQCONV_OK : EQCONV_ERR_UNSUPPORTED;
+    }
     const eqc::KernelSet* f = eqc::find_instance(plan->lin, plan->lsh, plan->lout, fwd_vec);
     const eqc::KernelSet* b = eqc::find_instance(plan->lin, plan->lsh, plan->lout, bwd_vec);
     if (!f || !b) return EQCONV_ERR_UNSUPPORTED;
@@ -304,23 +357,39 @@ int eqconv_plan_info(eqconv_plan_t plan, int* P, int* D_in, int* D_sh, int* D_ou
     return EQCONV_OK;
 }
 
+int eqconv_plan_path_rows(eqconv_plan_t plan, int* out_rows) {
+    if (!plan || !out_rows) return EQCONV_ERR_INVALID_ARG;
+    for (int i = 0; i < plan->P; ++i) out_rows[i] = plan->path_rows[i];
+    return EQCONV_OK;
+}
+
 int eqconv_enumerate_paths(const char* irreps_in, int L_sh, const char* irreps_out, int* P, int* paths_l1l2l3,
                            int max_paths) {
+    return eqconv_enumerate_paths_ex(irreps_in, L_sh, irreps_out, 0u, P, paths_l1l2l3, nullptr, nullptr, max_paths);
+}
+
+int eqconv_enumerate_paths_ex(const char* irreps_in, int L_sh, const char* irreps_out, unsigned out_mode, int* P,
+                              int* paths_l1l2l3, int* out_rows, int* D_out, int max_paths) {
     if (!P) return EQCONV_ERR_INVALID_ARG;
-    const int lin = parse_natural_prefix(irreps_in);
-    const int lout = parse_natural_prefix(irreps_out);
-    if (lin == -1 || lout == -1 || L_sh < 0) return EQCONV_ERR_INVALID_ARG;
-    if (lin == -2 || lout == -2 || lin > eqc::kMaxL || lout > eqc::kMaxL || L_sh > eqc::kMaxL)
-        return EQCONV_ERR_UNSUPPORTED;
-    const eqc::PathList PL = eqc::make_paths(lin, L_sh, lout);
+    int lin = 0, lout = 0;
+    eqc::PathList PL{};
+    const int rc = plan_paths(irreps_in, L_sh, irreps_out, out_mode, lin, lout, PL);
+    if (rc == EQCONV_ERR_UNSUPPORTED && lin >= 0 && lout >= 0 && L_sh <= eqc::kMaxL && PL.n == 0) {
+        *P = 0;   // well-formed, no admissible path
+        if (D_out) *D_out = 0;
+        return EQCONV_OK;
+    }
+    if (rc != EQCONV_OK) return rc;
     *P = PL.n;
-    if (paths_l1l2l3) {
-        if (max_paths < PL.n) return EQCONV_ERR_INVALID_ARG;
-        for (int i = 0; i < PL.n; ++i) {
+    if (D_out) *D_out = PL.dout;
+    if ((paths_l1l2l3 || out_rows) && max_paths < PL.n) return EQCONV_ERR_INVALID_ARG;
+    for (int i = 0; i < PL.n; ++i) {
+        if (paths_l1l2l3) {
             paths_l1l2l3[3 * i] = PL.l1[i];
             paths_l1l2l3[3 * i + 1] = PL.l2[i];
             paths_l1l2l3[3 * i + 2] = PL.l3[i];
         }
+        if (out_rows) out_rows[i] = PL.o3[i];
     }
     return EQCONV_OK;
 }
@@ -329,7 +398,7 @@ int eqconv_cg_table(int l1, int l2, int l3, double* out, int out_len) {
     if (!out) return EQCONV_ERR_INVALID_ARG;
     if (l1 < 0 || l2 < 0 || l3 < 0 || l1 > eqc::kMaxL || l2 > eqc::kMaxL || l3 > eqc::kMaxL)
         return EQCONV_ERR_UNSUPPORTED;
-    if (l3 < eqc::iabs(l1 - l2) || l3 > l1 + l2 || ((l1 + l2 + l3) & 1)) return EQCONV_ERR_UNSUPPORTED;
+    if (l3 < eqc::iabs(l1 - l2) || l3 > l1 + l2) return EQCONV_ERR_UNSUPPORTED;
     const int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
     if (out_len < d1 * d2 * d3) return EQCONV_ERR_INVALID_ARG;
     const eqc::CG3 t = eqc::make_real_cg(l1, l2, l3);

@@ -11,7 +11,7 @@
 // Mapping (one warp = one node x one channel tile of 32*VEC channels; each
 // lane owns VEC consecutive channels, so every x / w / y row segment is a
 // coalesced 512 B (VEC=4) run):
-//   * edges are processed in chunks of CHUNK: lane t of the warp reads edge t
+//   * edges are processed in chunks (Cfg::chunk): lane t of the warp reads edge t
 //     of the chunk, evaluates Y(r_e) and the per-edge coupling matrices
 //       A_p[m3][m1] = sum_m2 C_p[m1,m2,m3] Y_{l2 m2}(r_e)        (l2 > 0)
 //     with the CG as compile-time immediates (zeros skipped), and stores
@@ -44,6 +44,15 @@
 #ifndef EQC_CHUNK_SMALL
 #define EQC_CHUNK_SMALL 0   // 0: 16 edges at VEC=4, 8 at narrower tiles
 #endif
+#ifndef EQC_CHUNK_LARGE
+#define EQC_CHUNK_LARGE 4   // edges per coupling sub-batch when A is large (l = 3)
+#endif
+#ifndef EQC_CHUNK_LARGE_ATOMIC
+#define EQC_CHUNK_LARGE_ATOMIC 8   // the same for the atomic backward (register-bound, 2 CTAs/SM)
+#endif
+#ifndef EQC_FWD_PRED
+#define EQC_FWD_PRED 1      // 1: predicate the forward row reads at VEC = 4; 2: at every width
+#endif
 
 namespace eqc {
 
@@ -64,30 +73,30 @@ constexpr int pad_odd4(int n) {
     return m;
 }
 
-template <int LIN_, int LSH_, int LOUT_, int VEC_>
+// MODE: output variant bits (kModeAllParity, kModePerPath; 0 = natural-parity
+// outputs summed over paths).
+template <int LIN_, int LSH_, int LOUT_, int VEC_, int MODE_ = 0>
 struct Cfg {
-    static constexpr int LIN = LIN_, LSH = LSH_, LOUT = LOUT_, VEC = VEC_;
-    static constexpr PathList PL = make_paths(LIN, LSH, LOUT);
+    static constexpr int LIN = LIN_, LSH = LSH_, LOUT = LOUT_, VEC = VEC_, MODE = MODE_;
+    static constexpr PathList PL = make_paths(LIN, LSH, LOUT, MODE);
     static constexpr int NP = PL.n;
     static constexpr int D_IN = (LIN + 1) * (LIN + 1);
     static constexpr int D_SH = (LSH + 1) * (LSH + 1);
-    static constexpr int D_OUT = (LOUT + 1) * (LOUT + 1);
+    static constexpr int D_OUT = PL.dout;
     static constexpr int G = D_SH - 1;              // dr needs gY for l2 > 0 only
     static constexpr AOffsets AO = make_aoffsets(PL);
     static constexpr int NA = AO.total;
     static constexpr int NA_PAD = pad_odd4(NA);     // row stride; NA_PAD/4 odd: conflict-free STS.128
-    // edges whose coupling matrices A sit in shared memory at a time
-    static constexpr int CHUNK = NA_PAD > 128 ? 8 : (EQC_CHUNK_SMALL > 0 ? EQC_CHUNK_SMALL : (VEC >= 4 ? 16 : 8));
+    // edges whose coupling matrices A sit in shared memory at a time; the
+    // atomic backward is held to two CTAs per SM by its registers, so it
+    // takes the larger batch, the other kernels gain occupancy from a small one
+    static constexpr int chunk(bool atomic_bwd) {
+        return NA_PAD > 128 ? (atomic_bwd ? EQC_CHUNK_LARGE_ATOMIC : EQC_CHUNK_LARGE)
+                            : (EQC_CHUNK_SMALL > 0 ? EQC_CHUNK_SMALL : (VEC >= 4 ? 16 : 8));
+    }
     static constexpr int GS = G | 1;                // gY row stride in shared memory (odd)
     static constexpr int TILE_C = 32 * VEC;
     static constexpr int STAGES = EQC_STAGES;       // edges staged ahead per warp (ring depth)
-    // per-warp shared memory (bytes) of the largest kernel of this instance,
-    // used to size the CTA so that two CTAs fit on one SM (<= 113 KB each)
-    static constexpr int WARP_BYTES_EST =
-        4 * (32 + ((CHUNK * NA_PAD + 31) & ~31) + ((CHUNK * GS + 31) & ~31) +
-             STAGES * (NP + (D_IN > D_OUT ? D_IN : D_OUT)) * TILE_C);
-    static constexpr int WARPS_FIT = (113 * 1024) / WARP_BYTES_EST;
-    static constexpr int WARPS = WARPS_FIT < 1 ? 1 : (WARPS_FIT > 4 ? 4 : WARPS_FIT);
     static_assert(NP > 0, "no admissible path");
 };
 
@@ -239,7 +248,7 @@ __device__ __forceinline__ void fwd_edge(const float* As, const float (&xv)[K::D
     static_for<K::NP>([&](auto pc) {
         constexpr int p = EQC_CV(pc);
         constexpr int l1 = K::PL.l1[p], l2 = K::PL.l2[p], l3 = K::PL.l3[p];
-        constexpr int d1 = 2 * l1 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o3 = l3 * l3;
+        constexpr int d1 = 2 * l1 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o3 = K::PL.o3[p];
         if constexpr (l2 == 0) {
             static_assert(l1 == l3, "l x 0 -> l");
 #pragma unroll
@@ -329,7 +338,7 @@ __device__ __forceinline__ void bwd_edge(const float* As, const XR& X, const GR&
     static_for<K::NP>([&](auto pc) {
         constexpr int p = EQC_CV(pc);
         constexpr int l1 = K::PL.l1[p], l2 = K::PL.l2[p], l3 = K::PL.l3[p];
-        constexpr int d1 = 2 * l1 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o3 = l3 * l3;
+        constexpr int d1 = 2 * l1 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o3 = K::PL.o3[p];
         [[maybe_unused]] constexpr bool first_of_block = (p == 0) || (K::PL.l1[p == 0 ? 0 : p - 1] != l1);
         [[maybe_unused]] constexpr bool last_of_block = (p == K::NP - 1) || (K::PL.l1[p + 1 < K::NP ? p + 1 : p] != l1);
         if constexpr (!DIRECT && first_of_block) {
@@ -534,17 +543,54 @@ __device__ __forceinline__ void stage_fill(float* st, uint64_t* bar, const CUten
 
 
 // Per-warp shared-memory layout (floats), every region 128-byte aligned:
-// [stages: S x FLOATS] [mbarriers: 16 B each] [A: CHUNK x NA_PAD] [gY: CHUNK x GS]
-template <class K, int NG, bool WITH_GY>
+// [stages: S x FLOATS] [mbarriers: 16 B each] [A: CH x NA_PAD] [gY: CH x GS]
+template <class K, int NG, bool WITH_GY, int CH>
 struct WarpSmem {
     static constexpr int S = K::STAGES;
     static constexpr int up32(int f) { return (f + 31) & ~31; }
     static constexpr int ST_F = S * Stage<K, NG>::FLOATS;
     static constexpr int BAR_F = up32(4 * S);
-    static constexpr int A_F = up32(K::CHUNK * K::NA_PAD);
-    static constexpr int GY_F = WITH_GY ? up32(K::CHUNK * K::GS) : 0;
+    static constexpr int A_F = up32(CH * K::NA_PAD);
+    static constexpr int GY_F = WITH_GY ? up32(CH * K::GS) : 0;
     static constexpr int TOTAL_F = ST_F + BAR_F + A_F + GY_F;
     static constexpr int BYTES = TOTAL_F * 4;
+};
+
+// Warps resident on one SM when CTAs of w warps take `warp_bytes` of shared
+// memory per warp (228 KB per SM, 1 KB of it reserved per CTA, at most 227 KB
+// per CTA).
+constexpr int resident_warps(int w, int warp_bytes) {
+    return w * warp_bytes > 227 * 1024 ? 0 : (228 * 1024 / (w * warp_bytes + 1024)) * w;
+}
+
+// Warps per CTA (1..4): the largest CTA that keeps within 10% of the most
+// warps resident any CTA size allows (larger CTAs mean fewer CTA launches
+// and tensor-map prefetches per SM).
+constexpr int best_warps(int warp_bytes) {
+    int most = 0;
+    for (int w = 1; w <= 4; ++w)
+        if (resident_warps(w, warp_bytes) > most) most = resident_warps(w, warp_bytes);
+    for (int w = 4; w > 1; --w)
+        if (10 * resident_warps(w, warp_bytes) >= 9 * most) return w;
+    return 1;
+}
+
+// Shared-memory layout and CTA shape of the forward and the backward kernels.
+template <class K>
+struct FwdShape {
+    static constexpr int CH = K::chunk(false);
+    using L = WarpSmem<K, K::D_IN, false, CH>;
+    static constexpr int WARPS = best_warps(L::BYTES);
+};
+template <class K, bool DET>
+struct BwdShape {
+    static constexpr int CH = K::chunk(!DET);
+    static constexpr int DL = DET ? K::D_OUT : K::D_IN;     // rows gathered per edge
+    using L = WarpSmem<K, DL, true, CH>;
+    // the atomic kernel keeps the receiver's gy rows in registers and is held
+    // by them (up to 255 per thread at l = 3), not by shared memory: it takes
+    // 4-warp CTAs, which the register file fits twice
+    static constexpr int WARPS = (!DET && resident_warps(4, L::BYTES) > 0) ? 4 : best_warps(L::BYTES);
 };
 
 // Collects the next window of up to 32 edges of a node's list whose gathered
@@ -598,16 +644,18 @@ __device__ __forceinline__ int gather_window(const int* perm, const int* other, 
 // ---------------------------------------------------------------- forward
 
 template <class K>
-__global__ void __launch_bounds__(K::WARPS * 32)
+__global__ void __launch_bounds__(FwdShape<K>::WARPS * 32)
     eqconv_fwd_kernel(const FwdParams prm, const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_x) {
     constexpr int V = K::VEC;
     constexpr int S = K::STAGES;
-    using L = WarpSmem<K, K::D_IN, false>;
+    constexpr int CH = FwdShape<K>::CH;
+    constexpr int WARPS = FwdShape<K>::WARPS;
+    using L = typename FwdShape<K>::L;
     constexpr int SF = Stage<K, K::D_IN>::FLOATS;
     extern __shared__ __align__(128) float4 smem4[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int node = blockIdx.x * K::WARPS + warp;
+    const int node = blockIdx.x * WARPS + warp;
     if (node >= prm.N) return;
     float* stages = reinterpret_cast<float*>(smem4) + warp * L::TOTAL_F;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + L::ST_F);
@@ -650,8 +698,8 @@ __global__ void __launch_bounds__(K::WARPS * 32)
             stage_fill<K, K::D_IN>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_x, e, s, c0,
                                    pol_stream, pol_keep, lane);
         }
-        for (int b0 = 0; b0 < n && ok_all; b0 += K::CHUNK) {
-            const int nb = min(K::CHUNK, n - b0);
+        for (int b0 = 0; b0 < n && ok_all; b0 += CH) {
+            const int nb = min(CH, n - b0);
             if (lane >= b0 && lane < b0 + nb) {
                 float ux, uy, uz, il;
                 const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
@@ -668,12 +716,15 @@ __global__ void __launch_bounds__(K::WARPS * 32)
                     ok_all = false;
                     break;
                 }
-                // inactive lanes (past C in a ragged tile) compute on zeros; the
-                // predicate also keeps the compiler from hoisting every row load
+                // Lanes past C in a ragged tile read the tensor map's zero fill, so
+                // the reads need no predicate for correctness; at wide tiles the
+                // predicate keeps ptxas from hoisting every row load (registers).
+                constexpr bool kPred = EQC_FWD_PRED == 2 || (EQC_FWD_PRED == 1 && V >= 4);
+                const bool rd = !kPred || active;
                 float xv[K::D_IN][V], wv[K::NP][V];
 #pragma unroll
                 for (int p = 0; p < K::NP; ++p) {
-                    if (active)
+                    if (rd)
                         lds_vec<V>(wv[p], st + p * K::TILE_C + cl);
                     else
 #pragma unroll
@@ -681,7 +732,7 @@ __global__ void __launch_bounds__(K::WARPS * 32)
                 }
 #pragma unroll
                 for (int d = 0; d < K::D_IN; ++d) {
-                    if (active)
+                    if (rd)
                         lds_vec<V>(xv[d], st + (K::NP + d) * K::TILE_C + cl);
                     else
 #pragma unroll
@@ -735,18 +786,20 @@ __device__ __forceinline__ void warp_sum(float (&v)[G]) {
 // !DET: node = receiver i, resident gy_i, dx scattered with atomic adds.
 // FUSED: the tile covers every channel (T == 1): dr is finished in-kernel.
 template <class K, bool DET, bool FUSED>
-__global__ void __launch_bounds__(K::WARPS * 32)
+__global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
     eqconv_bwd_kernel(const BwdParams prm, const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_g) {
     constexpr int V = K::VEC;
     constexpr int S = K::STAGES;
     constexpr int GG = K::G > 0 ? K::G : 1;
-    constexpr int DL = DET ? K::D_OUT : K::D_IN;     // rows gathered per edge
-    using L = WarpSmem<K, DL, true>;
+    constexpr int DL = BwdShape<K, DET>::DL;         // rows gathered per edge
+    constexpr int CH = BwdShape<K, DET>::CH;
+    constexpr int WARPS = BwdShape<K, DET>::WARPS;
+    using L = typename BwdShape<K, DET>::L;
     constexpr int SF = Stage<K, DL>::FLOATS;
     extern __shared__ __align__(128) float4 smem4[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int node = blockIdx.x * K::WARPS + warp;
+    const int node = blockIdx.x * WARPS + warp;
     if (node >= prm.N) return;
     float* stages = reinterpret_cast<float*>(smem4) + warp * L::TOTAL_F;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + L::ST_F);
@@ -813,8 +866,8 @@ __global__ void __launch_bounds__(K::WARPS * 32)
             stage_fill<K, DL>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e, o, c0, pol_stream,
                               pol_keep, lane);
         }
-        for (int b0 = 0; b0 < n && ok_all; b0 += K::CHUNK) {
-            const int nb = min(K::CHUNK, n - b0);
+        for (int b0 = 0; b0 < n && ok_all; b0 += CH) {
+            const int nb = min(CH, n - b0);
             if (lane >= b0 && lane < b0 + nb) {
                 float ux, uy, uz, il;
                 const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);

@@ -17,7 +17,7 @@ struct FwdParams;
 struct BwdParams;
 
 struct KernelSet {
-    int lin, lsh, lout, vec, tile_c, g;
+    int lin, lsh, lout, vec, mode, tile_c, g;
     // `bands` launches over consecutive ranges of the gathered node index
     cudaError_t (*fwd)(const FwdParams&, int tiles, int bands, cudaStream_t);
     cudaError_t (*bwd)(const BwdParams&, bool det, bool fused, int bands, cudaStream_t);
@@ -40,6 +40,34 @@ const KernelSet* instances_l3_s0(int lout, int vec);
 const KernelSet* instances_l3_s1(int lout, int vec);
 const KernelSet* instances_l3_s2(int lout, int vec);
 const KernelSet* instances_l3_s3(int lout, int vec);
+
+// Instances of the output variants (mode 1: both parities, 2: per-path, 3:
+// both) for one L_in, every L_sh and L_out in 1..3, one channel width each;
+// defined in eqc_inst_m<mode>_l<L_in>.cu.
+#define EQC_DECLARE_MODE(m)                                  \
+    const KernelSet* instances_m##m##_l0(int lsh, int lout); \
+    const KernelSet* instances_m##m##_l1(int lsh, int lout); \
+    const KernelSet* instances_m##m##_l2(int lsh, int lout); \
+    const KernelSet* instances_m##m##_l3(int lsh, int lout);
+EQC_DECLARE_MODE(1)
+EQC_DECLARE_MODE(2)
+EQC_DECLARE_MODE(3)
+#undef EQC_DECLARE_MODE
+
+// Channel width of the output-variant instances: 1 where an l = 3 block makes
+// the unrolled per-edge code large, else 2.
+constexpr int mode_vec(int lin, int lsh, int lout) { return (lin == 3 || lsh == 3 || lout == 3) ? 1 : 2; }
+
+inline const KernelSet* find_mode_instance(int lin, int lsh, int lout, int mode) {
+    using Fn = const KernelSet* (*)(int, int);
+    static const Fn fns[3][4] = {
+        {instances_m1_l0, instances_m1_l1, instances_m1_l2, instances_m1_l3},
+        {instances_m2_l0, instances_m2_l1, instances_m2_l2, instances_m2_l3},
+        {instances_m3_l0, instances_m3_l1, instances_m3_l2, instances_m3_l3},
+    };
+    if (mode < 1 || mode > 3 || lin < 0 || lin > 3) return nullptr;
+    return fns[mode - 1][lin](lsh, lout);
+}
 
 inline const KernelSet* find_instance(int lin, int lsh, int lout, int vec) {
     using Fn = const KernelSet* (*)(int, int);

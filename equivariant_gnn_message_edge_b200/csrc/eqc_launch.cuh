@@ -31,7 +31,8 @@ struct Launch {
         FwdParams prm = prm_in;
         auto kern = eqconv_fwd_kernel<K>;
         static bool done[64] = {};
-        constexpr int smem = K::WARPS * WarpSmem<K, K::D_IN, false>::BYTES;
+        constexpr int W = FwdShape<K>::WARPS;
+        constexpr int smem = W * FwdShape<K>::L::BYTES;
         cudaError_t err = ensure_smem(kern, smem, done);
         if (err != cudaSuccess) return err;
         // with no edges the weight map is never read: give it a valid stand-in
@@ -41,12 +42,12 @@ struct Launch {
                              K::TILE_C) ||
             !encode_rows_map(&tx, prm.x, (uint64_t)prm.N, K::D_IN, prm.C, K::TILE_C))
             return cudaErrorInvalidValue;
-        dim3 grid((prm.N + K::WARPS - 1) / K::WARPS, tiles);
+        dim3 grid((prm.N + W - 1) / W, tiles);
         for (int b = 0; b < bands; ++b) {
             prm.band_lo = (int)((int64_t)prm.N * b / bands);
             prm.band_hi = (int)((int64_t)prm.N * (b + 1) / bands);
             prm.accumulate = b > 0;
-            kern<<<grid, K::WARPS * 32, smem, st>>>(prm, tw, tx);
+            kern<<<grid, W * 32, smem, st>>>(prm, tw, tx);
             count_launch();
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
         }
@@ -57,7 +58,8 @@ struct Launch {
         BwdParams prm = prm_in;
         auto kern = eqconv_bwd_kernel<K, DET, FUSED>;
         static bool done[64] = {};
-        constexpr int smem = K::WARPS * WarpSmem<K, DET ? K::D_OUT : K::D_IN, true>::BYTES;
+        constexpr int W = BwdShape<K, DET>::WARPS;
+        constexpr int smem = W * BwdShape<K, DET>::L::BYTES;
         cudaError_t err = ensure_smem(kern, smem, done);
         if (err != cudaSuccess) return err;
         CUtensorMap tw, tg;
@@ -65,12 +67,12 @@ struct Launch {
         if (!encode_rows_map(&tw, prm.w, (uint64_t)prm.E, K::NP, prm.C, K::TILE_C) ||
             !encode_rows_map(&tg, g, (uint64_t)prm.N, DET ? K::D_OUT : K::D_IN, prm.C, K::TILE_C))
             return cudaErrorInvalidValue;
-        dim3 grid((prm.N + K::WARPS - 1) / K::WARPS, prm.T);
+        dim3 grid((prm.N + W - 1) / W, prm.T);
         for (int b = 0; b < bands; ++b) {
             prm.band_lo = (int)((int64_t)prm.N * b / bands);
             prm.band_hi = (int)((int64_t)prm.N * (b + 1) / bands);
             prm.accumulate = b > 0;
-            kern<<<grid, K::WARPS * 32, smem, st>>>(prm, tw, tg);
+            kern<<<grid, W * 32, smem, st>>>(prm, tw, tg);
             count_launch();
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
         }
@@ -81,7 +83,7 @@ struct Launch {
         return fused ? bwd_one<false, true>(prm, bands, st) : bwd_one<false, false>(prm, bands, st);
     }
     static constexpr KernelSet make() {
-        return KernelSet{K::LIN, K::LSH, K::LOUT, K::VEC, K::TILE_C, K::G, &fwd, &bwd};
+        return KernelSet{K::LIN, K::LSH, K::LOUT, K::VEC, K::MODE, K::TILE_C, K::G, &fwd, &bwd};
     }
 };
 

@@ -2,13 +2,16 @@
 //
 // FlashCart (arXiv 2610.06409), App. B: an admissible path (l1, l2, l3)
 // satisfies the triangle inequalities and its equivariant bilinear coupling is
-// unique up to normalisation; the convolution uses natural-parity outputs.
+// unique up to normalisation.  Natural-parity outputs take the paths with an
+// even l1 + l2 + l3; both-parity outputs also take the odd ones (the
+// antisymmetric couplings, e.g. 1 x 1 -> 1 is the cross product).
 // The coefficients are fixed here as:
 //   * complex CG <l1 m1 l2 m2 | l3 m3> by the Racah formula (Condon-Shortley);
 //   * real basis U^l (rows real m, columns complex mu):
 //       m > 0: ((-1)^m |m> + |-m>)/sqrt2,  m = 0: |0>,  m < 0: i(|m> - (-1)^m |-m>)/sqrt2,
 //     C[m1,m2,m3] = sum U3[m3,mu3] conj(U1[m1,mu1]) conj(U2[m2,mu2]) <..|..>
-//     (real for natural-parity paths);
+//     (real when l1 + l2 + l3 is even, imaginary when it is odd: the
+//     coupling is its real or its imaginary part);
 //   * sign: the first entry with |c| > 1e-9 in (m1, m2, m3) order is positive;
 //   * orthonormal: sum_{m1,m2} C[m1,m2,m3] C[m1,m2,m3'] = delta.
 // Everything is constexpr, so kernels read the coefficients as immediates and
@@ -89,12 +92,13 @@ constexpr cplx umat(int m, int mu) {
 
 struct CG3 {
     double v[2 * kMaxL + 1][2 * kMaxL + 1][2 * kMaxL + 1];  // [m1+l1][m2+l2][m3+l3]
-    double max_imag;
+    double max_dropped;   // largest |part| that must vanish (imag if even, real if odd)
 };
 
 constexpr CG3 make_real_cg(int l1, int l2, int l3) {
     CG3 t{};
-    t.max_imag = 0.0;
+    t.max_dropped = 0.0;
+    const bool odd = ((l1 + l2 + l3) & 1) != 0;
     for (int m1 = -l1; m1 <= l1; ++m1)
         for (int m2 = -l2; m2 <= l2; ++m2)
             for (int m3 = -l3; m3 <= l3; ++m3) {
@@ -112,9 +116,10 @@ constexpr CG3 make_real_cg(int l1, int l2, int l3) {
                             acc.re += u.re * c;
                             acc.im += u.im * c;
                         }
-                const double ai = acc.im < 0 ? -acc.im : acc.im;
-                if (ai > t.max_imag) t.max_imag = ai;
-                t.v[m1 + l1][m2 + l2][m3 + l3] = acc.re;
+                const double drop = odd ? acc.re : acc.im;
+                const double ad = drop < 0 ? -drop : drop;
+                if (ad > t.max_dropped) t.max_dropped = ad;
+                t.v[m1 + l1][m2 + l2][m3 + l3] = odd ? acc.im : acc.re;
             }
     // clean rounding residue so that zero entries are exactly zero
     for (int a = 0; a < 2 * l1 + 1; ++a)
@@ -141,28 +146,56 @@ constexpr CG3 make_real_cg(int l1, int l2, int l3) {
 template <int L1, int L2, int L3>
 struct RealCG {
     static constexpr CG3 t = make_real_cg(L1, L2, L3);
-    static_assert(t.max_imag < 1e-12, "natural-parity coupling must be real");
+    static_assert(t.max_dropped < 1e-12, "coupling must be purely real or purely imaginary");
 };
 
-// Natural-parity paths for irreps 0..LIN (in), SH degrees 0..LSH, 0..LOUT (out),
-// ordered by (l1, l2, l3).
+// Output variants (bits of the plan's mode):
+//   kModeAllParity - outputs of both parities for every l3 >= 1, laid out
+//                    0e, 1o, 1e, 2e, 2o, 3o, 3e (natural parity first; 0o has
+//                    no path from natural-parity inputs), and the paths with
+//                    odd l1 + l2 + l3 that reach the second block of each l3;
+//   kModePerPath   - every path writes its own output block, in path order
+//                    (no summation over paths that share an output irrep).
+constexpr int kModeAllParity = 1;
+constexpr int kModePerPath = 2;
+
+// Row offset of output irrep (l, natural or not) in the summed layouts.
+constexpr int out_row(int l, bool natural, int mode) {
+    if (!(mode & kModeAllParity)) return l * l;
+    if (l == 0) return 0;
+    return natural ? 2 * l * l - 1 : 2 * l * l + 2 * l;
+}
+
+// Paths for natural-parity inputs 0..LIN, SH degrees 0..LSH and outputs of
+// degree 0..LOUT, ordered by (l1, l2, l3); o3 is the path's output row and
+// dout the row count of the output layout.
 struct PathList {
-    int n;
-    int l1[kMaxPaths], l2[kMaxPaths], l3[kMaxPaths];
+    int n, dout;
+    int l1[kMaxPaths], l2[kMaxPaths], l3[kMaxPaths], o3[kMaxPaths];
 };
 
-constexpr PathList make_paths(int LIN, int LSH, int LOUT) {
+constexpr PathList make_paths(int LIN, int LSH, int LOUT, int MODE = 0) {
     PathList P{};
     P.n = 0;
+    int row = 0;
     for (int a = 0; a <= LIN; ++a)
         for (int b = 0; b <= LSH; ++b)
-            for (int c = 0; c <= LOUT; ++c)
-                if (c >= iabs(a - b) && c <= a + b && ((a + b + c) & 1) == 0) {
-                    P.l1[P.n] = a;
-                    P.l2[P.n] = b;
-                    P.l3[P.n] = c;
-                    ++P.n;
-                }
+            for (int c = 0; c <= LOUT; ++c) {
+                const bool natural = ((a + b + c) & 1) == 0;
+                if (c < iabs(a - b) || c > a + b) continue;
+                if (!natural && !(MODE & kModeAllParity)) continue;
+                P.l1[P.n] = a;
+                P.l2[P.n] = b;
+                P.l3[P.n] = c;
+                P.o3[P.n] = (MODE & kModePerPath) ? row : out_row(c, natural, MODE);
+                row += 2 * c + 1;
+                ++P.n;
+            }
+    if (MODE & kModePerPath)
+        P.dout = row;
+    else
+        P.dout = (MODE & kModeAllParity) ? (LOUT == 0 ? 1 : 2 * (LOUT + 1) * (LOUT + 1) - 1)
+                                         : (LOUT + 1) * (LOUT + 1);
     return P;
 }
 

@@ -43,6 +43,8 @@ class Workload:
     mean_degree: float = 45.0
     box: float = 10.0
     cutoff: float = 3.5
+    all_parity: bool = False   # outputs of both parities (irreps_out a both-parity prefix)
+    per_path: bool = False     # one output block per path (no summation over paths)
 
 
 def _natural(L: int) -> str:
@@ -54,6 +56,14 @@ WORKLOADS = {
     "lmax2": Workload("lmax2", 32768, 128, _natural(2), 2, _natural(2), "poisson"),
     "lmax3": Workload("lmax3", 16384, 128, _natural(3), 3, _natural(3), "poisson"),
 }
+# output variants of the lmax=2 / lmax=3 graphs: per-path blocks (MACE's
+# "mid" irreps) and both-parity outputs
+WORKLOADS["lmax2_perpath"] = Workload("lmax2_perpath", 32768, 128, _natural(2), 2, _natural(2), "poisson",
+                                      per_path=True)
+WORKLOADS["lmax2_both"] = Workload("lmax2_both", 32768, 128, _natural(2), 2, "0e+1o+1e+2e+2o", "poisson",
+                                   all_parity=True)
+WORKLOADS["lmax3_perpath"] = Workload("lmax3_perpath", 16384, 128, _natural(3), 3, _natural(3), "poisson",
+                                      per_path=True)
 for _C in (64, 128, 256, 512, 1024):
     WORKLOADS[f"sweepC{_C}"] = Workload(f"sweepC{_C}", (1 << 22) // _C, _C, _natural(2), 2,
                                         _natural(2), "poisson")
@@ -62,6 +72,17 @@ for _C in (64, 128, 256, 512, 1024):
 def natural_irreps(L: int) -> str:
     """'0e+1o+...' up to L (natural parity)."""
     return _natural(L)
+
+
+def both_parity_irreps(L: int) -> str:
+    """'0e+1o+1e+2e+2o+...' up to L: for every l >= 1 the natural-parity irrep
+    and then the other one (0o is left out: no path from natural-parity inputs
+    reaches it)."""
+    names = ["0e"]
+    for l in range(1, L + 1):
+        nat = "e" if l % 2 == 0 else "o"
+        names += [f"{l}{nat}", f"{l}{'o' if nat == 'e' else 'e'}"]
+    return "+".join(names)
 
 
 def poisson_graph(N: int, mean_degree: float, seed: int = SEED_GRAPH):

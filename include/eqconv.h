@@ -96,6 +96,41 @@ typedef struct eqconv_graph_s {
 EQCONV_API int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh,
                        const char* irreps_out, int C);
 
+/* Output variants (bits of out_mode in eqconv_plan_create_ex).
+ * FlashCart (arXiv 2610.06409), App. B: a path may also join irreps whose
+ * parities multiply to the opposite of (-1)^l3 (odd l1 + l2 + l3: the
+ * antisymmetric couplings, such as 1 x 1 -> 1, the cross product); App. D:
+ * the channel-diagonal product may keep every path's output or sum the paths
+ * that land on the same irrep.
+ *   EQCONV_OUT_ALL_PARITY: outputs of both parities.  irreps_out must then be
+ *     the both-parity prefix "0e+1o+1e+2e+2o+3o+3e" up to L_out (for each
+ *     l >= 1 the natural-parity irrep first; 0o is absent: no path from
+ *     natural-parity inputs reaches it), D_out = 2 (L_out+1)^2 - 1, and the
+ *     odd paths feed the second block of each l.  Their coupling is the
+ *     imaginary part of the real-basis CG sum (eqconv_cg_table).
+ *   EQCONV_OUT_PER_PATH: no summation over paths.  Every path p writes its
+ *     own block of 2 l3 + 1 rows, in path order, starting at row
+ *     eqconv_plan_path_rows()[p]; D_out = sum over paths of (2 l3 + 1) (the
+ *     "mid" irreps that MACE feeds to its next linear layer).  irreps_out
+ *     still names the allowed output irreps as a natural-parity prefix (or
+ *     with EQCONV_OUT_ALL_PARITY, a both-parity prefix) and only selects
+ *     paths.  gy has the same per-path layout; dx, dw and dr are as usual.
+ * Both bits may be combined.  The variants exist for L_sh and L_out in 1..3
+ * (L_in 0..3) with one channel width per plan (1 where an l = 3 block is
+ * present, else 2); other combinations return EQCONV_ERR_UNSUPPORTED. */
+#define EQCONV_OUT_ALL_PARITY 1u
+#define EQCONV_OUT_PER_PATH 2u
+
+/* eqconv_plan_create with an output variant (out_mode: 0 or the bits above;
+ * 0 is eqconv_plan_create). */
+EQCONV_API int eqconv_plan_create_ex(eqconv_plan_t* out, const char* irreps_in, int L_sh,
+                                     const char* irreps_out, int C, unsigned out_mode);
+
+/* First output row of every path (P ints): l3^2 for natural-parity summed
+ * outputs, the block of the path's (l3, parity) for EQCONV_OUT_ALL_PARITY,
+ * the path's own block for EQCONV_OUT_PER_PATH. */
+EQCONV_API int eqconv_plan_path_rows(eqconv_plan_t plan, int* out_rows);
+
 /* Channel vector width of the forward / backward kernels (1, 2 or 4 channels
  * per lane, i.e. channel tiles of 32, 64 or 128 channels; width 1 exists only
  * for plans with an l = 3 block and falls back to 2 otherwise).  Defaults
@@ -130,10 +165,19 @@ EQCONV_API int eqconv_plan_info(eqconv_plan_t plan, int* P, int* D_in, int* D_sh
 EQCONV_API int eqconv_enumerate_paths(const char* irreps_in, int L_sh, const char* irreps_out,
                                       int* P, int* paths_l1l2l3, int max_paths);
 
+/* Host only.  eqconv_enumerate_paths for an output variant (out_mode as in
+ * eqconv_plan_create_ex): also gives every path's first output row
+ * (out_rows, room for max_paths ints, may be NULL) and the output row count
+ * (*D_out, may be NULL).  Does not check that kernels exist for the variant. */
+EQCONV_API int eqconv_enumerate_paths_ex(const char* irreps_in, int L_sh, const char* irreps_out,
+                                         unsigned out_mode, int* P, int* paths_l1l2l3, int* out_rows,
+                                         int* D_out, int max_paths);
+
 /* Host only, no device needed.  The real-basis CG tensor the kernels use for
- * the natural-parity path (l1, l2, l3), fp64 row-major [2l1+1][2l2+1][2l3+1];
- * out_len must be at least that size.  EQCONV_ERR_UNSUPPORTED for odd or
- * inadmissible triples or l > 3. */
+ * the path (l1, l2, l3), fp64 row-major [2l1+1][2l2+1][2l3+1]: the real part
+ * of the basis-change sum for even l1 + l2 + l3, its imaginary part for odd
+ * (both-parity outputs).  out_len must be at least that size.
+ * EQCONV_ERR_UNSUPPORTED for triples outside the triangle rule or l > 3. */
 EQCONV_API int eqconv_cg_table(int l1, int l2, int l3, double* out, int out_len);
 
 /* Device workspace bytes needed by eqconv_graph_build for (N, E). */

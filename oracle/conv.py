@@ -16,6 +16,12 @@ energy gradients; App. C/D: gradients for both inputs and the weight):
     gY[e,l2,m2]   = sum_c sum_{p with l2} w[e,p,c] sum_{m1,m3} C_p x gy
     dr[e]         = (dY/dr_e)^T gY[e]
 
+Per-path retention (FlashCart App. D: the channel-diagonal product may keep
+each path's output or sum the paths that land on the same irrep): with
+``per_path=True`` every path writes its own output block, in path order, so
+y[i, o3(p)+m3, c] holds path p alone and D_out = sum_p (2 l3 + 1); summing
+the blocks of each output irrep gives the summed layout back.
+
 Readings where the pages are silent: no 1/sqrt(P), fan-in or 1/avg-degree
 factor inside the op (the weights carry all scaling); zero-length edges have
 Y_0 = 1, Y_{l>0} = 0 and dr = 0; isolated receivers give y = 0.
@@ -46,17 +52,30 @@ class Problem:
     L_sh: int
     irreps_out: str
     C: int
+    per_path: bool = False
     paths: list = field(init=False)
     D_in: int = field(init=False)
     D_sh: int = field(init=False)
     D_out: int = field(init=False)
+    layout_out: str = field(init=False)
 
     def __post_init__(self):
         ins, outs = parse_irreps(self.irreps_in), parse_irreps(self.irreps_out)
         self.paths = enumerate_paths(ins, self.L_sh, outs)
         self.D_in = block_offsets(ins)[1]
-        self.D_out = block_offsets(outs)[1]
         self.D_sh = (self.L_sh + 1) ** 2
+        if self.per_path:
+            # one block per path, in path order
+            off, names = 0, []
+            for q in self.paths:
+                q["off3"] = off
+                off += 2 * q["l3"] + 1
+                names.append(f"{q['l3']}{'e' if outs[q['i3']][1] > 0 else 'o'}")
+            self.D_out = off
+            self.layout_out = "+".join(names)
+        else:
+            self.D_out = block_offsets(outs)[1]
+            self.layout_out = self.irreps_out
 
     @property
     def P(self) -> int:

@@ -21,8 +21,9 @@ def to_dev(a, dtype=None):
     return t.cuda()
 
 
-def run_gpu(ins, L_sh, outs, C, N, senders, receivers, r, x, w, gy=None, det=True, vec=None):
-    conv = EqConv(ins, L_sh, outs, C)
+def run_gpu(ins, L_sh, outs, C, N, senders, receivers, r, x, w, gy=None, det=True, vec=None, all_parity=False,
+            per_path=False):
+    conv = EqConv(ins, L_sh, outs, C, all_parity=all_parity, per_path=per_path)
     if vec is not None:
         conv.set_vec(*vec)
     s_d, r_d = to_dev(senders), to_dev(receivers)
@@ -38,6 +39,7 @@ def run_gpu(ins, L_sh, outs, C, N, senders, receivers, r, x, w, gy=None, det=Tru
     status = conv_status(conv)
     res = {k: v.cpu().numpy() for k, v in out.items()}
     res["status"] = status
+    res["D_out"], res["path_rows"], res["paths"] = conv.D_out, conv.path_rows, conv.paths
     return res
 
 
@@ -46,8 +48,8 @@ def conv_status(conv):
     return B.eqconv_get_device_error(conv.plan)
 
 
-def oracle_full(ins, L_sh, outs, C, N, senders, receivers, r, x, w, gy=None):
-    prob = oconv.Problem(ins, L_sh, outs, C)
+def oracle_full(ins, L_sh, outs, C, N, senders, receivers, r, x, w, gy=None, per_path=False):
+    prob = oconv.Problem(ins, L_sh, outs, C, per_path=per_path)
     return oconv.full(prob, N, senders, receivers, r, x, w, gy)
 
 

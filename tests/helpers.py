@@ -51,11 +51,13 @@ def within_tol(got, ref, rel=1e-5, abs_=1e-6):
     return err <= bound, err, bound
 
 
-def small_problem(N=12, E=40, C=8, L_in=2, L_sh=2, L_out=2, seed=0, irreps_in=None, irreps_out=None):
+def small_problem(N=12, E=40, C=8, L_in=2, L_sh=2, L_out=2, seed=0, irreps_in=None, irreps_out=None,
+                  per_path=False):
     from oracle.conv import Problem
     from equivariant_gnn_message_edge_b200.workloads import natural_irreps
     rng = np.random.default_rng(seed)
-    prob = Problem(irreps_in or natural_irreps(L_in), L_sh, irreps_out or natural_irreps(L_out), C)
+    prob = Problem(irreps_in or natural_irreps(L_in), L_sh, irreps_out or natural_irreps(L_out), C,
+                   per_path=per_path)
     senders = rng.integers(0, N, E).astype(np.int32)
     receivers = rng.integers(0, N, E).astype(np.int32)
     r = rng.standard_normal((E, 3)).astype(np.float32) * 2

@@ -56,18 +56,47 @@ def test_only_the_abi_is_exported():
 
 
 @pytest.mark.parametrize("l1,l2,l3", [(a, b, c) for a in range(4) for b in range(4) for c in range(4)
-                                      if abs(a - b) <= c <= a + b and (a + b + c) % 2 == 0])
+                                      if abs(a - b) <= c <= a + b])
 def test_library_cg_matches_oracle(l1, l2, l3):
     """The library's compile-time Racah evaluation vs the oracle's exact
-    rationals: same real basis, phase and sign convention."""
+    rationals: same real basis, phase and sign convention; odd l1 + l2 + l3
+    (both-parity outputs) included."""
     assert np.max(np.abs(B.eqconv_cg_table(l1, l2, l3) - real_cg(l1, l2, l3))) < 1e-12
 
 
-def test_library_rejects_odd_or_inadmissible_cg():
-    for t in [(1, 1, 1), (1, 1, 3), (4, 0, 4)]:
+def test_library_rejects_inadmissible_cg():
+    for t in [(1, 1, 3), (4, 0, 4), (0, 2, 1)]:
         with pytest.raises(B.EqconvError) as e:
             B.eqconv_cg_table(*t)
         assert e.value.status == B.EQCONV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("all_parity", [False, True])
+@pytest.mark.parametrize("per_path", [False, True])
+@pytest.mark.parametrize("lin,lsh,lout", [(a, b, c) for a in range(4) for b in range(4) for c in range(4)])
+def test_library_variant_layouts_match_oracle(lin, lsh, lout, all_parity, per_path):
+    """Both-parity and per-path layouts: the library's paths, the first
+    output row of each path and D_out equal the oracle's."""
+    from equivariant_gnn_message_edge_b200.workloads import both_parity_irreps
+    from oracle.conv import Problem
+    ins = natural_irreps(lin)
+    outs = both_parity_irreps(lout) if all_parity else natural_irreps(lout)
+    mode = (B.EQCONV_OUT_ALL_PARITY if all_parity else 0) | (B.EQCONV_OUT_PER_PATH if per_path else 0)
+    prob = Problem(ins, lsh, outs, 4, per_path=per_path)
+    got = B.eqconv_enumerate_paths_ex(ins, lsh, outs, mode)
+    assert got["paths"] == [(q["l1"], q["l2"], q["l3"]) for q in prob.paths]
+    assert got["rows"] == [q["off3"] for q in prob.paths]
+    assert got["D_out"] == prob.D_out
+
+
+def test_variant_plans_validate_before_device_work():
+    cases = [("0e+1o", 1, "0e+1o", B.EQCONV_OUT_ALL_PARITY, B.EQCONV_ERR_UNSUPPORTED),  # natural string
+             ("0e+1o", 1, "0e+1o+1e", 0, B.EQCONV_ERR_UNSUPPORTED),                     # both-parity string
+             ("0e+1o", 1, "0e+1o", 4, B.EQCONV_ERR_INVALID_ARG)]                        # unknown bit
+    for ins, lsh, outs, mode, status in cases:
+        with pytest.raises(B.EqconvError) as e:
+            B.eqconv_plan_create_ex(ins, lsh, outs, 8, mode)
+        assert e.value.status == status
 
 
 @pytest.mark.parametrize("lin,lsh,lout", [(a, b, c) for a in range(4) for b in range(4) for c in range(4)])
