@@ -103,3 +103,103 @@ def sh_grad(r: np.ndarray, L: int) -> np.ndarray:
     g = g / safe[..., None, None]
     g[zero] = 0.0
     return g
+
+
+# --------------------------------------------------------------------------
+# Second derivatives (double backward of the convolution)
+# --------------------------------------------------------------------------
+# An independent construction: Y_lm(r) = P_lm(r) / |r|^l with P_lm the
+# homogeneous degree-l polynomial that equals Y_lm on the unit sphere,
+#     P_lm = N_lm sum_k q_k z^k (x^2+y^2+z^2)^((l-|m|-k)/2) A_m(x, y),
+# q_k the coefficients of d^|m| P_l / dz^|m| (only k = l-|m| mod 2 occur) and
+# A_m = Re or Im of (x + i y)^|m|.  Polynomials are dicts {(i, j, k): c}.
+
+def _pmul(p, q):
+    out = {}
+    for (a, b, c), u in p.items():
+        for (d, e, f), v in q.items():
+            key = (a + d, b + e, c + f)
+            out[key] = out.get(key, 0.0) + u * v
+    return out
+
+
+def _padd(p, q, s=1.0):
+    out = dict(p)
+    for k, v in q.items():
+        out[k] = out.get(k, 0.0) + s * v
+    return out
+
+
+def _pderiv(p, var):
+    out = {}
+    for key, c in p.items():
+        if key[var] == 0:
+            continue
+        k2 = list(key)
+        k2[var] -= 1
+        out[tuple(k2)] = out.get(tuple(k2), 0.0) + c * key[var]
+    return out
+
+
+def _peval(p, r):
+    x, y, z = r[..., 0], r[..., 1], r[..., 2]
+    out = np.zeros(r.shape[:-1])
+    for (a, b, c), v in p.items():
+        out = out + v * x ** a * y ** b * z ** c
+    return out
+
+
+def _homogeneous(l: int, m: int) -> dict:
+    am = abs(m)
+    Q = nppoly.polyder(_legendre_power_coeffs(l), am) if am <= l else np.zeros(1)
+    rho2 = {(2, 0, 0): 1.0, (0, 2, 0): 1.0, (0, 0, 2): 1.0}
+    # (x + i y)^am expanded: sum_j binom(am, j) x^(am-j) (i y)^j
+    from math import comb
+    A = {}
+    for j in range(am + 1):
+        ij = 1j ** j
+        part = ij.real if m >= 0 else ij.imag
+        if abs(part) > 0:
+            A[(am - j, j, 0)] = A.get((am - j, j, 0), 0.0) + comb(am, j) * part
+    P = {}
+    for k, qk in enumerate(Q):
+        if qk == 0.0:
+            continue
+        e = l - am - k
+        assert e % 2 == 0 and e >= 0
+        term = {(0, 0, k): qk}
+        for _ in range(e // 2):
+            term = _pmul(term, rho2)
+        P = _padd(P, term)
+    P = _pmul(P, A) if A else {}
+    return {key: _norm(l, am) * v for key, v in P.items()}
+
+
+def sh_hessian(r: np.ndarray, L: int) -> np.ndarray:
+    """d^2 Y / dr dr^T, shape [..., (L+1)^2, 3, 3] (fp64); zero-length edges
+    give 0.  Built from the homogeneous polynomials above (quotient rule on
+    P / |r|^l), not from ``sh_grad``."""
+    r = np.asarray(r, dtype=np.float64)
+    n = np.linalg.norm(r, axis=-1)
+    zero = n < ZERO_LEN
+    rs = np.where(zero[..., None], 1.0, r)
+    ns = np.where(zero, 1.0, n)
+    H = np.zeros(r.shape[:-1] + ((L + 1) ** 2, 3, 3))
+    eye = np.eye(3)
+    for l in range(1, L + 1):
+        s = ns ** (-l)
+        ds = -l * ns[..., None] ** (-l - 2) * rs                                    # grad |r|^-l
+        hs = (-l * ns[..., None, None] ** (-l - 2) * eye +
+              l * (l + 2) * ns[..., None, None] ** (-l - 4) * rs[..., :, None] * rs[..., None, :])
+        for m in range(-l, l + 1):
+            P = _homogeneous(l, m)
+            g = [_pderiv(P, a) for a in range(3)]
+            Pv = _peval(P, rs)
+            gv = np.stack([_peval(g[a], rs) for a in range(3)], axis=-1)
+            hv = np.stack([np.stack([_peval(_pderiv(g[a], b), rs) for b in range(3)], axis=-1)
+                           for a in range(3)], axis=-2)
+            k = l * l + m + l
+            H[..., k, :, :] = (s[..., None, None] * hv + gv[..., :, None] * ds[..., None, :] +
+                               ds[..., :, None] * gv[..., None, :] + Pv[..., None, None] * hs)
+    H[zero] = 0.0
+    return H

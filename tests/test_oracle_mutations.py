@@ -86,3 +86,45 @@ def test_missing_radial_projection_fails_finite_differences(monkeypatch):
     h = 1e-6
     fd_radial = (shmod.sh(r + h * u, 2) - shmod.sh(r - h * u, 2)) / (2 * h)
     assert np.max(np.abs(fd_radial)) < 1e-8
+
+
+def _dbl_fd_failures(dbl_fn):
+    """Names of the inputs whose central-difference pin (test_oracle_dbl.py)
+    a double-backward implementation fails."""
+    from tests.test_oracle_dbl import CASES, _S, _setup
+    prob, s, rcv, r, x, w, gy, a, b, q = _setup(CASES[1], seed=3)
+    grads = dbl_fn(prob, 8, s, rcv, r, x, w, gy, a, b, q)
+    rng = np.random.default_rng(11)
+    h, fails, args = 1e-6, [], dict(r=r, x=x, w=w, gy=gy)
+    for name, g in zip(("x", "w", "gy", "r"), grads):
+        d = rng.standard_normal(args[name].shape)
+        p, m = dict(args), dict(args)
+        p[name] = args[name] + h * d
+        m[name] = args[name] - h * d
+        fd = (_S(prob, 8, s, rcv, p["r"], p["x"], p["w"], p["gy"], a, b, q)[0] -
+              _S(prob, 8, s, rcv, m["r"], m["x"], m["w"], m["gy"], a, b, q)[0]) / (2 * h)
+        an = float((g * d).sum())
+        if abs(fd - an) >= 1e-6 * max(1.0, abs(an)):
+            fails.append(name)
+    return fails
+
+
+def test_double_backward_mistakes_fail_the_difference_pins():
+    """A dropped Hessian term, the wrong cotangent in gY, a dropped rho term
+    and a flipped sign each fail the central-difference pin of one input."""
+    import inspect
+    from oracle import dbl
+    src = inspect.getsource(dbl)
+    assert _dbl_fd_failures(dbl.double_backward_bruteforce) == []
+    mistakes = {
+        "r": ('+ np.einsum("ekij,ek,ej->ei", H, gY1, q)', ""),
+        "r ": ('np.einsum("ebc,ec->eb", Gx, b[:, p])', 'np.einsum("ebc,ec->eb", Ga, b[:, p])'),
+        "gy": ("+ wp * msg(Rb, xb)", ""),
+        "x": ("g_x_e[:, o1:o1 + d1, :] += bp * uY + wp * uR", "g_x_e[:, o1:o1 + d1, :] += bp * uY - wp * uR"),
+    }
+    for expect, (good, bad) in mistakes.items():
+        assert good in src
+        ns = {}
+        code = src.replace(good, bad).replace("from .conv import", "from oracle.conv import")
+        exec(compile(code.replace("from .sh import", "from oracle.sh import"), "planted", "exec"), ns)
+        assert expect.strip() in _dbl_fd_failures(ns["double_backward_bruteforce"])
