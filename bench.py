@@ -61,6 +61,17 @@ def byte_counts(N, E, C, D_in, D_out, P):
     return dict(fwd=fwd, bwd=bwd, graph=graph, step=step, h2d=h2d, d2h=d2h, kernels=graph + fwd + bwd)
 
 
+def dbl_bytes(N, E, C, D_in, D_out, P, part_bytes):
+    """Algorithmic bytes of one double backward: receiver pass, sender pass
+    and r epilogue, each kernel's inputs and outputs counted once."""
+    t = tensor_bytes(N, E, C, D_in, D_out, P)
+    recv = 2 * t["x"] + 2 * t["r"] + 2 * t["w"] + t["recv_ptr"] + t["recv_perm"] + t["senders"] + t["y"]
+    send = (2 * t["x"] + 2 * t["r"] + 2 * t["w"] + t["gy"] + t["send_ptr"] + t["send_perm"] + t["receivers"] +
+            t["dx"] + t["dw"] + part_bytes)
+    epi = part_bytes + 3 * t["r"]
+    return recv + send + epi
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -297,6 +308,37 @@ def run_native(args, rank, world, local_rank):
     stream.synchronize()
     nd_ms = [a.elapsed_time(b) for a, b in nd_ms[1:]]
 
+    # double backward (VJP of the backward), timed separately (not part of the step)
+    dbl = None
+    dws_n = B.eqconv_double_backward_workspace_bytes(conv.plan, E)
+    if W.all_parity is False and W.per_path is False and not args.no_double_backward:
+        gen = torch.Generator(device=dev).manual_seed(wl.SEED_GY + 1)
+        with torch.cuda.stream(stream):
+            cot_a = torch.randn(ds0.x.shape, generator=gen, device=dev)
+            cot_b = torch.randn(ds0.w.shape, generator=gen, device=dev)
+            cot_q = torch.randn(ds0.rv.shape, generator=gen, device=dev)
+            outs = (torch.empty_like(ds0.x), torch.empty_like(ds0.w), torch.empty_like(ds0.gy),
+                    torch.empty_like(ds0.rv))
+            dws = torch.empty(max(dws_n, 1), dtype=torch.uint8, device=dev)
+        dbl_ev = []
+        for k in range(max(3, args.steps // 2) + 1):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            B.eqconv_double_backward(conv.plan, ds0.g.c, ds0.x, ds0.rv, ds0.w, ds0.gy, cot_a, cot_b, cot_q,
+                                     *outs, dws, dws_n, sh)
+            a1.record(stream)
+            dbl_ev.append((a0, a1))
+        stream.synchronize()
+        assert B.eqconv_get_device_error(conv.plan, sh) == B.EQCONV_OK
+        dbl_ms = [a.elapsed_time(b) for a, b in dbl_ev[1:]]
+        nbytes = dbl_bytes(N, E, C, D_in, D_out, P, dws_n)
+        dbl_med = statistics.median(dbl_ms)
+        dbl = {"ms": round(dbl_med, 4), "gbps": round(nbytes / (dbl_med * 1e-3) / 1e9, 1),
+               "frac_of_measured_hbm": round(nbytes / (dbl_med * 1e-3) / 1e9 / measured_peak()[0], 4),
+               "algorithmic_bytes": nbytes, "launches_per_call": 3,
+               "bytes": "per kernel: receiver pass, sender pass, r epilogue, each tensor once per kernel"}
+        del cot_a, cot_b, cot_q, outs, dws
+
     # End to end through the public API with host buffers (pinned), copies
     # timed: every step uploads its inputs and downloads its results.  Steps
     # are pipelined over two device sets and three streams, so step k's
@@ -396,6 +438,7 @@ def run_native(args, rank, world, local_rank):
                          "achieved": round(bc["fwd"] / (fwd_avg * 1e-3) / 1e9, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(bc["fwd"] / (fwd_avg * 1e-3) / 1e9 / peak, 4), "traffic": traffic.get("fwd"),
                          "algorithmic_bytes": bc["fwd"]},
+        "double_backward": dbl,
         "gpu_launches": int(launches),
         "clocks": clk.summary((w0, w1)),
     }
@@ -529,6 +572,7 @@ def main():
                     help="L2 budget of one gather band in MiB (0: no banding)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-double-backward", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--nodes", type=int, default=None,

@@ -35,6 +35,7 @@ ABI_FUNCTIONS = (
     "eqconv_get_device_error", "eqconv_plan_destroy", "eqconv_status_string", "eqconv_launch_count",
     "eqconv_last_error", "eqconv_graph_build_noalloc", "eqconv_plan_set_gather_budget",
     "eqconv_plan_create_ex", "eqconv_plan_path_rows", "eqconv_enumerate_paths_ex",
+    "eqconv_double_backward_workspace_bytes", "eqconv_double_backward",
 )
 
 
@@ -77,6 +78,8 @@ _SIGS = {
     "eqconv_forward": (_ci, [_vp, _pg, _vp, _vp, _vp, _vp, _cu, _vp]),
     "eqconv_backward_workspace_bytes": (_sz, [_vp, _ci]),
     "eqconv_backward": (_ci, [_vp, _pg, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _cu, _vp]),
+    "eqconv_double_backward_workspace_bytes": (_sz, [_vp, _ci]),
+    "eqconv_double_backward": (_ci, [_vp, _pg] + [_vp] * 12 + [_sz, _vp]),
     "eqconv_spherical_harmonics": (_ci, [_vp, _ci, _vp, _vp, _vp]),
     "eqconv_get_device_error": (_ci, [_vp, _vp, _pi]),
     "eqconv_plan_destroy": (None, [_vp]),
@@ -259,6 +262,19 @@ def eqconv_backward(plan: int, graph: eqconv_graph_t, x, r, w, gy, dx, dw, dr, w
     _check(lib().eqconv_backward(plan, ctypes.byref(graph), _ptr(x, f), _ptr(r, f), _ptr(w, f), _ptr(gy, f),
                                  _ptr(dx, f), _ptr(dw, f), _ptr(dr, f), _ptr(workspace), int(workspace_bytes),
                                  int(flags), _stream(stream)), "eqconv_backward")
+
+
+def eqconv_double_backward_workspace_bytes(plan: int, E: int) -> int:
+    return int(lib().eqconv_double_backward_workspace_bytes(plan, int(E)))
+
+
+def eqconv_double_backward(plan: int, graph: eqconv_graph_t, x, r, w, gy, ga, gb, gq, g_x, g_w, g_gy, g_r,
+                           workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    f = _f32()
+    _check(lib().eqconv_double_backward(plan, ctypes.byref(graph), _ptr(x, f), _ptr(r, f), _ptr(w, f), _ptr(gy, f),
+                                        _ptr(ga, f), _ptr(gb, f), _ptr(gq, f), _ptr(g_x, f), _ptr(g_w, f),
+                                        _ptr(g_gy, f), _ptr(g_r, f), _ptr(workspace), int(workspace_bytes),
+                                        _stream(stream)), "eqconv_double_backward")
 
 
 def eqconv_spherical_harmonics(plan: int, E: int, r, Y, stream=None) -> None:

@@ -94,6 +94,19 @@ class EqConv:
                           B.EQCONV_DETERMINISTIC if deterministic else 0, stream)
         return dx, dw, dr
 
+    def double_backward_raw(self, g: Graph, x, r, w, gy, ga, gb, gq, out=None, workspace=None, stream=None):
+        """Gradient of <ga, dx> + <gb, dw> + <gq, dr> w.r.t. (x, w, gy, r); see
+        include/eqconv.h.  Returns (g_x, g_w, g_gy, g_r)."""
+        if out is None:
+            out = (torch.empty_like(x), torch.empty_like(w), torch.empty_like(gy), torch.empty_like(r))
+        g_x, g_w, g_gy, g_r = out
+        nbytes = B.eqconv_double_backward_workspace_bytes(self.plan, g.E)
+        if nbytes and workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+        B.eqconv_double_backward(self.plan, g.c, x, r, w, gy, ga, gb, gq, g_x, g_w, g_gy, g_r, workspace, nbytes,
+                                 stream)
+        return g_x, g_w, g_gy, g_r
+
     def __call__(self, g: Graph, x, r, w, deterministic=True):
         return _EqConvFn.apply(self, g, deterministic, x, r, w)
 
@@ -109,5 +122,27 @@ class _EqConvFn(torch.autograd.Function):
     @staticmethod
     def backward(ctx, gy):
         x, r, w = ctx.saved_tensors
-        dx, dw, dr = ctx.conv.backward_raw(ctx.g, x, r, w, gy.contiguous(), ctx.det)
+        if torch.is_grad_enabled():
+            # create_graph=True (force training): a differentiable backward
+            dx, dw, dr = _EqConvBwdFn.apply(ctx.conv, ctx.g, ctx.det, x, r, w, gy.contiguous())
+        else:
+            dx, dw, dr = ctx.conv.backward_raw(ctx.g, x, r, w, gy.contiguous(), ctx.det)
         return None, None, None, dx, dr, dw
+
+
+class _EqConvBwdFn(torch.autograd.Function):
+    """The backward as a function of (x, r, w, gy), differentiated by the
+    library's double backward."""
+
+    @staticmethod
+    def forward(ctx, conv: EqConv, g: Graph, deterministic: bool, x, r, w, gy):
+        ctx.conv, ctx.g = conv, g
+        ctx.save_for_backward(x, r, w, gy)
+        return conv.backward_raw(g, x, r, w, gy, deterministic)
+
+    @staticmethod
+    def backward(ctx, ga, gb, gq):
+        x, r, w, gy = ctx.saved_tensors
+        z = lambda t, like: torch.zeros_like(like) if t is None else t.contiguous()
+        g_x, g_w, g_gy, g_r = ctx.conv.double_backward_raw(ctx.g, x, r, w, gy, z(ga, x), z(gb, w), z(gq, r))
+        return None, None, None, g_x, g_r, g_w, g_gy

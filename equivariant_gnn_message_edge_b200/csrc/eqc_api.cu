@@ -21,6 +21,7 @@
 #include <vector>
 
 #include "eqc_conv.cuh"
+#include "eqc_dbl.cuh"
 #include "eqc_dispatch.h"
 #include "eqc_graph.h"
 #include "eqconv.h"
@@ -126,6 +127,7 @@ struct eqconv_plan_s {
     const eqc::KernelSet* fwd_ks;
     const eqc::KernelSet* det_ks;      // deterministic backward
     const eqc::KernelSet* atomic_ks;   // atomic backward
+    const eqc::DblKernelSet* dbl_ks;   // double backward (summed natural-parity outputs only)
 };
 
 namespace {
@@ -302,6 +304,7 @@ int eqconv_plan_create_ex(eqconv_plan_t* out, const char* irreps_in, int L_sh, c
         p->fwd_vec = p->det_vec = p->atomic_vec = eqc::mode_vec(lin, L_sh, lout);
         p->fwd_ks = p->det_ks = p->atomic_ks = eqc::find_mode_instance(lin, L_sh, lout, mode);
     }
+    p->dbl_ks = mode == 0 ? eqc::find_dbl_instance(lin, L_sh, lout) : nullptr;
     if (!p->fwd_ks || !p->det_ks || !p->atomic_ks) {
         delete p;
         return EQCONV_ERR_UNSUPPORTED;
@@ -532,6 +535,58 @@ int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
     if (err != cudaSuccess) return cuda_status(err, det ? "backward (deterministic)" : "backward (atomic)");
     if (!fused) err = eqc::launch_dr_epilogue(plan->lsh, prm.gy_part, T, r, dr, g->E, st);
     return cuda_status(err, "dr epilogue");
+}
+
+size_t eqconv_double_backward_workspace_bytes(eqconv_plan_t plan, int E) {
+    if (!plan || E < 0 || !plan->dbl_ks) return 0;
+    const int T = tiles_for(plan->C, plan->dbl_ks->tile_c);
+    return (size_t)E * (size_t)T * 2u * (size_t)(plan->D_sh - 1) * sizeof(float);
+}
+
+int eqconv_double_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r,
+                           const float* w, const float* gy, const float* ga, const float* gb, const float* gq,
+                           float* g_x, float* g_w, float* g_gy, float* g_r, void* workspace, size_t workspace_bytes,
+                           eqconv_stream_t stream) {
+    if (!plan) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_graph(g);
+    if (rc != EQCONV_OK) return rc;
+    if ((rc = check_device(plan)) != EQCONV_OK) return rc;
+    if (!plan->dbl_ks) return EQCONV_ERR_UNSUPPORTED;
+    if (g->N == 0) return EQCONV_OK;
+    if (!x || !gy || !ga || !g_x || !g_gy) return EQCONV_ERR_INVALID_ARG;
+    if (g->E > 0 && (!r || !w || !gb || !gq || !g_w || !g_r)) return EQCONV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gy) || !aligned16(ga) || !aligned16(g_x) || !aligned16(g_gy) ||
+        !aligned16(w) || !aligned16(gb) || !aligned16(g_w))
+        return EQCONV_ERR_INVALID_ARG;
+    const size_t need = eqconv_double_backward_workspace_bytes(plan, g->E);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return EQCONV_ERR_WORKSPACE;
+    eqc::DblParams prm{};
+    prm.x = x;
+    prm.a = ga;
+    prm.r = r;
+    prm.q = gq;
+    prm.w = w;
+    prm.b = gb;
+    prm.gy = gy;
+    prm.g_x = g_x;
+    prm.g_w = g_w;
+    prm.g_gy = g_gy;
+    prm.g_r = g_r;
+    prm.part = static_cast<float*>(workspace);
+    prm.N = g->N;
+    prm.C = plan->C;
+    prm.T = tiles_for(plan->C, plan->dbl_ks->tile_c);
+    prm.E = g->E;
+    prm.status = plan->d_status;
+    // the receiver pass walks the receiver CSR, the sender pass the sender CSR
+    eqc::DblParams recv = prm, send = prm;
+    recv.ptr = g->recv_ptr;
+    recv.perm = g->recv_perm;
+    recv.other = g->senders;
+    send.ptr = g->send_ptr;
+    send.perm = g->send_perm;
+    send.other = g->receivers;
+    return cuda_status(plan->dbl_ks->run(recv, send, (cudaStream_t)stream), "double backward");
 }
 
 int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y, eqconv_stream_t stream) {

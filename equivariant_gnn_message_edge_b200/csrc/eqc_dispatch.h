@@ -81,6 +81,28 @@ inline const KernelSet* find_instance(int lin, int lsh, int lout, int vec) {
     return fns[lin][lsh](lout, vec);
 }
 
+// Double backward (natural-parity summed outputs): receiver pass, sender pass
+// and r epilogue of one (L_in, L_sh, L_out) at one channel width.
+struct DblParams;
+struct DblKernelSet {
+    int lin, lsh, lout, vec, tile_c, g;
+    // recv: receiver CSR and senders; send: sender CSR and receivers
+    cudaError_t (*run)(const DblParams& recv, const DblParams& send, cudaStream_t);
+};
+
+// Defined in eqc_dbl_l<L_in>.cu.
+const DblKernelSet* dbl_instances_l0(int lsh, int lout);
+const DblKernelSet* dbl_instances_l1(int lsh, int lout);
+const DblKernelSet* dbl_instances_l2(int lsh, int lout);
+const DblKernelSet* dbl_instances_l3(int lsh, int lout);
+
+inline const DblKernelSet* find_dbl_instance(int lin, int lsh, int lout) {
+    using Fn = const DblKernelSet* (*)(int, int);
+    static const Fn fns[4] = {dbl_instances_l0, dbl_instances_l1, dbl_instances_l2, dbl_instances_l3};
+    if (lin < 0 || lin > 3) return nullptr;
+    return fns[lin](lsh, lout);
+}
+
 // Harmonics-only kernels (depend on L_sh only); defined in eqc_api.cu.
 cudaError_t launch_dr_epilogue(int lsh, const float* gy_part, int T, const float* r, float* dr, int E,
                                cudaStream_t st);

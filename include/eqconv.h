@@ -231,6 +231,38 @@ EQCONV_API int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, cons
                     float* dr, void* workspace, size_t workspace_bytes, unsigned flags,
                     eqconv_stream_t stream);
 
+/* Device workspace bytes eqconv_double_backward needs for E edges (the
+ * per-channel-tile partials of two harmonic-gradient vectors, [E][T][2 G]
+ * fp32 with G = (L_sh+1)^2 - 1); 0 for plans without a double backward. */
+EQCONV_API size_t eqconv_double_backward_workspace_bytes(eqconv_plan_t plan, int E);
+
+/* Double backward: the VJP of eqconv_backward, for training on forces
+ * (FlashCart, arXiv 2610.06409, §2 and §3 / App. C: the VJP-of-VJP of a
+ * weighted bilinear product follows from bilinearity; App. D: it sums
+ * receiver contributions to the incoming-gradient derivative).
+ * Given the inputs of eqconv_backward (x, r, w, gy) and cotangents
+ * ga [N][D_in][C] of dx, gb [E][P][C] of dw and gq [E][3] of dr, writes the
+ * gradient of S = <ga, dx> + <gb, dw> + <gq, dr> with respect to every input:
+ *   g_x  [N][D_in][C]  = sum over out-edges of  gb_p A_p(Y)^T gy_i + w_p A_p(rho)^T gy_i
+ *   g_w  [E][P][C]     = ga_s . A_p(Y)^T gy_i + x_s . A_p(rho)^T gy_i
+ *   g_gy [N][D_out][C] = sum over in-edges of  w_p (A_p(Y) ga_s + A_p(rho) x_s) + gb_p A_p(Y) x_s
+ *   g_r  [E][3]        = (dY/dr)^T gYv + H(r; gY1) gq
+ * with rho = (dY/dr) gq, A_p(v) = sum_m2 C_p[., m2, .] v[l2 m2], gYv the
+ * harmonic gradient of (ga, w) plus that of (x, gb), gY1 that of (x, w), and
+ * H the Hessian of the harmonics.  Zero-length edges contribute no rho and
+ * no g_r.  Deterministic (bitwise reproducible): three launches on
+ * `stream` (a receiver pass, a sender pass and a per-edge epilogue), no
+ * atomics.  All outputs are overwritten.
+ *   - Plans made with an output variant (out_mode != 0) return
+ *     EQCONV_ERR_UNSUPPORTED.
+ *   - Pointers as in eqconv_backward (16-byte aligned rows); the workspace
+ *     must hold eqconv_double_backward_workspace_bytes(plan, E) bytes. */
+EQCONV_API int eqconv_double_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
+                                      const float* r, const float* w, const float* gy, const float* ga,
+                                      const float* gb, const float* gq, float* g_x, float* g_w, float* g_gy,
+                                      float* g_r, void* workspace, size_t workspace_bytes,
+                                      eqconv_stream_t stream);
+
 /* The spherical harmonics the kernels use, Y [E][(L_sh+1)^2] (a test hook
  * for the in-kernel harmonics; not on the hot path). */
 EQCONV_API int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y,

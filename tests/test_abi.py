@@ -49,6 +49,23 @@ def test_binding_covers_the_header():
     assert sorted(B.ABI_FUNCTIONS) == declared_functions()
 
 
+def declared_arities():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"EQCONV_API\s+[\w\s\*]+?\b(eqconv_\w+)\s*\(([^)]*)\)", text):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header_arity():
+    """Every ctypes signature has as many arguments as the C declaration (a
+    short list would pass trailing arguments with default conversions)."""
+    ar = declared_arities()
+    for name, (_, args) in B._SIGS.items():
+        assert len(args) == ar[name], (name, len(args), ar[name])
+
+
 def test_only_the_abi_is_exported():
     extra = [s for s in exported_symbols() if not s.startswith("eqconv_") and not s.startswith("_")]
     # the static CUDA runtime may export nothing else of ours

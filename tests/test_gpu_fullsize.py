@@ -79,3 +79,50 @@ def test_fullsize_lmax2_sampled():
 
 def test_fullsize_lmax3_sampled():
     run_case("lmax3")
+
+
+def run_double_backward_case(name, n_sample=64):
+    """Double backward at full size: g_gy on sampled receivers, g_x on
+    sampled senders, g_w and g_r on all their edges, against the oracle run
+    on exactly those edges (which hold every term of the sampled rows)."""
+    from oracle.dbl import double_backward_bruteforce
+    W = wl.WORKLOADS[name]
+    s, rcv, r = wl.make_graph(W)
+    E = len(s)
+    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    x = wl.features(W.N, prob.D_in, W.C, wl.SEED_X)
+    gy = wl.features(W.N, prob.D_out, W.C, wl.SEED_GY)
+    w = wl.weights(E, prob.P, W.C)
+    rng = np.random.default_rng(2024)
+    a = rng.standard_normal((W.N, prob.D_in, W.C), dtype=np.float32)
+    q = rng.standard_normal((E, 3), dtype=np.float32)
+    b = rng.standard_normal((E, prob.P, W.C), dtype=np.float32)
+
+    conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    g = conv.graph(to_dev(s), to_dev(rcv), W.N)
+    out = conv.double_backward_raw(g, to_dev(x), to_dev(r), to_dev(w), to_dev(gy), to_dev(a), to_dev(b), to_dev(q))
+    torch.cuda.synchronize()
+    g_x, g_w, g_gy, g_r = out
+    assert all(torch.isfinite(t).all() for t in out)
+
+    rows = np.sort(rng.choice(W.N, n_sample, replace=False))
+    srows = np.sort(rng.choice(W.N, n_sample, replace=False))
+    rp, rperm = csr(rcv, W.N)
+    sp, sperm = csr(s, W.N)
+    edges = np.unique(np.concatenate([rperm[rp[i]:rp[i + 1]] for i in rows] +
+                                     [sperm[sp[j]:sp[j + 1]] for j in srows])).astype(np.int64)
+    ref_x, ref_w, ref_gy, ref_r = double_backward_bruteforce(prob, W.N, s[edges], rcv[edges], r[edges], x, w[edges],
+                                                             gy, a, b[edges], q[edges])
+    ed = torch.from_numpy(edges).cuda()
+    assert_close("g_gy(sampled)", g_gy[torch.from_numpy(rows).cuda()].cpu().numpy(), ref_gy[rows])
+    assert_close("g_x(sampled)", g_x[torch.from_numpy(srows).cuda()].cpu().numpy(), ref_x[srows])
+    assert_close("g_w(sampled)", g_w[ed].cpu().numpy(), ref_w)
+    assert_close("g_r(sampled)", g_r[ed].cpu().numpy(), ref_r)
+
+
+def test_fullsize_double_backward_lmax2_sampled():
+    run_double_backward_case("lmax2")
+
+
+def test_fullsize_double_backward_lmax3_sampled():
+    run_double_backward_case("lmax3")
