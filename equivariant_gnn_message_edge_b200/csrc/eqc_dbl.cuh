@@ -55,8 +55,15 @@ struct DblParams {
     unsigned* status;
 };
 
+#ifndef EQC_DBL_PREFETCH
+#define EQC_DBL_PREFETCH 1   // load the next edge's rows while the current edge is computed
+#endif
+
 template <class K>
 struct DblShape {
+    // prefetching doubles the row registers: it paid at lmax 2 (17.3 -> 16.7 ms)
+    // and cost at lmax 3 (41.6 -> 46.8 ms), where the per-edge code is larger
+    static constexpr bool PF = EQC_DBL_PREFETCH && K::NA_PAD <= 128;
     static constexpr int CH = K::NA_PAD > 128 ? 4 : 8;        // edges per coupling batch
     static constexpr int WARP_FLOATS = 2 * CH * K::NA_PAD;    // A(Y) and A(rho)
     static constexpr int WARPS = 4;
@@ -238,6 +245,18 @@ __device__ __forceinline__ void dbl_send_edge(const float* AY, const float* AR, 
     });
 }
 
+// Rows of one edge for the receiver pass (weights, weight cotangent, sender
+// features and their cotangent) and for the sender pass (weights, weight
+// cotangent, receiver output gradient), this lane's channels.
+template <class K>
+struct RecvRows {
+    float w[K::NP][K::VEC], b[K::NP][K::VEC], x[K::D_IN][K::VEC], a[K::D_IN][K::VEC];
+};
+template <class K>
+struct SendRows {
+    float w[K::NP][K::VEC], b[K::NP][K::VEC], g[K::D_OUT][K::VEC];
+};
+
 // Receiver pass: g_gy.
 template <class K>
 __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_recv_kernel(const DblParams prm) {
@@ -271,16 +290,26 @@ __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_recv_kerne
             }
         }
         __syncwarp();
-        for (int t = 0; t < nb; ++t) {
+        RecvRows<K> cur, nxt;
+        const auto load = [&](RecvRows<K>& rw, int t) {
             const int e = __shfl_sync(0xffffffffu, my_e, t);
             const int s = __shfl_sync(0xffffffffu, my_s, t);
-            if (s < 0) continue;
-            float wv[K::NP][V], bv[K::NP][V], xv[K::D_IN][V], av[K::D_IN][V];
-            load_rows<V>(wv, prm.w + (size_t)e * K::NP * C + c0 + cl, C, on);
-            load_rows<V>(bv, prm.b + (size_t)e * K::NP * C + c0 + cl, C, on);
-            load_rows<V>(xv, prm.x + (size_t)s * K::D_IN * C + c0 + cl, C, on);
-            load_rows<V>(av, prm.a + (size_t)s * K::D_IN * C + c0 + cl, C, on);
-            dbl_recv_edge<K>(AY + t * K::NA_PAD, AR + t * K::NA_PAD, xv, av, wv, bv, acc);
+            const bool ld = on && s >= 0;
+            load_rows<V>(rw.w, prm.w + (size_t)e * K::NP * C + c0 + cl, C, ld);
+            load_rows<V>(rw.b, prm.b + (size_t)e * K::NP * C + c0 + cl, C, ld);
+            load_rows<V>(rw.x, prm.x + (size_t)max(s, 0) * K::D_IN * C + c0 + cl, C, ld);
+            load_rows<V>(rw.a, prm.a + (size_t)max(s, 0) * K::D_IN * C + c0 + cl, C, ld);
+        };
+        if (DblShape<K>::PF) load(cur, 0);
+        for (int t = 0; t < nb; ++t) {
+            if (DblShape<K>::PF) {
+                if (t + 1 < nb) load(nxt, t + 1);
+            } else {
+                load(cur, t);
+            }
+            if (__shfl_sync(0xffffffffu, my_s, t) >= 0)
+                dbl_recv_edge<K>(AY + t * K::NA_PAD, AR + t * K::NA_PAD, cur.x, cur.a, cur.w, cur.b, acc);
+            if (DblShape<K>::PF) cur = nxt;
         }
         __syncwarp();
     }
@@ -328,19 +357,34 @@ __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_send_kerne
             }
         }
         __syncwarp();
-        for (int t = 0; t < nb; ++t) {
+        SendRows<K> cur, nxt;
+        const auto load = [&](SendRows<K>& rw, int t) {
             const int e = __shfl_sync(0xffffffffu, my_e, t);
             const int i = __shfl_sync(0xffffffffu, my_i, t);
-            if (i < 0) continue;
-            float wv[K::NP][V], bv[K::NP][V], gv[K::D_OUT][V];
-            load_rows<V>(wv, prm.w + (size_t)e * K::NP * C + c0 + cl, C, on);
-            load_rows<V>(bv, prm.b + (size_t)e * K::NP * C + c0 + cl, C, on);
-            load_rows<V>(gv, prm.gy + (size_t)i * K::D_OUT * C + c0 + cl, C, on);
+            const bool ld = on && i >= 0;
+            load_rows<V>(rw.w, prm.w + (size_t)e * K::NP * C + c0 + cl, C, ld);
+            load_rows<V>(rw.b, prm.b + (size_t)e * K::NP * C + c0 + cl, C, ld);
+            load_rows<V>(rw.g, prm.gy + (size_t)max(i, 0) * K::D_OUT * C + c0 + cl, C, ld);
+        };
+        if (DblShape<K>::PF) load(cur, 0);
+        for (int t = 0; t < nb; ++t) {
+            if (DblShape<K>::PF) {
+                if (t + 1 < nb) load(nxt, t + 1);
+            } else {
+                load(cur, t);
+            }
+            const int e = __shfl_sync(0xffffffffu, my_e, t);
+            const int i = __shfl_sync(0xffffffffu, my_i, t);
+            if (i < 0) {
+                if (DblShape<K>::PF) cur = nxt;
+                continue;
+            }
             float gYv[G], gY1[G];
 #pragma unroll
             for (int k = 0; k < G; ++k) gYv[k] = gY1[k] = 0.f;
-            dbl_send_edge<K>(AY + t * K::NA_PAD, AR + t * K::NA_PAD, xv, av, gv, wv, bv, gacc,
+            dbl_send_edge<K>(AY + t * K::NA_PAD, AR + t * K::NA_PAD, xv, av, cur.g, cur.w, cur.b, gacc,
                              prm.g_w + (size_t)e * K::NP * C + c0 + cl, C, on, gYv, gY1);
+            if (DblShape<K>::PF) cur = nxt;
             if constexpr (K::G > 0) {
                 warp_sum<G>(gYv);
                 warp_sum<G>(gY1);

@@ -43,7 +43,12 @@ struct DblLaunch {
     static constexpr DblKernelSet make() { return DblKernelSet{K::LIN, K::LSH, K::LOUT, K::VEC, K::TILE_C, K::G, &run}; }
 };
 
-#define EQC_DI(LSH, LOUT) DblLaunch<Cfg<EQC_LIN, LSH, LOUT, mode_vec(EQC_LIN, LSH, LOUT)>>::make()
+#ifndef EQC_DBL_VEC
+#define EQC_DBL_VEC 1   // channel width of every instance (0: 1 where an l = 3 block is present, else 2)
+#endif
+constexpr int dbl_vec(int lin, int lsh, int lout) { return EQC_DBL_VEC > 0 ? EQC_DBL_VEC : mode_vec(lin, lsh, lout); }
+
+#define EQC_DI(LSH, LOUT) DblLaunch<Cfg<EQC_LIN, LSH, LOUT, dbl_vec(EQC_LIN, LSH, LOUT)>>::make()
 #define EQC_DROW(LSH) {EQC_DI(LSH, 0), EQC_DI(LSH, 1), EQC_DI(LSH, 2), EQC_DI(LSH, 3)}
 #define EQC_DNAME2(a) dbl_instances_l##a
 #define EQC_DNAME(a) EQC_DNAME2(a)
