@@ -61,6 +61,51 @@ def byte_counts(N, E, C, D_in, D_out, P):
     return dict(fwd=fwd, bwd=bwd, graph=graph, step=step, h2d=h2d, d2h=d2h, kernels=graph + fwd + bwd)
 
 
+def time_node_product(W, Nn, dev, stream, reps):
+    """Median device time and GB/s of the node-local product (forward, and
+    backward with dw) on Nn nodes; bytes = each tensor read or written once
+    per kernel (u, v, w, y; u, v, w, gy, du, dv, dw partials, dw)."""
+    import torch
+
+    from equivariant_gnn_message_edge_b200 import binding as B
+    from equivariant_gnn_message_edge_b200.conv import NodeProduct
+    op = NodeProduct(W.irreps_in, W.L_sh, W.irreps_out, W.C, per_path=W.per_path)
+    gen = torch.Generator(device=dev).manual_seed(wl.SEED_X + 7)
+    C, P = W.C, op.P
+    with torch.cuda.stream(stream):
+        u = torch.randn((Nn, op.D_u, C), generator=gen, device=dev)
+        v = torch.randn((Nn, op.D_v, C), generator=gen, device=dev)
+        w = torch.randn((P, C), generator=gen, device=dev)
+        gy = torch.randn((Nn, op.D_out, C), generator=gen, device=dev)
+        y = torch.empty_like(gy)
+        du, dv, dw = torch.empty_like(u), torch.empty_like(v), torch.empty_like(w)
+        nws = B.eqconv_node_product_workspace_bytes(op.plan, Nn)
+        ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+    h = stream.cuda_stream
+    fe, be = [], []
+    for _ in range(reps + 1):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        B.eqconv_node_product(op.plan, Nn, u, v, w, y, h)
+        ev[1].record(stream)
+        B.eqconv_node_product_backward(op.plan, Nn, u, v, w, gy, du, dv, dw, ws, nws, h)
+        ev[2].record(stream)
+        fe.append(ev)
+    stream.synchronize()
+    f_ms = statistics.median([e[0].elapsed_time(e[1]) for e in fe[1:]])
+    b_ms = statistics.median([e[1].elapsed_time(e[2]) for e in fe[1:]])
+    row = 4 * C * Nn
+    fb = row * (op.D_u + op.D_v + op.D_out) + 4 * P * C
+    bb = row * (2 * op.D_u + 2 * op.D_v + op.D_out) + 4 * P * C + 2 * nws + 4 * P * C
+    peak = measured_peak()[0]
+    return {"nodes": Nn, "paths": P, "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
+            "fwd_gbps": round(fb / (f_ms * 1e-3) / 1e9, 1), "bwd_gbps": round(bb / (b_ms * 1e-3) / 1e9, 1),
+            "fwd_frac_of_measured_hbm": round(fb / (f_ms * 1e-3) / 1e9 / peak, 4),
+            "bwd_frac_of_measured_hbm": round(bb / (b_ms * 1e-3) / 1e9 / peak, 4),
+            "bytes": "fwd: u, v, w read, y written; bwd: u, v, w, gy read, du, dv written, dw partials written "
+                     "and read, dw written"}
+
+
 def dbl_bytes(N, E, C, D_in, D_out, P, part_bytes):
     """Algorithmic bytes of one double backward: receiver pass, sender pass
     and r epilogue, each kernel's inputs and outputs counted once."""
@@ -339,6 +384,12 @@ def run_native(args, rank, world, local_rank):
                "bytes": "per kernel: receiver pass, sender pass, r epilogue, each tensor once per kernel"}
         del cot_a, cot_b, cot_q, outs, dws
 
+    # node-local channel-diagonal product on 4N nodes of the same irreps (inputs
+    # well above L2), forward and backward, timed separately
+    nprod = None
+    if not W.all_parity and not args.no_node_product:
+        nprod = time_node_product(W, 4 * N, dev, stream, max(3, args.steps // 2))
+
     # End to end through the public API with host buffers (pinned), copies
     # timed: every step uploads its inputs and downloads its results.  Steps
     # are pipelined over two device sets and three streams, so step k's
@@ -439,6 +490,7 @@ def run_native(args, rank, world, local_rank):
                          "frac": round(bc["fwd"] / (fwd_avg * 1e-3) / 1e9 / peak, 4), "traffic": traffic.get("fwd"),
                          "algorithmic_bytes": bc["fwd"]},
         "double_backward": dbl,
+        "node_product": nprod,
         "gpu_launches": int(launches),
         "clocks": clk.summary((w0, w1)),
     }
@@ -573,6 +625,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-double-backward", action="store_true")
+    ap.add_argument("--no-node-product", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--nodes", type=int, default=None,

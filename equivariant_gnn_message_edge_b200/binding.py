@@ -36,6 +36,8 @@ ABI_FUNCTIONS = (
     "eqconv_last_error", "eqconv_graph_build_noalloc", "eqconv_plan_set_gather_budget",
     "eqconv_plan_create_ex", "eqconv_plan_path_rows", "eqconv_enumerate_paths_ex",
     "eqconv_double_backward_workspace_bytes", "eqconv_double_backward",
+    "eqconv_node_product_plan_create", "eqconv_node_product", "eqconv_node_product_workspace_bytes",
+    "eqconv_node_product_backward",
 )
 
 
@@ -80,6 +82,11 @@ _SIGS = {
     "eqconv_backward": (_ci, [_vp, _pg, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _cu, _vp]),
     "eqconv_double_backward_workspace_bytes": (_sz, [_vp, _ci]),
     "eqconv_double_backward": (_ci, [_vp, _pg] + [_vp] * 12 + [_sz, _vp]),
+    "eqconv_node_product_plan_create": (_ci, [ctypes.POINTER(_vp), ctypes.c_char_p, _ci, ctypes.c_char_p, _ci,
+                                                _cu]),
+    "eqconv_node_product": (_ci, [_vp, _ci, _vp, _vp, _vp, _vp, _vp]),
+    "eqconv_node_product_workspace_bytes": (_sz, [_vp, _ci]),
+    "eqconv_node_product_backward": (_ci, [_vp, _ci] + [_vp] * 8 + [_sz, _vp]),
     "eqconv_spherical_harmonics": (_ci, [_vp, _ci, _vp, _vp, _vp]),
     "eqconv_get_device_error": (_ci, [_vp, _vp, _pi]),
     "eqconv_plan_destroy": (None, [_vp]),
@@ -275,6 +282,31 @@ def eqconv_double_backward(plan: int, graph: eqconv_graph_t, x, r, w, gy, ga, gb
                                         _ptr(ga, f), _ptr(gb, f), _ptr(gq, f), _ptr(g_x, f), _ptr(g_w, f),
                                         _ptr(g_gy, f), _ptr(g_r, f), _ptr(workspace), int(workspace_bytes),
                                         _stream(stream)), "eqconv_double_backward")
+
+
+def eqconv_node_product_plan_create(irreps_u: str, L_v: int, irreps_out: str, C: int, out_mode: int = 0) -> int:
+    h = _vp()
+    _check(lib().eqconv_node_product_plan_create(ctypes.byref(h), irreps_u.encode(), int(L_v), irreps_out.encode(),
+                                                 int(C), int(out_mode)), "eqconv_node_product_plan_create")
+    return h.value
+
+
+def eqconv_node_product(plan: int, N: int, u, v, w, y, stream=None) -> None:
+    f = _f32()
+    _check(lib().eqconv_node_product(plan, int(N), _ptr(u, f), _ptr(v, f), _ptr(w, f), _ptr(y, f), _stream(stream)),
+           "eqconv_node_product")
+
+
+def eqconv_node_product_workspace_bytes(plan: int, N: int) -> int:
+    return int(lib().eqconv_node_product_workspace_bytes(plan, int(N)))
+
+
+def eqconv_node_product_backward(plan: int, N: int, u, v, w, gy, du, dv, dw, workspace=None,
+                                 workspace_bytes: int = 0, stream=None) -> None:
+    f = _f32()
+    _check(lib().eqconv_node_product_backward(plan, int(N), _ptr(u, f), _ptr(v, f), _ptr(w, f), _ptr(gy, f),
+                                              _ptr(du, f), _ptr(dv, f), _ptr(dw, f), _ptr(workspace),
+                                              int(workspace_bytes), _stream(stream)), "eqconv_node_product_backward")
 
 
 def eqconv_spherical_harmonics(plan: int, E: int, r, Y, stream=None) -> None:

@@ -146,3 +146,60 @@ class _EqConvBwdFn(torch.autograd.Function):
         z = lambda t, like: torch.zeros_like(like) if t is None else t.contiguous()
         g_x, g_w, g_gy, g_r = ctx.conv.double_backward_raw(ctx.g, x, r, w, gy, z(ga, x), z(gb, w), z(gq, r))
         return None, None, None, g_x, g_r, g_w, g_gy
+
+
+class NodeProduct:
+    """Node-local channel-diagonal product of two node features (see
+    include/eqconv.h): y = sum_p w_p C_p u_l1 v_l2, summed per output irrep or
+    kept per path (per_path=True)."""
+
+    def __init__(self, irreps_u: str, L_v: int, irreps_out: str, C: int, per_path: bool = False):
+        self.irreps_u, self.L_v, self.irreps_out, self.C = irreps_u, L_v, irreps_out, C
+        self.plan = B.eqconv_node_product_plan_create(irreps_u, L_v, irreps_out, C,
+                                                      B.EQCONV_OUT_PER_PATH if per_path else 0)
+        info = B.eqconv_plan_info(self.plan)
+        self.P, self.D_u, self.D_v, self.D_out = info["P"], info["D_in"], info["D_sh"], info["D_out"]
+        self.paths = info["paths"]
+        self.path_rows = B.eqconv_plan_path_rows(self.plan)
+
+    def __del__(self):
+        try:
+            B.eqconv_plan_destroy(self.plan)
+        except Exception:
+            pass
+
+    def forward_raw(self, u, v, w=None, y=None, stream=None):
+        if y is None:
+            y = torch.empty((u.shape[0], self.D_out, self.C), dtype=torch.float32, device=u.device)
+        B.eqconv_node_product(self.plan, u.shape[0], u, v, w, y, stream)
+        return y
+
+    def backward_raw(self, u, v, w, gy, need_dw=True, workspace=None, stream=None):
+        N = u.shape[0]
+        du, dv = torch.empty_like(u), torch.empty_like(v)
+        dw = torch.empty((self.P, self.C), dtype=torch.float32, device=u.device) if need_dw else None
+        nbytes = B.eqconv_node_product_workspace_bytes(self.plan, N) if need_dw else 0
+        if nbytes and workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=u.device)
+        B.eqconv_node_product_backward(self.plan, N, u, v, w, gy, du, dv, dw, workspace, nbytes, stream)
+        return du, dv, dw
+
+    def __call__(self, u, v, w=None):
+        return _NodeProductFn.apply(self, u, v, w)
+
+
+class _NodeProductFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, op: NodeProduct, u, v, w):
+        u, v = u.contiguous(), v.contiguous()
+        w = None if w is None else w.contiguous()
+        ctx.op, ctx.has_w = op, w is not None
+        ctx.save_for_backward(u, v, w)
+        return op.forward_raw(u, v, w)
+
+    @staticmethod
+    def backward(ctx, gy):
+        u, v, w = ctx.saved_tensors
+        need_dw = ctx.has_w and ctx.needs_input_grad[3]
+        du, dv, dw = ctx.op.backward_raw(u, v, w, gy.contiguous(), need_dw=need_dw)
+        return None, du, dv, dw

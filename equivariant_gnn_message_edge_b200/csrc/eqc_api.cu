@@ -22,6 +22,7 @@
 
 #include "eqc_conv.cuh"
 #include "eqc_dbl.cuh"
+#include "eqc_nodeprod.cuh"
 #include "eqc_dispatch.h"
 #include "eqc_graph.h"
 #include "eqconv.h"
@@ -128,6 +129,8 @@ struct eqconv_plan_s {
     const eqc::KernelSet* det_ks;      // deterministic backward
     const eqc::KernelSet* atomic_ks;   // atomic backward
     const eqc::DblKernelSet* dbl_ks;   // double backward (summed natural-parity outputs only)
+    bool node_product;                 // a node-local product plan (no convolution)
+    const eqc::NpKernelSet* np_ks;     // node-local product
 };
 
 namespace {
@@ -262,8 +265,26 @@ int eqconv_plan_create(eqconv_plan_t* out, const char* irreps_in, int L_sh, cons
     return eqconv_plan_create_ex(out, irreps_in, L_sh, irreps_out, C, 0u);
 }
 
+namespace {
+int create_plan(eqconv_plan_t* out, const char* irreps_in, int L_sh, const char* irreps_out, int C,
+                unsigned out_mode, bool node_product);
+}
+
 int eqconv_plan_create_ex(eqconv_plan_t* out, const char* irreps_in, int L_sh, const char* irreps_out, int C,
                           unsigned out_mode) {
+    return create_plan(out, irreps_in, L_sh, irreps_out, C, out_mode, false);
+}
+
+int eqconv_node_product_plan_create(eqconv_plan_t* out, const char* irreps_u, int L_v, const char* irreps_out, int C,
+                                    unsigned out_mode) {
+    return create_plan(out, irreps_u, L_v, irreps_out, C, out_mode, true);
+}
+
+}  // extern "C"
+
+namespace {
+int create_plan(eqconv_plan_t* out, const char* irreps_in, int L_sh, const char* irreps_out, int C,
+                unsigned out_mode, bool node_product) {
     if (!out) return EQCONV_ERR_INVALID_ARG;
     *out = nullptr;
     int lin = 0, lout = 0;
@@ -305,7 +326,10 @@ int eqconv_plan_create_ex(eqconv_plan_t* out, const char* irreps_in, int L_sh, c
         p->fwd_ks = p->det_ks = p->atomic_ks = eqc::find_mode_instance(lin, L_sh, lout, mode);
     }
     p->dbl_ks = mode == 0 ? eqc::find_dbl_instance(lin, L_sh, lout) : nullptr;
-    if (!p->fwd_ks || !p->det_ks || !p->atomic_ks) {
+    p->node_product = node_product;
+    p->np_ks = node_product ? eqc::find_np_instance(lin, L_sh, lout, mode) : nullptr;
+    const bool ok = node_product ? p->np_ks != nullptr : (p->fwd_ks && p->det_ks && p->atomic_ks);
+    if (!ok) {
         delete p;
         return EQCONV_ERR_UNSUPPORTED;
     }
@@ -321,9 +345,13 @@ int eqconv_plan_create_ex(eqconv_plan_t* out, const char* irreps_in, int L_sh, c
     *out = p;
     return EQCONV_OK;
 }
+}  // namespace
+
+extern "C" {
 
 int eqconv_plan_set_vec(eqconv_plan_t plan, int fwd_vec, int bwd_vec) {
     if (!plan) return EQCONV_ERR_INVALID_ARG;
+    if (plan->node_product) return EQCONV_ERR_UNSUPPORTED;
     const auto ok = [](int v) { return v == 1 || v == 2 || v == 4; };
     if (!ok(fwd_vec) || !ok(bwd_vec)) return EQCONV_ERR_UNSUPPORTED;
     if (plan->mode != 0) {
@@ -451,6 +479,7 @@ int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, 
                    float* y, unsigned flags, eqconv_stream_t stream) {
     (void)flags;
     if (!plan) return EQCONV_ERR_INVALID_ARG;
+    if (plan->node_product) return EQCONV_ERR_INVALID_ARG;   // not a convolution plan
     int rc = check_graph(g);
     if (rc != EQCONV_OK) return rc;
     if ((rc = check_device(plan)) != EQCONV_OK) return rc;
@@ -481,6 +510,7 @@ int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
                     const float* gy, float* dx, float* dw, float* dr, void* workspace, size_t workspace_bytes,
                     unsigned flags, eqconv_stream_t stream) {
     if (!plan) return EQCONV_ERR_INVALID_ARG;
+    if (plan->node_product) return EQCONV_ERR_INVALID_ARG;   // not a convolution plan
     int rc = check_graph(g);
     if (rc != EQCONV_OK) return rc;
     if ((rc = check_device(plan)) != EQCONV_OK) return rc;
@@ -548,6 +578,7 @@ int eqconv_double_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const fl
                            float* g_x, float* g_w, float* g_gy, float* g_r, void* workspace, size_t workspace_bytes,
                            eqconv_stream_t stream) {
     if (!plan) return EQCONV_ERR_INVALID_ARG;
+    if (plan->node_product) return EQCONV_ERR_INVALID_ARG;   // not a convolution plan
     int rc = check_graph(g);
     if (rc != EQCONV_OK) return rc;
     if ((rc = check_device(plan)) != EQCONV_OK) return rc;
@@ -587,6 +618,59 @@ int eqconv_double_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const fl
     send.perm = g->send_perm;
     send.other = g->receivers;
     return cuda_status(plan->dbl_ks->run(recv, send, (cudaStream_t)stream), "double backward");
+}
+
+size_t eqconv_node_product_workspace_bytes(eqconv_plan_t plan, int N) {
+    if (!plan || N < 0 || !plan->np_ks) return 0;
+    const int need = (N + eqc::kNpWarps - 1) / eqc::kNpWarps;
+    const int blocks = need < 2 * 148 ? (need > 0 ? need : 1) : 2 * 148;
+    return (size_t)blocks * eqc::kNpWarps * (size_t)plan->P * (size_t)plan->C * sizeof(float);
+}
+
+int eqconv_node_product(eqconv_plan_t plan, int N, const float* u, const float* v, const float* w, float* y,
+                        eqconv_stream_t stream) {
+    if (!plan || N < 0) return EQCONV_ERR_INVALID_ARG;
+    if (!plan->np_ks) return plan->node_product ? EQCONV_ERR_UNSUPPORTED : EQCONV_ERR_INVALID_ARG;
+    int rc = check_device(plan);
+    if (rc != EQCONV_OK) return rc;
+    if (N == 0) return EQCONV_OK;
+    if (!u || !v || !y || !aligned16(u) || !aligned16(v) || !aligned16(y) || (w && !aligned16(w)))
+        return EQCONV_ERR_INVALID_ARG;
+    eqc::NpParams prm{};
+    prm.u = u;
+    prm.v = v;
+    prm.w = w;
+    prm.y = y;
+    prm.N = N;
+    prm.C = plan->C;
+    return cuda_status(plan->np_ks->fwd(prm, (cudaStream_t)stream), "node product");
+}
+
+int eqconv_node_product_backward(eqconv_plan_t plan, int N, const float* u, const float* v, const float* w,
+                                 const float* gy, float* du, float* dv, float* dw, void* workspace,
+                                 size_t workspace_bytes, eqconv_stream_t stream) {
+    if (!plan || N < 0) return EQCONV_ERR_INVALID_ARG;
+    if (!plan->np_ks) return plan->node_product ? EQCONV_ERR_UNSUPPORTED : EQCONV_ERR_INVALID_ARG;
+    int rc = check_device(plan);
+    if (rc != EQCONV_OK) return rc;
+    if (!u || !v || !gy || !du || !dv) return EQCONV_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(v) || !aligned16(gy) || !aligned16(du) || !aligned16(dv) ||
+        (w && !aligned16(w)) || (dw && !aligned16(dw)))
+        return EQCONV_ERR_INVALID_ARG;
+    const size_t need = dw ? eqconv_node_product_workspace_bytes(plan, N) : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return EQCONV_ERR_WORKSPACE;
+    eqc::NpParams prm{};
+    prm.u = u;
+    prm.v = v;
+    prm.w = w;
+    prm.gy = gy;
+    prm.du = du;
+    prm.dv = dv;
+    prm.dw = dw;
+    prm.dw_part = dw ? static_cast<float*>(workspace) : nullptr;
+    prm.N = N;
+    prm.C = plan->C;
+    return cuda_status(plan->np_ks->bwd(prm, (cudaStream_t)stream), "node product backward");
 }
 
 int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y, eqconv_stream_t stream) {

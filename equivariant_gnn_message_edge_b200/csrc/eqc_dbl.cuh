@@ -261,7 +261,7 @@ struct SendRows {
 template <class K>
 __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_recv_kernel(const DblParams prm) {
     constexpr int V = K::VEC, CH = DblShape<K>::CH, W = DblShape<K>::WARPS;
-    extern __shared__ __align__(16) float4 smem4[];
+    extern __shared__ __align__(128) float4 smem4[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int node = blockIdx.x * W + warp;
     if (node >= prm.N) return;
@@ -325,7 +325,7 @@ template <class K>
 __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_send_kernel(const DblParams prm) {
     constexpr int V = K::VEC, CH = DblShape<K>::CH, W = DblShape<K>::WARPS;
     constexpr int G = K::G > 0 ? K::G : 1;
-    extern __shared__ __align__(16) float4 smem4[];
+    extern __shared__ __align__(128) float4 smem4[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int node = blockIdx.x * W + warp;
     if (node >= prm.N) return;

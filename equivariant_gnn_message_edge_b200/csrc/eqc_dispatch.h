@@ -103,6 +103,28 @@ inline const DblKernelSet* find_dbl_instance(int lin, int lsh, int lout) {
     return fns[lin](lsh, lout);
 }
 
+// Node-local channel-diagonal product (summed or per-path outputs) of one
+// (L_u, L_v, L_out) at one channel width.
+struct NpParams;
+struct NpKernelSet {
+    int lin, lsh, lout, vec, mode;
+    cudaError_t (*fwd)(const NpParams&, cudaStream_t);
+    cudaError_t (*bwd)(const NpParams&, cudaStream_t);
+};
+
+// Defined in eqc_np_l<L_u>.cu.
+const NpKernelSet* np_instances_l0(int lv, int lout, bool per_path);
+const NpKernelSet* np_instances_l1(int lv, int lout, bool per_path);
+const NpKernelSet* np_instances_l2(int lv, int lout, bool per_path);
+const NpKernelSet* np_instances_l3(int lv, int lout, bool per_path);
+
+inline const NpKernelSet* find_np_instance(int lu, int lv, int lout, int mode) {
+    using Fn = const NpKernelSet* (*)(int, int, bool);
+    static const Fn fns[4] = {np_instances_l0, np_instances_l1, np_instances_l2, np_instances_l3};
+    if (lu < 0 || lu > 3 || (mode != 0 && mode != 2)) return nullptr;
+    return fns[lu](lv, lout, mode == 2);
+}
+
 // Harmonics-only kernels (depend on L_sh only); defined in eqc_api.cu.
 cudaError_t launch_dr_epilogue(int lsh, const float* gy_part, int T, const float* r, float* dr, int E,
                                cudaStream_t st);

@@ -263,6 +263,44 @@ EQCONV_API int eqconv_double_backward(eqconv_plan_t plan, const eqconv_graph_t* 
                                       float* g_r, void* workspace, size_t workspace_bytes,
                                       eqconv_stream_t stream);
 
+/* ---- Node-local channel-diagonal product ----------------------------------
+ * FlashCart (arXiv 2610.06409) §5, App. B and App. D: the correlation ladder
+ * builds higher-order features by repeated pairwise products at each atom;
+ * each step couples same-index channels of two node features along the
+ * admissible paths and keeps every path's output (a learned linear map mixes
+ * paths and channels afterwards) or sums weighted paths.
+ *   y[i, o3(p)+m3, c] = sum_p w[p,c] sum_{m1,m2} C_p[m1,m2,m3] u[i, l1 m1, c] v[i, l2 m2, c]
+ * u [N][D_u][C] (irreps_u a natural-parity prefix), v [N][(L_v+1)^2][C]
+ * (degrees 0..L_v, natural parity, like the harmonics of the convolution),
+ * w [P][C] per-path, per-channel weights (NULL: all ones), y [N][D_out][C].
+ * Paths, their order, the CG tables and the output layouts (summed, or
+ * EQCONV_OUT_PER_PATH) are exactly those of a convolution plan with
+ * L_sh = L_v; eqconv_plan_info / eqconv_plan_path_rows describe them.
+ * Both-parity outputs are not offered for this op (out_mode 0 or
+ * EQCONV_OUT_PER_PATH).  A node-product plan is not a convolution plan: the
+ * convolution entry points reject it with EQCONV_ERR_INVALID_ARG. */
+EQCONV_API int eqconv_node_product_plan_create(eqconv_plan_t* out, const char* irreps_u, int L_v,
+                                               const char* irreps_out, int C, unsigned out_mode);
+
+/* y = the product above, on `stream`; one launch.  Rows 16-byte aligned. */
+EQCONV_API int eqconv_node_product(eqconv_plan_t plan, int N, const float* u, const float* v,
+                                   const float* w, float* y, eqconv_stream_t stream);
+
+/* Device workspace bytes eqconv_node_product_backward needs when dw is
+ * requested (per-warp partials of dw, [warps][P][C] fp32). */
+EQCONV_API size_t eqconv_node_product_workspace_bytes(eqconv_plan_t plan, int N);
+
+/* Backward given gy [N][D_out][C]:
+ *   du[i, l1 m1, c] = sum_p w[p,c] sum_{m2,m3} C_p v[i, l2 m2, c] gy[i, o3+m3, c]
+ *   dv[i, l2 m2, c] = sum_p w[p,c] sum_{m1,m3} C_p u[i, l1 m1, c] gy[i, o3+m3, c]
+ *   dw[p, c]        = sum_i sum C_p u v gy          (dw may be NULL: not computed)
+ * Deterministic: each warp sums dw over a fixed node set and a second launch
+ * adds the warps' partials in order.  All outputs are overwritten. */
+EQCONV_API int eqconv_node_product_backward(eqconv_plan_t plan, int N, const float* u, const float* v,
+                                            const float* w, const float* gy, float* du, float* dv,
+                                            float* dw, void* workspace, size_t workspace_bytes,
+                                            eqconv_stream_t stream);
+
 /* The spherical harmonics the kernels use, Y [E][(L_sh+1)^2] (a test hook
  * for the in-kernel harmonics; not on the hot path). */
 EQCONV_API int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y,
