@@ -50,6 +50,12 @@
 #ifndef EQC_CHUNK_LARGE_ATOMIC
 #define EQC_CHUNK_LARGE_ATOMIC 8   // the same for the atomic backward (register-bound, 2 CTAs/SM)
 #endif
+#ifndef EQC_BWD_H
+#define EQC_BWD_H 1         // 1: the backward takes t = A^T g from h = C.g (no coupling matrices)
+#endif
+#ifndef EQC_CHUNK_BWD_H
+#define EQC_CHUNK_BWD_H 0   // edges per harmonics batch of that backward (0: as the coupling batch)
+#endif
 #ifndef EQC_FWD_PRED
 #define EQC_FWD_PRED 1      // 1: predicate the forward row reads at VEC = 4; 2: at every width
 #endif
@@ -95,6 +101,8 @@ struct Cfg {
                             : (EQC_CHUNK_SMALL > 0 ? EQC_CHUNK_SMALL : (VEC >= 4 ? 16 : 8));
     }
     static constexpr int GS = G | 1;                // gY row stride in shared memory (odd)
+    static constexpr int YS = pad_odd4(D_SH);       // harmonics row (backward without coupling matrices)
+    static constexpr int A_ROW = NA_PAD > YS ? NA_PAD : YS;   // coupling-batch row stride in shared memory
     static constexpr int TILE_C = 32 * VEC;
     static constexpr int STAGES = EQC_STAGES;       // edges staged ahead per warp (ring depth)
     static_assert(NP > 0, "no admissible path");
@@ -354,11 +362,44 @@ __device__ __forceinline__ void bwd_edge(const float* As, const XR& X, const GR&
         for (int m = 0; m < d1; ++m) X.get(o1 + m, xv[m]);
         Wr.get(p, wp);
         float t[d1][V];
+        [[maybe_unused]] float hG[(l2 > 0 && EQC_BWD_H) ? 2 * l2 + 1 : 1][V];   // sum_m1 x[m1] h[m1][m2]
         if constexpr (l2 == 0) {
 #pragma unroll
             for (int m = 0; m < d1; ++m)
 #pragma unroll
                 for (int v = 0; v < V; ++v) t[m][v] = gv[m][v];
+        } else if constexpr (EQC_BWD_H) {
+            // h[m1][m2] = sum_m3 C_p[m1,m2,m3] g[m3] gives both t[m1] = sum_m2 Y[m2] h
+            // (= (A_p^T g)[m1]) and the harmonic gradient sum_m1 x[m1] h
+            constexpr int d2 = 2 * l2 + 1, o2 = l2 * l2;
+#pragma unroll
+            for (int m = 0; m < d1; ++m)
+#pragma unroll
+                for (int v = 0; v < V; ++v) t[m][v] = 0.f;
+#pragma unroll
+            for (int m = 0; m < d2; ++m)
+#pragma unroll
+                for (int v = 0; v < V; ++v) hG[m][v] = 0.f;
+            static_for<d2>([&](auto m2c) {
+                constexpr int m2 = EQC_CV(m2c);
+                const float y2 = As[o2 + m2];                 // this edge's Y, broadcast
+                static_for<d1>([&](auto m1c) {
+                    constexpr int m1 = EQC_CV(m1c);
+                    if constexpr (cg_row_nonzero<l1, l2, l3>(m1, m2)) {
+#pragma unroll
+                        for (int v = 0; v < V; ++v) {
+                            float h = 0.f;
+                            static_for<d3>([&](auto m3c) {
+                                constexpr int m3 = EQC_CV(m3c);
+                                constexpr double c = RealCG<l1, l2, l3>::t.v[m1][m2][m3];
+                                if constexpr (c != 0.0) h = fmaf((float)c, gv[m3][v], h);
+                            });
+                            t[m1][v] = fmaf(y2, h, t[m1][v]);
+                            hG[m2][v] = fmaf(xv[m1][v], h, hG[m2][v]);
+                        }
+                    }
+                });
+            });
         } else {
             constexpr int n4 = (d1 * d3 + 3) / 4;
             constexpr int aoff = K::AO.off[p];
@@ -395,7 +436,16 @@ __device__ __forceinline__ void bwd_edge(const float* As, const XR& X, const GR&
                 for (int v = 0; v < V; ++v) dxg[m1][v] = fmaf(wp[v], t[m1][v], dxg[m1][v]);
             if constexpr (last_of_block) dx_sink(o1, d1, dxg);
         }
-        if constexpr (l2 > 0) {
+        if constexpr (l2 > 0 && EQC_BWD_H) {
+            constexpr int d2 = 2 * l2 + 1, o2 = l2 * l2;
+#pragma unroll
+            for (int m2 = 0; m2 < d2; ++m2) {
+                float gsum = 0.f;
+#pragma unroll
+                for (int v = 0; v < V; ++v) gsum = fmaf(wp[v], hG[m2][v], gsum);
+                gyl[o2 + m2 - 1] += gsum;
+            }
+        } else if constexpr (l2 > 0) {
             constexpr int d2 = 2 * l2 + 1, o2 = l2 * l2;
             static_for<d2>([&](auto m2c) {
                 constexpr int m2 = EQC_CV(m2c);
@@ -550,7 +600,8 @@ struct WarpSmem {
     static constexpr int up32(int f) { return (f + 31) & ~31; }
     static constexpr int ST_F = S * Stage<K, NG>::FLOATS;
     static constexpr int BAR_F = up32(4 * S);
-    static constexpr int A_F = up32(CH * K::NA_PAD);
+    // the backward without coupling matrices keeps only each edge's harmonics
+    static constexpr int A_F = up32(CH * ((WITH_GY && EQC_BWD_H) ? K::YS : K::A_ROW));
     static constexpr int GY_F = WITH_GY ? up32(CH * K::GS) : 0;
     static constexpr int TOTAL_F = ST_F + BAR_F + A_F + GY_F;
     static constexpr int BYTES = TOTAL_F * 4;
@@ -584,7 +635,7 @@ struct FwdShape {
 };
 template <class K, bool DET>
 struct BwdShape {
-    static constexpr int CH = K::chunk(!DET);
+    static constexpr int CH = (EQC_BWD_H && EQC_CHUNK_BWD_H > 0) ? EQC_CHUNK_BWD_H : K::chunk(!DET);
     static constexpr int DL = DET ? K::D_OUT : K::D_IN;     // rows gathered per edge
     using L = WarpSmem<K, DL, true, CH>;
     // the atomic kernel keeps the receiver's gy rows in registers and is held
@@ -873,7 +924,13 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
                 const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
                 float Y[K::D_SH];
                 sh_eval<K::LSH>(ok, ux, uy, uz, Y);
-                compute_A<K>(Y, As + (lane - b0) * K::NA_PAD);
+                if constexpr (EQC_BWD_H) {
+                    float* yrow = As + (lane - b0) * K::YS;
+#pragma unroll
+                    for (int q = 0; q < K::D_SH; ++q) yrow[q] = Y[q];
+                } else {
+                    compute_A<K>(Y, As + (lane - b0) * K::NA_PAD);
+                }
             }
             __syncwarp();
             for (int t = b0; t < b0 + nb; ++t) {
@@ -898,7 +955,8 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
                 };
                 if constexpr (DET) {
                     auto no_sink = [](int, int, const float (&)[1][V]) {};
-                    bwd_edge<K, true>(As + (t - b0) * K::NA_PAD, RegRows<V, K::D_IN>{xres}, Lr, Wr, dxacc, no_sink,
+                    bwd_edge<K, true>(As + (t - b0) * (EQC_BWD_H ? K::YS : K::NA_PAD), RegRows<V, K::D_IN>{xres}, Lr,
+                                      Wr, dxacc, no_sink,
                                       gyl, store_dw);
                 } else {
                     float* dxs = prm.dx + (size_t)o * K::D_IN * C + c_off;
@@ -907,7 +965,8 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
 #pragma unroll
                             for (int m = 0; m < d1; ++m) red_add<V>(dxs + (size_t)(o1 + m) * C, blk[m]);
                     };
-                    bwd_edge<K, false>(As + (t - b0) * K::NA_PAD, Lr, RegRows<V, K::D_OUT>{gres}, Wr, dxacc, sink,
+                    bwd_edge<K, false>(As + (t - b0) * (EQC_BWD_H ? K::YS : K::NA_PAD), Lr,
+                                       RegRows<V, K::D_OUT>{gres}, Wr, dxacc, sink,
                                        gyl, store_dw);
                 }
                 if constexpr (K::G > 0) {
