@@ -23,7 +23,8 @@
 //     tile, sums in registers;
 //   * sender pass (sender CSR): g_x in registers, g_w stored per edge, the
 //     per-tile partials of gYv and gY1 (warp butterfly, fixed order) to a
-//     workspace [E][T][2G];
+//     workspace [E][T][2G]; it contracts through h = C.gy and needs only
+//     each edge's Y and rho, not its coupling matrices;
 //   * r epilogue (one thread per edge): sums the tiles in order and applies
 //     the gradient and the Hessian-vector product of the harmonics.
 // Rows are read with plain vector loads (no staging ring): the double
@@ -65,7 +66,8 @@ struct DblShape {
     // and cost at lmax 3 (41.6 -> 46.8 ms), where the per-edge code is larger
     static constexpr bool PF = EQC_DBL_PREFETCH && K::NA_PAD <= 128;
     static constexpr int CH = K::NA_PAD > 128 ? 4 : 8;        // edges per coupling batch
-    static constexpr int WARP_FLOATS = 2 * CH * K::NA_PAD;    // A(Y) and A(rho)
+    // receiver pass: A(Y) and A(rho); sender pass: Y and rho
+    static constexpr int WARP_FLOATS = 2 * CH * (K::NA_PAD > K::D_SH ? K::NA_PAD : K::D_SH);
     static constexpr int WARPS = 4;
     static constexpr int SMEM = WARPS * WARP_FLOATS * 4;
 };
@@ -115,6 +117,24 @@ __device__ __forceinline__ void dbl_couplings(const float* r, const float* q, in
     compute_A<K>(rho, AR);
 }
 
+// Lane t of the warp: the harmonics Y and rho = (dY/dr) q of edge e into
+// shared memory (rows of K::YS floats: Y first, then rho), for the sender
+// pass, which needs no coupling matrices.
+template <class K>
+__device__ __forceinline__ void dbl_harmonics(const float* r, const float* q, int e, float* Yrow) {
+    const float rx = r[3 * (size_t)e], ry = r[3 * (size_t)e + 1], rz = r[3 * (size_t)e + 2];
+    float ux, uy, uz, il;
+    const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
+    float Y[K::D_SH], rho[K::D_SH];
+    sh_eval<K::LSH>(ok, ux, uy, uz, Y);
+    sh_jvp<K::LSH>(rx, ry, rz, q[3 * (size_t)e], q[3 * (size_t)e + 1], q[3 * (size_t)e + 2], rho);
+#pragma unroll
+    for (int k = 0; k < K::D_SH; ++k) {
+        Yrow[k] = Y[k];
+        Yrow[K::D_SH + k] = rho[k];
+    }
+}
+
 // acc[o3] += w_p (A_p(Y) a + A_p(rho) x) + b_p A_p(Y) x for every path.
 template <class K>
 __device__ __forceinline__ void dbl_recv_edge(const float* AY, const float* AR, const float (&xv)[K::D_IN][K::VEC],
@@ -159,9 +179,13 @@ __device__ __forceinline__ void dbl_recv_edge(const float* AY, const float* AR, 
 }
 
 // Sender-side terms of one edge: g_x, g_w (stored per path), and this lane's
-// partials of gYv and gY1 (summed over its channels).
+// partials of gYv and gY1 (summed over its channels).  With
+// h[m1][m2] = sum_m3 C_p[m1,m2,m3] gy[m3] (per channel), one h serves all four
+// contractions: A_p(Y)^T gy = sum_m2 Y[m2] h, A_p(rho)^T gy = sum_m2 rho[m2] h,
+// G_p(a, gy) = sum_m1 a[m1] h and G_p(x, gy) = sum_m1 x[m1] h; so the pass
+// needs only each edge's Y and rho, not its coupling matrices.
 template <class K>
-__device__ __forceinline__ void dbl_send_edge(const float* AY, const float* AR, const float (&xv)[K::D_IN][K::VEC],
+__device__ __forceinline__ void dbl_send_edge(const float* Yrow, const float (&xv)[K::D_IN][K::VEC],
                                               const float (&av)[K::D_IN][K::VEC],
                                               const float (&gv)[K::D_OUT][K::VEC],
                                               const float (&wv)[K::NP][K::VEC], const float (&bv)[K::NP][K::VEC],
@@ -174,7 +198,7 @@ __device__ __forceinline__ void dbl_send_edge(const float* AY, const float* AR, 
         constexpr int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
         constexpr int o1 = l1 * l1, o2 = l2 * l2, o3 = K::PL.o3[p];
         float uY[d1][V], uR[d1][V];
-        if constexpr (l2 == 0) {
+        if constexpr (l2 == 0) {       // A(Y) = I, A(rho) = 0
 #pragma unroll
             for (int m = 0; m < d1; ++m)
 #pragma unroll
@@ -183,24 +207,40 @@ __device__ __forceinline__ void dbl_send_edge(const float* AY, const float* AR, 
                     uR[m][v] = 0.f;
                 }
         } else {
-            constexpr int n4 = (d1 * d3 + 3) / 4;
-            constexpr int aoff = K::AO.off[p];
-            float ay[n4 * 4], ar[n4 * 4];
-            load_A<n4>(AY + aoff, ay);
-            load_A<n4>(AR + aoff, ar);
 #pragma unroll
-            for (int m1 = 0; m1 < d1; ++m1)
+            for (int m = 0; m < d1; ++m)
+#pragma unroll
+                for (int v = 0; v < V; ++v) uY[m][v] = uR[m][v] = 0.f;
+            static_for<d2>([&](auto m2c) {
+                constexpr int m2 = EQC_CV(m2c);
+                const float y2 = Yrow[o2 + m2], r2 = Yrow[K::D_SH + o2 + m2];
+                float Ga[V], Gx[V];
+#pragma unroll
+                for (int v = 0; v < V; ++v) Ga[v] = Gx[v] = 0.f;
+                static_for<d1>([&](auto m1c) {
+                    constexpr int m1 = EQC_CV(m1c);
+                    if constexpr (cg_row_nonzero<l1, l2, l3>(m1, m2)) {
+#pragma unroll
+                        for (int v = 0; v < V; ++v) {
+                            float h = 0.f;
+                            static_for<d3>([&](auto m3c) {
+                                constexpr int m3 = EQC_CV(m3c);
+                                constexpr double c = RealCG<l1, l2, l3>::t.v[m1][m2][m3];
+                                if constexpr (c != 0.0) h = fmaf((float)c, gv[o3 + m3][v], h);
+                            });
+                            uY[m1][v] = fmaf(y2, h, uY[m1][v]);
+                            uR[m1][v] = fmaf(r2, h, uR[m1][v]);
+                            Ga[v] = fmaf(av[o1 + m1][v], h, Ga[v]);
+                            Gx[v] = fmaf(xv[o1 + m1][v], h, Gx[v]);
+                        }
+                    }
+                });
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    float sy = 0.f, sr = 0.f;
-#pragma unroll
-                    for (int m3 = 0; m3 < d3; ++m3) {
-                        sy = fmaf(ay[m3 * d1 + m1], gv[o3 + m3][v], sy);
-                        sr = fmaf(ar[m3 * d1 + m1], gv[o3 + m3][v], sr);
-                    }
-                    uY[m1][v] = sy;
-                    uR[m1][v] = sr;
+                    gYv[o2 + m2 - 1] = fmaf(wv[p][v], Ga[v], fmaf(bv[p][v], Gx[v], gYv[o2 + m2 - 1]));
+                    gY1[o2 + m2 - 1] = fmaf(wv[p][v], Gx[v], gY1[o2 + m2 - 1]);
                 }
+            });
         }
         float gw[V];
 #pragma unroll
@@ -213,35 +253,6 @@ __device__ __forceinline__ void dbl_send_edge(const float* AY, const float* AR, 
                 gw[v] = fmaf(av[o1 + m1][v], uY[m1][v], fmaf(xv[o1 + m1][v], uR[m1][v], gw[v]));
             }
         if (on) st_stream<V>(gw_row + (size_t)p * C, gw);
-        if constexpr (l2 > 0) {
-            // G_p(u, g)[m2] = sum C_p[m1,m2,m3] u[m1] g[m3], compile-time CG
-            static_for<d2>([&](auto m2c) {
-                constexpr int m2 = EQC_CV(m2c);
-                float Ga[V], Gx[V];
-#pragma unroll
-                for (int v = 0; v < V; ++v) Ga[v] = Gx[v] = 0.f;
-                static_for<d1>([&](auto m1c) {
-                    constexpr int m1 = EQC_CV(m1c);
-                    static_for<d3>([&](auto m3c) {
-                        constexpr int m3 = EQC_CV(m3c);
-                        constexpr double c = RealCG<l1, l2, l3>::t.v[m1][m2][m3];
-                        if constexpr (c != 0.0) {
-#pragma unroll
-                            for (int v = 0; v < V; ++v) {
-                                const float cg = (float)c * gv[o3 + m3][v];
-                                Ga[v] = fmaf(cg, av[o1 + m1][v], Ga[v]);
-                                Gx[v] = fmaf(cg, xv[o1 + m1][v], Gx[v]);
-                            }
-                        }
-                    });
-                });
-#pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    gYv[o2 + m2 - 1] = fmaf(wv[p][v], Ga[v], fmaf(bv[p][v], Gx[v], gYv[o2 + m2 - 1]));
-                    gY1[o2 + m2 - 1] = fmaf(wv[p][v], Gx[v], gY1[o2 + m2 - 1]);
-                }
-            });
-        }
     });
 }
 
@@ -329,8 +340,7 @@ __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_send_kerne
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int node = blockIdx.x * W + warp;
     if (node >= prm.N) return;
-    float* AY = reinterpret_cast<float*>(smem4) + warp * DblShape<K>::WARP_FLOATS;
-    float* AR = AY + CH * K::NA_PAD;
+    float* AY = reinterpret_cast<float*>(smem4) + warp * DblShape<K>::WARP_FLOATS;   // Y, rho rows
     const int C = prm.C;
     const int tile = blockIdx.y;
     const int c0 = tile * K::TILE_C, cl = lane * V;
@@ -353,7 +363,7 @@ __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_send_kerne
                 atomicOr(prm.status, 1u);
                 my_i = -1;
             } else {
-                dbl_couplings<K>(prm.r, prm.q, my_e, AY + lane * K::NA_PAD, AR + lane * K::NA_PAD);
+                dbl_harmonics<K>(prm.r, prm.q, my_e, AY + lane * 2 * K::D_SH);
             }
         }
         __syncwarp();
@@ -382,7 +392,7 @@ __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_send_kerne
             float gYv[G], gY1[G];
 #pragma unroll
             for (int k = 0; k < G; ++k) gYv[k] = gY1[k] = 0.f;
-            dbl_send_edge<K>(AY + t * K::NA_PAD, AR + t * K::NA_PAD, xv, av, cur.g, cur.w, cur.b, gacc,
+            dbl_send_edge<K>(AY + t * 2 * K::D_SH, xv, av, cur.g, cur.w, cur.b, gacc,
                              prm.g_w + (size_t)e * K::NP * C + c0 + cl, C, on, gYv, gY1);
             if (DblShape<K>::PF) cur = nxt;
             if constexpr (K::G > 0) {
