@@ -30,6 +30,9 @@ cg       complex CG by the Racah formula, complex->real change of basis
 sh       real spherical harmonics and their gradient w.r.t. the edge vector
 csr      receiver/sender CSR offsets and stable permutations
 conv     the convolution: NumPy brute force (per-edge messages) and the C
-         loop implementation in ``conv_ref.c`` (fp64 accumulation)
+         loop implementation in ``conv_ref.c`` (fp64 accumulation); output
+         variants (both parities, per-path blocks)
+dbl      the double backward (VJP of the backward), NumPy brute force
+nodeprod the node-local channel-diagonal product, forward and backward
 build    compiles ``conv_ref.c`` with gcc
 """

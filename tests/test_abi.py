@@ -175,3 +175,16 @@ def test_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         B._ptr(torch.zeros(4))
+
+
+def test_node_product_plans_validate_before_device_work():
+    cases = [("0e+1o", 1, "0e+1o+1e", B.EQCONV_OUT_ALL_PARITY, B.EQCONV_ERR_UNSUPPORTED),  # both parities
+             ("0e+2e", 1, "0e+1o", 0, B.EQCONV_ERR_UNSUPPORTED),                        # u not a prefix
+             ("0e+1o", 4, "0e+1o", 0, B.EQCONV_ERR_UNSUPPORTED),                        # L_v > 3
+             ("0e+1o", 1, "0e+1o", 8, B.EQCONV_ERR_INVALID_ARG)]                        # unknown bit
+    for ins, lv, outs, mode, status in cases:
+        with pytest.raises(B.EqconvError) as e:
+            B.eqconv_node_product_plan_create(ins, lv, outs, 8, mode)
+        assert e.value.status == status
+    assert B.eqconv_node_product_workspace_bytes(0, 10) == 0
+    assert B.eqconv_double_backward_workspace_bytes(0, 10) == 0
