@@ -480,8 +480,8 @@ def run_native(args, rank, world, local_rank):
         "ms": {"graph": round(med(graph_ms), 4), "fwd": round(med(fwd_ms), 4), "bwd_det": round(med(bwd_ms), 4),
                "bwd_atomic": round(med(nd_ms), 4) if nd_ms else None},
         "roofline": {"bound": "hbm",
-                     "kernel": "eqconv_bwd_kernel (deterministic, fused dr)" if bws_n == 0 else
-                               "eqconv_bwd_kernel (deterministic) + eqconv_dr_epilogue",
+                     "kernel": "eqconv_bwd_kernel (deterministic; dr finished in-kernel when one channel "
+                               "tile covers C, else by eqconv_dr_epilogue)",
                      "achieved": round(bc["bwd"] / (bwd_avg * 1e-3) / 1e9, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(bc["bwd"] / (bwd_avg * 1e-3) / 1e9 / peak, 4),
                      "traffic": traffic.get("bwd"), "algorithmic_bytes": bc["bwd"], "peak_kind": peak_kind},
