@@ -499,21 +499,33 @@ def run_native(args, rank, world, local_rank):
     return result, inp, (N, E, C, D_in, D_out, P)
 
 
+def kernel_code_hash(paths):
+    """sha256 of the kernel sources with comments and blank lines removed, so
+    that a comment edit does not mark the ncu counters stale but any code
+    change does."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+        h.update("\n".join(lines).encode())
+    return h.hexdigest()
+
+
 def load_traffic(workload):
     """DRAM bytes per launch of the forward and the deterministic backward
     for `workload` from the committed ncu summary; empty (so the roofline's
     traffic is null) when absent, when that workload was not captured, or
-    when the kernel sources have changed since the counters were taken."""
-    import hashlib
+    when the kernel code has changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        h = hashlib.sha256()
-        for rel in d["kernel_sources"]:
-            with open(os.path.join(ROOT, rel), "rb") as f:
-                h.update(f.read())
-        if h.hexdigest() != d["kernel_sources_sha256"]:
+        if kernel_code_hash(d["kernel_sources"]) != d["kernel_code_sha256"]:
             return {}
         return d["workloads"].get(workload, {})
     except Exception:

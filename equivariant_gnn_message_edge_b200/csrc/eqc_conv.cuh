@@ -11,17 +11,18 @@
 // Mapping (one warp = one node x one channel tile of 32*VEC channels; each
 // lane owns VEC consecutive channels, so every x / w / y row segment is a
 // coalesced 512 B (VEC=4) run):
-//   * edges are processed in chunks (Cfg::chunk): lane t of the warp reads edge t
-//     of the chunk, evaluates Y(r_e) and the per-edge coupling matrices
+//   * a warp walks its node's edge list in windows of up to 32 edges; lane 0
+//     keeps a 2-stage shared-memory ring filled by TMA bulk copies of each
+//     edge's rows (w_e and the gathered x_s or gy_i) two edges ahead;
+//   * in chunks (Cfg::chunk) lane t evaluates Y(r_e) of edge t and, for the
+//     forward, the per-edge coupling matrices
 //       A_p[m3][m1] = sum_m2 C_p[m1,m2,m3] Y_{l2 m2}(r_e)        (l2 > 0)
-//     with the CG as compile-time immediates (zeros skipped), and stores
-//     them in shared memory; paths with l2 = 0 have A = identity;
-//   * then the warp walks the chunk's edges; every lane reads A (broadcast)
-//     and applies it to its channels, with the next edge's w / x rows loaded
-//     into registers while the current edge is computed;
+//     with the CG as compile-time immediates (zeros skipped) into shared
+//     memory; paths with l2 = 0 have A = identity;
 //   * forward:  acc[l3 m3] += w_p * sum_m1 A_p[m3][m1] x[s, l1 m1]
-//   * backward: t = A_p^T gy_i,  dw_p = x_s . t,  dx_s += w_p t,
-//               gY[l2 m2] += w_p sum_{m1,m3} C_p[m1,m2,m3] x_s[m1] gy_i[m3]
+//   * backward (per channel): h[m1][m2] = sum_m3 C_p[m1,m2,m3] gy_i[m3],
+//               t[m1] = sum_m2 Y[m2] h = (A_p^T gy_i)[m1],  dw_p = x_s . t,
+//               dx_s += w_p t,  gY[l2 m2] += w_p sum_m1 x_s[m1] h
 //     (gY summed over the lane's channels, then across the warp by a fixed
 //     butterfly; dr = (dY/dr)^T gY).
 // Streams (w read, dw written) carry L2 evict-first hints; gathered rows

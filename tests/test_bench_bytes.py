@@ -25,3 +25,14 @@ def test_double_backward_bytes_per_unit():
     per_edge = 8 * P * C + 32 + 12 * P * C + 32 + 36
     per_node = 4 * (2 * D_in + D_out) * C + 4 + 4 * (3 * D_in + D_out) * C + 4
     assert nb == E * per_edge + N * per_node + 8 + 2 * part
+
+
+def test_kernel_code_hash_ignores_comments_only(tmp_path, monkeypatch):
+    src = tmp_path / "k.cuh"
+    src.write_text("// header\nint f(int a) {  // note\n    return a + 1; /* inline */\n}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_code_hash(["k.cuh"])
+    src.write_text("// a longer header\n// over two lines\nint f(int a) {\n\n    return a + 1;\n}\n")
+    assert bench.kernel_code_hash(["k.cuh"]) == h0
+    src.write_text("int f(int a) {\n    return a + 2;\n}\n")
+    assert bench.kernel_code_hash(["k.cuh"]) != h0
