@@ -34,5 +34,6 @@ conv     the convolution: NumPy brute force (per-edge messages) and the C
          variants (both parities, per-path blocks)
 dbl      the double backward (VJP of the backward), NumPy brute force
 nodeprod the node-local channel-diagonal product, forward and backward
+radial   Bessel basis, polynomial envelope and radial MLP with their VJP
 build    compiles ``conv_ref.c`` with gcc
 """
