@@ -177,6 +177,8 @@ class NodeProduct:
     def backward_raw(self, u, v, w, gy, need_dw=True, workspace=None, stream=None):
         N = u.shape[0]
         du, dv = torch.empty_like(u), torch.empty_like(v)
+        if N == 0:      # no nodes: nothing to launch, dw is an empty sum
+            return du, dv, (torch.zeros((self.P, self.C), dtype=torch.float32, device=u.device) if need_dw else None)
         dw = torch.empty((self.P, self.C), dtype=torch.float32, device=u.device) if need_dw else None
         nbytes = B.eqconv_node_product_workspace_bytes(self.plan, N) if need_dw else 0
         if nbytes and workspace is None:

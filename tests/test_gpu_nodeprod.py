@@ -66,8 +66,11 @@ def test_node_product_autograd_and_edge_cases():
     assert_close("du", ut.grad.cpu().numpy(), rdu)
     assert_close("dv", vt.grad.cpu().numpy(), rdv)
     assert_close("dw", wt.grad.cpu().numpy(), rdw)
-    e = op.forward_raw(torch.zeros((0, 9, 64), device="cuda"), torch.zeros((0, 9, 64), device="cuda"))
+    z = torch.zeros((0, 9, 64), device="cuda")
+    e = op.forward_raw(z, z)
     assert e.shape == (0, 9, 64)
+    du0, dv0, dw0 = op.backward_raw(z, z, to_dev(w), z)
+    assert du0.shape == (0, 9, 64) and torch.equal(dw0, torch.zeros_like(dw0))
     with pytest.raises(B.EqconvError) as err:       # both parities are not offered for this op
         B.eqconv_node_product_plan_create("0e+1o", 1, "0e+1o+1e", 8, B.EQCONV_OUT_ALL_PARITY)
     assert err.value.status == B.EQCONV_ERR_UNSUPPORTED
