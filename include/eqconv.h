@@ -16,7 +16,14 @@
  * spherical harmonics, component-normalised (sum_m Y_lm^2 = 2l+1), z polar,
  * m > 0 ~ cos(m phi), m < 0 ~ sin(|m| phi).  Paths are the admissible
  * (l1, l2, l3): |l1 - l2| <= l3 <= l1 + l2 and natural parity, ordered by
- * (l1, l2, l3); paths that land on the same l3 are summed.
+ * (l1, l2, l3); paths that land on the same l3 are summed (by default: see
+ * EQCONV_OUT_ALL_PARITY and EQCONV_OUT_PER_PATH for both-parity outputs and
+ * per-path output blocks).
+ *
+ * Besides the forward and the backward the library has the double backward
+ * (eqconv_double_backward, the VJP of the backward, for training on forces)
+ * and the node-local channel-diagonal product of two node features
+ * (eqconv_node_product*, one step of the correlation ladder).
  *
  * Layout (FlashCart App. D, Figure D1: rank blocks, then components, then
  * channels): every tensor is fp32, row-major, channels innermost.

@@ -188,3 +188,33 @@ def test_node_product_plans_validate_before_device_work():
         assert e.value.status == status
     assert B.eqconv_node_product_workspace_bytes(0, 10) == 0
     assert B.eqconv_double_backward_workspace_bytes(0, 10) == 0
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/eqconv.h compiles as C99 with warnings as errors, and a C
+    program links against libeqconv.so and calls the host-only entry points
+    (no device needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "eqconv.h"
+int main(void) {
+    int P = 0, paths[3 * 64];
+    double cg[7 * 7 * 7];
+    if (eqconv_enumerate_paths("0e+1o+2e", 2, "0e+1o+2e", &P, paths, 64) != EQCONV_OK || P != 11) return 1;
+    if (eqconv_cg_table(1, 1, 0, cg, 343) != EQCONV_OK) return 2;
+    if (eqconv_graph_workspace_bytes(10, 100) == 0) return 3;
+    printf("%d %s\n", P, eqconv_status_string(EQCONV_ERR_UNSUPPORTED));
+    return 0;
+}
+""")
+    libdir = os.path.dirname(B.LIB_PATH)
+    exe = tmp_path / "use"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-o", str(exe), "-L", libdir, "-leqconv", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    assert out.startswith("11 EQCONV_ERR_UNSUPPORTED")
