@@ -151,7 +151,10 @@ class Inputs:
         self.gy = mk((W.N, D_out, W.C), torch.float32)
         self.gy.numpy()[:] = wl.features(W.N, D_out, W.C, wl.SEED_GY)
         self.w = mk((self.E, P, W.C), torch.float32)
-        wl.weights_into(self.w.numpy())
+        if W.kind == "waterbox":           # radial-MLP weights, zero on the padding edges
+            self.w.numpy()[:] = wl.water_box_weights(P, W.C)
+        else:
+            wl.weights_into(self.w.numpy())
 
 
 # --------------------------------------------------------------------- clocks
@@ -464,7 +467,10 @@ def run_native(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded NumPy PCG64)",
         "config": {
             "workload": f"{W.name}: N={N}, C={C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}{layout}, L_sh={W.L_sh}, "
-                        f"P={P}, in-degree Poisson({W.mean_degree:g}), uniform senders",
+                        f"P={P}, " + (f"water box: {W.N} atoms, {W.box:g} A periodic cube, cutoff {W.cutoff:g} A, "
+                                      f"10% zero-weight padding edges, radial-MLP weights (one conv layer)"
+                                      if W.kind == "waterbox" else
+                                      f"in-degree Poisson({W.mean_degree:g}), uniform senders"),
             "step": "graph build (recv+send CSR) + fused forward + fused deterministic backward",
             "l2": "inputs larger than L2 (w alone is %.1f GB)" % (bc["step"] and 4 * E * P * C / 1e9),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

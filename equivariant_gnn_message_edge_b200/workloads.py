@@ -152,6 +152,9 @@ def make_graph(wl: Workload):
     """(senders, receivers, r) for a workload."""
     if wl.kind == "box":
         return periodic_box_graph(wl.N, wl.box, wl.cutoff)
+    if wl.kind == "waterbox":
+        s, rcv, r, _ = water_box_graph()
+        return s, rcv, r
     s, rcv = poisson_graph(wl.N, wl.mean_degree)
     return s, rcv, random_edge_vectors(len(s))
 
@@ -236,3 +239,30 @@ def radial_weights(r: np.ndarray, cutoff: float, params, P: int, C: int, is_dumm
     if is_dummy is not None:
         w[is_dummy] = 0.0
     return w
+
+
+_WATER_GRAPH = None
+
+
+def water_box_graph():
+    """(senders, receivers, r, is_dummy) of the MACE(a)-shaped water box
+    (WATER_BOX settings), built once per process."""
+    global _WATER_GRAPH
+    if _WATER_GRAPH is None:
+        c = WATER_BOX
+        pos = random_sequential_packing(c["n_atoms"], c["box"], c["min_dist"])
+        _WATER_GRAPH = padded_box_graph(pos, c["box"], c["cutoff"], c["pad"])
+    return _WATER_GRAPH
+
+
+def water_box_weights(P: int, C: int) -> np.ndarray:
+    """Radial weights w[E, P, C] of the water box's edges (zero on dummies)."""
+    _, _, r, is_dummy = water_box_graph()
+    params = radial_mlp_params(P, C, WATER_BOX["hidden"], WATER_BOX["n_bessel"])
+    return radial_weights(r, WATER_BOX["cutoff"], params, P, C, is_dummy=is_dummy,
+                          n_bessel=WATER_BOX["n_bessel"])
+
+
+WORKLOADS["waterbox"] = Workload("waterbox", WATER_BOX["n_atoms"], WATER_BOX["C"], _natural(WATER_BOX["L"]),
+                                 WATER_BOX["L"], _natural(WATER_BOX["L"]), "waterbox", box=WATER_BOX["box"],
+                                 cutoff=WATER_BOX["cutoff"])

@@ -43,3 +43,14 @@ def test_weights_into_matches_weights():
     out = np.empty((500, 7, 12), dtype=np.float32)
     wl.weights_into(out, chunk_edges=64)
     assert np.array_equal(out, wl.weights(500, 7, 12, chunk_edges=200))
+
+
+def test_water_box_workload():
+    from equivariant_gnn_message_edge_b200 import workloads as wl
+    W = wl.WORKLOADS["waterbox"]
+    s, rcv, r = wl.make_graph(W)
+    _, _, _, dummy = wl.water_box_graph()
+    assert len(s) == 82909 and int(dummy.sum()) == 7537
+    assert np.all(np.diff(rcv) >= 0)                       # receiver-sorted
+    w = wl.water_box_weights(23, W.C)
+    assert w.shape == (82909, 23, 128) and np.all(w[dummy] == 0.0) and np.all(np.isfinite(w))
