@@ -61,7 +61,7 @@ def byte_counts(N, E, C, D_in, D_out, P):
     return dict(fwd=fwd, bwd=bwd, graph=graph, step=step, h2d=h2d, d2h=d2h, kernels=graph + fwd + bwd)
 
 
-def time_node_product(W, Nn, dev, stream, reps):
+def time_node_product(W, Nn, dev, stream, reps, reduce=lambda t: t):
     """Median device time and GB/s of the node-local product (forward, and
     backward with dw) on Nn nodes; bytes = each tensor read or written once
     per kernel (u, v, w, y; u, v, w, gy, du, dv, dw partials, dw)."""
@@ -92,8 +92,8 @@ def time_node_product(W, Nn, dev, stream, reps):
         ev[2].record(stream)
         fe.append(ev)
     stream.synchronize()
-    f_ms = statistics.median([e[0].elapsed_time(e[1]) for e in fe[1:]])
-    b_ms = statistics.median([e[1].elapsed_time(e[2]) for e in fe[1:]])
+    f_ms = reduce(statistics.median([e[0].elapsed_time(e[1]) for e in fe[1:]]))     # max over ranks
+    b_ms = reduce(statistics.median([e[1].elapsed_time(e[2]) for e in fe[1:]]))
     row = 4 * C * Nn
     fb = row * (op.D_u + op.D_v + op.D_out) + 4 * P * C
     bb = row * (2 * op.D_u + 2 * op.D_v + op.D_out) + 4 * P * C + 2 * nws + 4 * P * C
@@ -380,7 +380,7 @@ def run_native(args, rank, world, local_rank):
         assert B.eqconv_get_device_error(conv.plan, sh) == B.EQCONV_OK
         dbl_ms = [a.elapsed_time(b) for a, b in dbl_ev[1:]]
         nbytes = dbl_bytes(N, E, C, D_in, D_out, P, dws_n)
-        dbl_med = statistics.median(dbl_ms)
+        dbl_med = reduce_max(statistics.median(dbl_ms), world, dev)     # max over ranks
         dbl = {"ms": round(dbl_med, 4), "gbps": round(nbytes / (dbl_med * 1e-3) / 1e9, 1),
                "frac_of_measured_hbm": round(nbytes / (dbl_med * 1e-3) / 1e9 / measured_peak()[0], 4),
                "algorithmic_bytes": nbytes, "launches_per_call": 3,
@@ -391,7 +391,8 @@ def run_native(args, rank, world, local_rank):
     # well above L2), forward and backward, timed separately
     nprod = None
     if not W.all_parity and not args.no_node_product:
-        nprod = time_node_product(W, 4 * N, dev, stream, max(3, args.steps // 2))
+        nprod = time_node_product(W, 4 * N, dev, stream, max(3, args.steps // 2),
+                                  lambda t: reduce_max(t, world, dev))
 
     # End to end through the public API with host buffers (pinned), copies
     # timed: every step uploads its inputs and downloads its results.  Steps
