@@ -94,3 +94,22 @@ def radial_weights_vjp(d, rc: float, params, gw, p: int = P_ENV):
     g_b = g_z1 @ W1.T
     g_d = (g_b * bessel_grad(d, rc, W1.shape[0])).sum(1) + g_u * envelope_grad(d, rc, p)
     return g_d, [g_W1, g_W2, g_W3]
+
+
+def conv_with_radial(prob, N: int, senders, receivers, r, x, rc: float, params, gy=None):
+    """The convolution with its weights produced from the edge lengths by the
+    radial MLP: y = conv(x, r, w(|r|)).  With gy, also the backward through
+    both routes of r: dr = (dY/dr)^T gY + g_d(|r|) r / |r|, plus dx and the
+    MLP weight gradients.  Returns y or (y, dx, dr, [g_W1, g_W2, g_W3])."""
+    from . import conv as oconv
+    r64 = np.asarray(r, dtype=np.float64)
+    d = np.linalg.norm(r64, axis=1)
+    w = radial_weights(d, rc, params, prob.P, prob.C)
+    if gy is None:
+        return oconv.forward_bruteforce(prob, N, senders, receivers, r, x, w)
+    y = oconv.forward_bruteforce(prob, N, senders, receivers, r, x, w)
+    dx, dw, dr_ang = oconv.backward_bruteforce(prob, N, senders, receivers, r, x, w, gy)
+    g_d, g_W = radial_weights_vjp(d, rc, params, dw)
+    safe = np.where(d > 0, d, 1.0)
+    dr = dr_ang + (g_d / safe)[:, None] * r64 * (d > 0)[:, None]
+    return y, dx, dr, g_W

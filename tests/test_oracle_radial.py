@@ -98,3 +98,36 @@ def test_water_box_generator_matches_the_oracle():
     ref[dummy] = 0.0
     assert np.max(np.abs(w - ref)) < 1e-5 * np.max(np.abs(ref)) + 1e-6
     assert np.all(w[dummy] == 0.0)
+
+
+def test_conv_with_radial_weights_backward_matches_differences():
+    """The fused path's oracle: y = conv(x, r, w(|r|)); the gradient of
+    <gy, y> in r has an angular part (harmonics) and a radial part (the MLP),
+    and in the MLP weights; central differences of the composition check
+    both routes (everything fp64)."""
+    from oracle.conv import Problem
+    prob = Problem("0e+1o+2e", 2, "0e+1o+2e", 3)
+    rng = np.random.default_rng(9)
+    N, E = 6, 20
+    s = rng.integers(0, N, E).astype(np.int32)
+    rcv = rng.integers(0, N, E).astype(np.int32)
+    r = rng.standard_normal((E, 3)) * 1.5
+    x = rng.standard_normal((N, prob.D_in, 3))
+    gy = rng.standard_normal((N, prob.D_out, 3))
+    params = _params(prob.P, prob.C, seed=10)
+    y, dx, dr, g_W = R.conv_with_radial(prob, N, s, rcv, r, x, RC, params, gy)
+
+    def S(rr, pp):
+        return float((gy * R.conv_with_radial(prob, N, s, rcv, rr, x, RC, pp)).sum())
+    h = 1e-5
+    dirn = rng.standard_normal(r.shape)
+    fd = (S(r + h * dirn, params) - S(r - h * dirn, params)) / (2 * h)
+    assert abs(fd - (dr * dirn).sum()) < 1e-4 * max(1.0, abs(fd))
+    for k in range(3):
+        dW = rng.standard_normal(params[k].shape)
+        pp = [W.copy() for W in params]
+        pm = [W.copy() for W in params]
+        pp[k] += h * dW
+        pm[k] -= h * dW
+        fd = (S(r, pp) - S(r, pm)) / (2 * h)
+        assert abs(fd - (g_W[k] * dW).sum()) < 1e-4 * max(1.0, abs(fd))
