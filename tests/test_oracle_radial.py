@@ -13,7 +13,6 @@ Table 3: 8 radial functions, 5 Angstrom cutoff.  What pins the oracle:
 * the seeded water-box generator gives the oracle's weights (fp32).
 """
 import numpy as np
-import pytest
 import torch
 from numpy.polynomial import Polynomial
 
