@@ -128,3 +128,48 @@ def test_double_backward_mistakes_fail_the_difference_pins():
         code = src.replace(good, bad).replace("from .conv import", "from oracle.conv import")
         exec(compile(code.replace("from .sh import", "from oracle.sh import"), "planted", "exec"), ns)
         assert expect.strip() in _dbl_fd_failures(ns["double_backward_bruteforce"])
+
+
+def test_variant_mistakes_fail_the_variant_pins():
+    """Both-parity and per-path outputs: taking the real part for an odd
+    path (which is zero, so the pseudo-tensor block vanishes), or swapping
+    the output blocks of two paths of opposite parity, each fail a pin of
+    test_oracle_modes.py (the cross product; the inversion signs)."""
+    from equivariant_gnn_message_edge_b200.workloads import both_parity_irreps, natural_irreps
+    # (1) odd coupling taken as the real part: the cross-product pin fails
+    real = cgmod._real_cg_cached.__wrapped__
+
+    def real_part(l1, l2, l3):
+        C = real(l1, l2, l3)
+        return np.zeros_like(C) if (l1 + l2 + l3) % 2 else C
+    C_bad = real_part(1, 1, 1)
+    u, v = np.array([0.3, -1.0, 0.4]), np.array([1.1, 0.2, -0.7])
+    perm = [1, 2, 0]
+    want = np.cross(u, v)[perm] / np.sqrt(2.0)
+    assert np.max(np.abs(np.abs(np.einsum("abk,a,b->k", C_bad, u[perm], v[perm])) - np.abs(want))) > 1e-3
+    # (2) two per-path blocks of the same size but opposite parity swapped
+    # ((1,1,2) -> 2e and (2,1,2) -> 2o): the inversion-sign pin fails
+    from tests.helpers import parity_signs
+    N = 6
+    pp = conv.Problem(natural_irreps(2), 2, both_parity_irreps(2), 3, per_path=True)
+    rng = np.random.default_rng(1)
+    s = rng.integers(0, N, 30).astype(np.int32)
+    rcv = rng.integers(0, N, 30).astype(np.int32)
+    r = rng.standard_normal((30, 3))
+    x = rng.standard_normal((N, pp.D_in, 3))
+    w = rng.standard_normal((30, pp.P, 3))
+    pin, pout = parity_signs(pp.irreps_in), parity_signs(pp.layout_out)
+
+    def parity_error():
+        y = conv.forward_bruteforce(pp, N, s, rcv, r, x, w)
+        y_inv = conv.forward_bruteforce(pp, N, s, rcv, -r, pin[None, :, None] * x, w)
+        return np.max(np.abs(y_inv - pout[None, :, None] * y)) / np.max(np.abs(y))
+    assert parity_error() < 1e-12
+    a = next(k for k, q in enumerate(pp.paths) if (q["l1"], q["l2"], q["l3"]) == (1, 1, 2))
+    b = next(k for k, q in enumerate(pp.paths) if (q["l1"], q["l2"], q["l3"]) == (2, 1, 2))
+    qa, qb = pp.paths[a], pp.paths[b]
+    qa["off3"], qb["off3"] = qb["off3"], qa["off3"]
+    try:
+        assert parity_error() > 1e-3
+    finally:
+        qa["off3"], qb["off3"] = qb["off3"], qa["off3"]
