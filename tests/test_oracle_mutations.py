@@ -173,3 +173,36 @@ def test_variant_mistakes_fail_the_variant_pins():
         assert parity_error() > 1e-3
     finally:
         qa["off3"], qb["off3"] = qb["off3"], qa["off3"]
+
+
+def test_node_product_mistakes_fail_the_derivative_pin():
+    """In the node-local product's backward, a flipped sign in dv or a
+    dropped weight in du fails the exact directional-derivative pin."""
+    import inspect
+    from oracle import nodeprod
+    from tests.test_oracle_nodeprod import _setup
+    src = inspect.getsource(nodeprod)
+    prob, u, v, w, gy = _setup(2, 2, 2, seed=6)
+
+    def fails(mod_src):
+        ns = {}
+        exec(compile(mod_src.replace("from .conv import", "from oracle.conv import"), "planted", "exec"), ns)
+        du, dv, dw = ns["node_product_backward"](prob, u, v, w, gy)
+        S = lambda uu, vv, ww: float((gy * nodeprod.node_product(prob, uu, vv, ww)).sum())
+        s0 = S(u, v, w)
+        rng = np.random.default_rng(3)
+        bad = []
+        for name, g in (("u", du), ("v", dv), ("w", dw)):
+            d = rng.standard_normal(g.shape)
+            args = dict(u=u, v=v, w=w)
+            args[name] = args[name] + d
+            if abs(S(args["u"], args["v"], args["w"]) - s0 - (g * d).sum()) > 1e-8 * max(1.0, abs(s0)):
+                bad.append(name)
+        return bad
+    assert fails(src) == []
+    good = 'dv[:, q["off2"]:q["off2"] + d2, :] += w[p] * '
+    assert good in src
+    assert "v" in fails(src.replace(good, 'dv[:, q["off2"]:q["off2"] + d2, :] -= w[p] * '))
+    good = 'du[:, q["off1"]:q["off1"] + d1, :] += w[p] * '
+    assert good in src
+    assert "u" in fails(src.replace(good, 'du[:, q["off1"]:q["off1"] + d1, :] += '))
