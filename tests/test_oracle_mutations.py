@@ -206,3 +206,31 @@ def test_node_product_mistakes_fail_the_derivative_pin():
     good = 'du[:, q["off1"]:q["off1"] + d1, :] += w[p] * '
     assert good in src
     assert "u" in fails(src.replace(good, 'du[:, q["off1"]:q["off1"] + d1, :] += '))
+
+
+def test_radial_mistakes_fail_the_radial_pins():
+    """In the radial weights' VJP, a dropped envelope-derivative term or a
+    missing SiLU derivative fails the central-difference / autograd pins."""
+    import inspect
+    from oracle import radial
+    from tests.test_oracle_radial import RC, _params
+    src = inspect.getsource(radial)
+    P, C = 2, 3
+    params = _params(P, C, seed=4)
+    rng = np.random.default_rng(5)
+    d = rng.uniform(0.5, 4.9, 20)
+    gw = rng.standard_normal((20, P, C))
+
+    def err(mod_src):
+        ns = {}
+        exec(compile(mod_src, "planted", "exec"), ns)
+        g_d, _ = ns["radial_weights_vjp"](d, RC, params, gw)
+        h = 1e-6
+        fd = ((radial.radial_weights(d + h, RC, params, P, C) - radial.radial_weights(d - h, RC, params, P, C)) *
+              gw).sum((1, 2)) / (2 * h)
+        return np.max(np.abs(fd - g_d)) / max(1.0, np.max(np.abs(fd)))
+    assert err(src) < 1e-6
+    good = " + g_u * envelope_grad(d, rc, p)"
+    assert good in src and err(src.replace(good, "")) > 1e-3
+    good = "g_z2 = (g_z3 @ W3.T) * _silu_grad(z2)"
+    assert good in src and err(src.replace(good, "g_z2 = (g_z3 @ W3.T)")) > 1e-3
