@@ -54,11 +54,41 @@ def byte_counts(N, E, C, D_in, D_out, P):
     fwd = sum(t[k] for k in ("x", "r", "w", "recv_ptr", "recv_perm", "senders", "y"))
     bwd = sum(t[k] for k in ("x", "r", "w", "gy", "send_ptr", "send_perm", "receivers", "dx", "dw", "dr"))
     graph = sum(t[k] for k in ("senders", "receivers", "recv_ptr", "recv_perm", "send_ptr", "send_perm"))
+    # the step's unique bytes: every tensor the step reads or writes counted
+    # once over the whole step (graph build + forward + backward) - the
+    # headline; `kernels` counts each kernel's own tensors (the roofline's)
     step = sum(t.values())
     h2d = sum(t[k] for k in ("senders", "receivers", "x", "r", "w", "gy"))
     d2h = sum(t[k] for k in ("y", "dx", "dw", "dr"))
-    # headline bytes: each kernel's own inputs and outputs, each counted once
     return dict(fwd=fwd, bwd=bwd, graph=graph, step=step, h2d=h2d, d2h=d2h, kernels=graph + fwd + bwd)
+
+
+FP32_PEAK_SM_MHZ = 1965.0     # clocks.max.sm of the B200s this runs on
+
+
+def fp32_peak_tflops(sm_mhz=FP32_PEAK_SM_MHZ):
+    """FP32 FMA peak: 148 SMs x 128 FMA lanes x 2 flop x clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def fma_counts(paths, cg_table):
+    """FMA per (edge, channel) of the forward and of the backward's h-form
+    contraction as the kernels issue them, counted from the real CG tables
+    (zero coefficients are skipped at compile time).  cg_table(l1, l2, l3)
+    gives the [2l1+1][2l2+1][2l3+1] table."""
+    fwd = bwd = 0
+    for l1, l2, l3 in paths:
+        d1, d2, d3 = 2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1
+        if l2 == 0:
+            fwd += d1
+            bwd += 2 * d1                      # dw = x . g, dx += w g
+            continue
+        fwd += d1 * d3 + min(d1, d3)           # A x (d3 x d1), then the weight
+        t = np.asarray(cg_table(l1, l2, l3))
+        nz = np.abs(t) > 0
+        rows = int(nz.any(axis=2).sum())       # (m1, m2) rows with a nonzero coefficient
+        bwd += int(nz.sum()) + 2 * rows + 2 * d1 + d2
+    return fwd, bwd
 
 
 def time_node_product(W, Nn, dev, stream, reps, reduce=lambda t: t):
@@ -104,6 +134,172 @@ def time_node_product(W, Nn, dev, stream, reps, reduce=lambda t: t):
             "bwd_frac_of_measured_hbm": round(bb / (b_ms * 1e-3) / 1e9 / peak, 4),
             "bytes": "fwd: u, v, w read, y written; bwd: u, v, w, gy read, du, dv written, dw partials written "
                      "and read, dw written"}
+
+
+def device_inputs(W, D_in, D_out, P, dev, seed_offset=0):
+    """Graph of workload W from the seeded NumPy generators; features, weights
+    and output gradients drawn on the device by a seeded torch generator with
+    the stated laws (x, gy ~ N(0, 1), w ~ N(0, 1/P)), which is much faster
+    than drawing several GB on the host.  Returns (s, rcv, r, x, w, gy)."""
+    import torch
+    s, rcv, r = wl.make_graph(W)
+    gen = torch.Generator(device=dev).manual_seed(wl.SEED_X + 100 + seed_offset)
+    E = len(s)
+    x = torch.randn((W.N, D_in, W.C), generator=gen, device=dev)
+    w = torch.randn((E, P, W.C), generator=gen, device=dev).mul_(1.0 / np.sqrt(P))
+    gy = torch.randn((W.N, D_out, W.C), generator=gen, device=dev)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    return to(s), to(rcv), to(r), x, w, gy
+
+
+def conv_leg(name, dev, stream, reps, reduce, atomic=True, warmup=3):
+    """One of the stated convolution workloads timed kernel by kernel: the
+    forward, the deterministic backward and (atomic=True) the atomic
+    backward, each median over `reps` launches (max over ranks), with its
+    HBM roofline (each kernel's tensors counted once, against the measured
+    copy peak) and its FP32 issue fraction (FMAs counted from the CG tables,
+    against the FP32 FMA peak at the maximum SM clock)."""
+    import torch
+
+    from equivariant_gnn_message_edge_b200 import binding as B
+    from equivariant_gnn_message_edge_b200.conv import EqConv
+    W = wl.WORKLOADS[name]
+    conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C, all_parity=W.all_parity, per_path=W.per_path)
+    P, D_in, D_out = conv.P, conv.D_in, conv.D_out
+    with torch.cuda.stream(stream):
+        s, rcv, r, x, w, gy = device_inputs(W, D_in, D_out, P, dev)
+        g = conv.graph(s, rcv, W.N, stream=stream)
+        y, dx, dw, dr = (torch.empty((W.N, D_out, W.C), device=dev), torch.empty_like(x), torch.empty_like(w),
+                         torch.empty_like(r))
+        nws = B.eqconv_backward_workspace_bytes(conv.plan, g.E)
+        ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+    h = stream.cuda_stream
+    modes = [("fwd", None), ("bwd_det", B.EQCONV_DETERMINISTIC)] + ([("bwd_atomic", 0)] if atomic else [])
+    times = {}
+    for key, flag in modes:
+        evs = []
+        for k in range(warmup + reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            if flag is None:
+                B.eqconv_forward(conv.plan, g.c, x, r, w, y, 0, h)
+            else:
+                B.eqconv_backward(conv.plan, g.c, x, r, w, gy, dx, dw, dr, ws, nws, flag, h)
+            b.record(stream)
+            if k >= warmup:
+                evs.append((a, b))
+        stream.synchronize()
+        times[key] = reduce(statistics.median([a.elapsed_time(b) for a, b in evs]))
+    assert B.eqconv_get_device_error(conv.plan, h) == B.EQCONV_OK
+    bc = byte_counts(W.N, g.E, W.C, D_in, D_out, P)
+    fma_f, fma_b = fma_counts(conv.paths, B.eqconv_cg_table)
+    peak, peak_kind = measured_peak()
+    fpk = fp32_peak_tflops()
+    out = {"N": W.N, "E": g.E, "C": W.C, "P": P, "irreps": f"{W.irreps_in} -> {W.irreps_out}", "L_sh": W.L_sh,
+           "ms": {k: round(v, 4) for k, v in times.items()},
+           "fma_per_edge_channel": {"fwd": fma_f, "bwd": fma_b}}
+    for key in times:
+        nbytes = bc["fwd"] if key == "fwd" else bc["bwd"]
+        fma = fma_f if key == "fwd" else fma_b
+        sec = times[key] * 1e-3
+        gbs = nbytes / sec / 1e9
+        tfl = 2.0 * fma * g.E * W.C / sec / 1e12
+        out[key] = {"gbps": round(gbs, 1), "edges_per_s": round(g.E / sec, 1),
+                    "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                                 "frac": round(gbs / peak, 4), "traffic": None, "algorithmic_bytes": nbytes,
+                                 "peak_kind": peak_kind},
+                    "roofline_fp32": {"bound": "alu", "achieved": round(tfl, 2), "peak": round(fpk, 2),
+                                      "unit": "TFLOP/s", "frac": round(tfl / fpk, 4),
+                                      "flop": "2 x FMA per (edge, channel) from the CG tables x E x C"}}
+    fb = (bc["fwd"] + bc["bwd"]) / ((times["fwd"] + times["bwd_det"]) * 1e-3) / 1e9
+    out["fwd_bwd_gbps_per_kernel_bytes"] = round(fb, 1)
+    # every tensor of forward + backward counted once (the edge layout included)
+    out["fwd_bwd_gbps_unique_bytes"] = round(bc["step"] / ((times["fwd"] + times["bwd_det"]) * 1e-3) / 1e9, 1)
+    out["fwd_bwd_frac_unique"] = round(out["fwd_bwd_gbps_unique_bytes"] / peak, 4)
+    del x, w, gy, y, dx, dw, dr, ws, g
+    torch.cuda.empty_cache()
+    return out
+
+
+def radial_weights_torch(r, rc, params, P, C):
+    """w[E, P, C] = u(d) * MLP(b(d)) with d = |r| in fp32 torch ops (cuBLAS
+    GEMMs for the layers): the unfused radial path the water-box step uses
+    as its baseline.  The same Bessel basis, C2 polynomial envelope (p = 6)
+    and bias-free SiLU MLP as the seeded workload."""
+    import torch
+    d = torch.linalg.vector_norm(r, dim=1)
+    n = torch.arange(1, params[0].shape[0] + 1, device=r.device, dtype=r.dtype)
+    x = (d / rc).clamp(0.0, 1.0)
+    p = 6.0
+    env = (1.0 - (p + 1) * (p + 2) / 2 * x ** 6 + p * (p + 2) * x ** 7 - p * (p + 1) / 2 * x ** 8)
+    bes = (2.0 / rc) ** 0.5 * torch.sin(n[None, :] * (np.pi / rc) * d[:, None]) / d.clamp_min(1e-9)[:, None]
+    h = torch.nn.functional.silu(bes @ params[0])
+    h = torch.nn.functional.silu(h @ params[1])
+    return (env[:, None] * (h @ params[2])).view(-1, P, C)
+
+
+def waterbox_leg(dev, stream, reps, reduce, warmup=3):
+    """The MACE(a)-shaped water box step as stated: two stacked conv layers
+    (C = 128, L = 3) with radial-MLP weights (8 Bessel functions, 8 -> 64 ->
+    64 -> P*C SiLU MLP, a seeded set per layer), layer 2 fed y1 / <degree>,
+    an energy-like readout E = <gy, y2>, then the gradient of E with respect
+    to the 1503 positions (forces) through both routes of every edge vector
+    (the harmonics and the radial weights) and to both MLPs' weights.
+    Timed on the device per step, L2 flushed between steps (the box's inputs
+    fit in L2)."""
+    import torch
+
+    from equivariant_gnn_message_edge_b200 import binding as B
+    from equivariant_gnn_message_edge_b200.conv import EqConv
+    cfg = wl.WATER_BOX
+    ins = wl.natural_irreps(cfg["L"])
+    C, N, rc = cfg["C"], cfg["n_atoms"], cfg["cutoff"]
+    conv = EqConv(ins, cfg["L"], ins, C)
+    P = conv.P
+    pos, s, rcv, shift, dummy = wl.water_box_system()
+    avg = float((~dummy).sum()) / N
+    torch.backends.cuda.matmul.allow_tf32 = False
+    to = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    with torch.cuda.stream(stream):
+        s_d, r_d = to(s, torch.int32), to(rcv, torch.int32)
+        g = conv.graph(s_d, r_d, N, stream=stream)
+        pos_d, shift_d = to(pos), to(shift)
+        s_l, r_l = s_d.long(), r_d.long()
+        params = [[to(p) for p in wl.radial_mlp_params(P, C, cfg["hidden"], cfg["n_bessel"], seed=wl.SEED_W + 10 * k)]
+                  for k in range(2)]
+        x1 = to(wl.features(N, conv.D_in, C, wl.SEED_X))
+        readout = to(wl.features(N, conv.D_out, C, wl.SEED_GY))
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        p = pos_d.detach().requires_grad_(True)
+        Ws = [[t.detach().requires_grad_(True) for t in ps] for ps in params]
+        r = p[s_l] - p[r_l] + shift_d
+        y1 = conv(g, x1, r, radial_weights_torch(r, rc, Ws[0], P, C))
+        y2 = conv(g, y1 / avg, r, radial_weights_torch(r, rc, Ws[1], P, C))
+        e = (y2 * readout).sum()
+        grads = torch.autograd.grad(e, [p] + Ws[0] + Ws[1])
+        return grads
+
+    ms = []
+    with torch.cuda.stream(stream):
+        for k in range(warmup + reps):
+            flush.fill_(k & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b.record(stream)
+            if k >= warmup:
+                ms.append((a, b))
+    stream.synchronize()
+    assert B.eqconv_get_device_error(conv.plan, stream.cuda_stream) == B.EQCONV_OK
+    t = reduce(statistics.median([a.elapsed_time(b) for a, b in ms]))
+    return {"atoms": N, "edges": int(len(s)), "dummy_edges": int(dummy.sum()), "C": C, "L": cfg["L"], "P": P,
+            "unfused_ms_per_step": round(t, 4),
+            "unfused": "radial MLP in fp32 torch ops (cuBLAS GEMMs, TF32 off) writing w [E][P][C] to HBM per "
+                       "layer + libeqconv forward/backward (deterministic) + torch autograd glue",
+            "step": "2 conv layers forward + gradient of <gy, y2> w.r.t. positions (forces) and MLP weights; "
+                    "L2 flushed between steps"}
 
 
 def dbl_bytes(N, E, C, D_in, D_out, P, part_bytes):
@@ -443,20 +639,36 @@ def run_native(args, rank, world, local_rank):
         b.record(down)
         torch.cuda.synchronize(dev)
         e_ms = reduce_max(a.elapsed_time(b), world, dev)
-        e2e = {"value": round(aggregate_gbs(bc["kernels"], e2e_steps, world, e_ms), 2), "unit": UNIT,
+        e2e = {"value": round(aggregate_gbs(bc["step"], e2e_steps, world, e_ms), 2), "unit": UNIT,
                "h2d_bytes_per_step": bc["h2d"], "d2h_bytes_per_step": bc["d2h"],
                "ms_per_step": round(e_ms / e2e_steps, 3),
                "pipeline": "2 device sets; upload / compute / download streams overlap across steps"}
         del sets[1]
 
+    # the other stated workloads, timed kernel by kernel after the main
+    # step: lmax=3 with both backward modes, the channel sweep at lmax=2, and
+    # the water-box step
+    legs = {}
+    want = set(args.legs.split(",")) if args.legs else set()
+    red = lambda t: reduce_max(t, world, dev)
+    reps = max(5, args.steps // 2)
+    if "lmax3" in want:
+        legs["lmax3"] = conv_leg("lmax3", dev, stream, reps, red, atomic=True)
+    if "sweep" in want:
+        legs["sweepC"] = [conv_leg(f"sweepC{c}", dev, stream, reps, red, atomic=False)
+                          for c in (64, 128, 256, 512, 1024)]
+    if "waterbox" in want:
+        legs["waterbox"] = waterbox_leg(dev, stream, reps, red)
+
     peak, peak_kind = measured_peak()
     ms_step = t_max / args.steps
     med = statistics.median
-    value = aggregate_gbs(bc["kernels"], args.steps, world, t_max)
-    unique_gbs = aggregate_gbs(bc["step"], args.steps, world, t_max)
+    value = aggregate_gbs(bc["step"], args.steps, world, t_max)           # unique bytes of the step
+    kernel_gbs = aggregate_gbs(bc["kernels"], args.steps, world, t_max)   # each kernel's own tensors
     fwd_gbs = bc["fwd"] / (med(fwd_ms) * 1e-3) / 1e9
     bwd_gbs = bc["bwd"] / (med(bwd_ms) * 1e-3) / 1e9
     fb_gbs = (bc["fwd"] + bc["bwd"]) / ((med(fwd_ms) + med(bwd_ms)) * 1e-3) / 1e9
+    fwdbwd_unique_gbs = bc["step"] / ((med(fwd_ms) + med(bwd_ms)) * 1e-3) / 1e9
     bwd_avg = sum(bwd_ms) / len(bwd_ms)
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
     layout = f" (per-path blocks, D_out={D_out})" if W.per_path else ""
@@ -466,22 +678,14 @@ def run_native(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded NumPy PCG64)",
-        "config": {
-            "workload": f"{W.name}: N={N}, C={C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}{layout}, L_sh={W.L_sh}, "
-                        f"P={P}, " + (f"water box: {W.N} atoms, {W.box:g} A periodic cube, cutoff {W.cutoff:g} A, "
-                                      f"10% zero-weight padding edges, radial-MLP weights (one conv layer)"
-                                      if W.kind == "waterbox" else
-                                      f"in-degree Poisson({W.mean_degree:g}), uniform senders"),
-            "step": "graph build (recv+send CSR) + fused forward + fused deterministic backward",
-            "l2": "inputs larger than L2 (w alone is %.1f GB)" % (bc["step"] and 4 * E * P * C / 1e9),
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "bytes_per_step": bc["kernels"],
-            "bytes": "per kernel: every tensor it reads or writes, counted once (graph build + forward + "
-                     "backward); GB/s = bytes / device time",
-        },
-        "unique_bytes_step_gbps": round(unique_gbs, 1),
-        "fwd_gbps": round(fwd_gbs, 1), "bwd_gbps": round(bwd_gbs, 1), "fwd_bwd_gbps": round(fb_gbs, 1),
-        "hbm_frac_fwd_bwd": round(fb_gbs / peak, 4),
+        "config": step_config(W, N, E, C, D_in, D_out, P, world, layout),
+        "kernel_bytes_step_gbps": round(kernel_gbs, 1),
+        "kernel_bytes_per_step": bc["kernels"],
+        "fwd_gbps": round(fwd_gbs, 1), "bwd_gbps": round(bwd_gbs, 1),
+        "fwd_bwd_gbps_unique": round(fwdbwd_unique_gbs, 1),
+        "hbm_frac_fwd_bwd_unique": round(fwdbwd_unique_gbs / peak, 4),
+        "fwd_bwd_gbps_per_kernel_bytes": round(fb_gbs, 1),
+        "hbm_frac_fwd_bwd_per_kernel_bytes": round(fb_gbs / peak, 4),
         "edges_per_s_fwd": round(E / (med(fwd_ms) * 1e-3), 1),
         "edges_per_s_fwd_bwd": round(E / ((med(fwd_ms) + med(bwd_ms)) * 1e-3), 1),
         "ms": {"graph": round(med(graph_ms), 4), "fwd": round(med(fwd_ms), 4), "bwd_det": round(med(bwd_ms), 4),
@@ -498,12 +702,31 @@ def run_native(args, rank, world, local_rank):
                          "algorithmic_bytes": bc["fwd"]},
         "double_backward": dbl,
         "node_product": nprod,
+        "workloads": legs,
         "gpu_launches": int(launches),
         "clocks": clk.summary((w0, w1)),
     }
     if e2e:
         result["e2e"] = e2e
     return result, inp, (N, E, C, D_in, D_out, P)
+
+
+def step_config(W, N, E, C, D_in, D_out, P, world, layout=""):
+    """The `config` object of the JSON line; the same for both arms."""
+    bc_step = byte_counts(N, E, C, D_in, D_out, P)["step"]
+    return {
+        "workload": f"{W.name}: N={N}, C={C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}{layout}, L_sh={W.L_sh}, "
+                    f"P={P}, " + (f"water box: {W.N} atoms, {W.box:g} A periodic cube, cutoff {W.cutoff:g} A, "
+                                  f"10% zero-weight padding edges, radial-MLP weights (one conv layer)"
+                                  if W.kind == "waterbox" else
+                                  f"in-degree Poisson({W.mean_degree:g}), uniform senders"),
+        "step": "graph build (recv+send CSR) + fused forward + fused deterministic backward",
+        "l2": "inputs larger than L2 (w alone is %.1f GB)" % (4 * E * P * C / 1e9),
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        "bytes_per_step": bc_step,
+        "bytes": "unique: every tensor the step reads or writes (senders, receivers, CSR arrays, x, r, w, gy, "
+                 "y, dx, dw, dr) counted once over the whole step; GB/s = bytes / device time",
+    }
 
 
 def kernel_code_hash(paths):
@@ -611,16 +834,14 @@ def run_reference(args, rank, world):
         t, k = oracle_sample_step(args.workload, n_recv, prob.D_in, prob.D_out, prob.P, x, gy)
         tot += t
     frac = k / E
-    value = bc["kernels"] * frac * args.steps / tot / 1e9
+    value = bc["step"] * frac * args.steps / tot / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot / args.steps, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded NumPy PCG64)",
-        "config": {"workload": f"{W.name}: N={W.N}, C={W.C}, E={E}, irreps {W.irreps_in} -> {W.irreps_out}"
-                               f"{' (per-path blocks)' if W.per_path else ''}, "
-                               f"L_sh={W.L_sh}, P={prob.P}",
-                   "step": "graph build + forward + backward (dx, dw, dr), oracle on a bounded sample"},
+        "config": step_config(W, W.N, E, W.C, prob.D_in, prob.D_out, prob.P, world,
+                              f" (per-path blocks, D_out={prob.D_out})" if W.per_path else ""),
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oconv.max_threads(), "kind": "oracle",
                          "sample": f"in-edges of receivers 0..{n_recv - 1} ({k} of {E} edges) per step; "
                                    f"bytes scaled by {frac:.5f}"},
@@ -647,6 +868,9 @@ def main():
     ap.add_argument("--no-node-product", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
+    ap.add_argument("--legs", default="lmax3,sweep,waterbox",
+                    help="other stated workloads to time after the main step (comma list of lmax3, sweep, "
+                         "waterbox; empty for none)")
     ap.add_argument("--nodes", type=int, default=None,
                     help="override the workload's node count (smaller profiling captures)")
     args = ap.parse_args()
@@ -682,7 +906,7 @@ def main():
             obuild.build()
             N, E, C, D_in, D_out, P = dims
             result["cpu_baseline"] = cpu_baseline(args.workload, D_in, D_out, P, args.cpu_seconds,
-                                                  byte_counts(N, E, C, D_in, D_out, P)["kernels"], E)
+                                                  byte_counts(N, E, C, D_in, D_out, P)["step"], E)
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:

@@ -37,7 +37,7 @@ ABI_FUNCTIONS = (
     "eqconv_plan_create_ex", "eqconv_plan_path_rows", "eqconv_enumerate_paths_ex",
     "eqconv_double_backward_workspace_bytes", "eqconv_double_backward",
     "eqconv_node_product_plan_create", "eqconv_node_product", "eqconv_node_product_workspace_bytes",
-    "eqconv_node_product_backward",
+    "eqconv_node_product_backward", "eqconv_radial_workspace_bytes", "eqconv_radial_weights",
 )
 
 
@@ -88,6 +88,8 @@ _SIGS = {
     "eqconv_node_product_workspace_bytes": (_sz, [_vp, _ci]),
     "eqconv_node_product_backward": (_ci, [_vp, _ci] + [_vp] * 8 + [_sz, _vp]),
     "eqconv_spherical_harmonics": (_ci, [_vp, _ci, _vp, _vp, _vp]),
+    "eqconv_radial_workspace_bytes": (_sz, [_vp, _ci]),
+    "eqconv_radial_weights": (_ci, [_vp, _ci] + [_vp] * 4 + [_ci, ctypes.c_float, _vp, _vp, _sz, _vp]),
     "eqconv_get_device_error": (_ci, [_vp, _vp, _pi]),
     "eqconv_plan_destroy": (None, [_vp]),
     "eqconv_status_string": (ctypes.c_char_p, [_ci]),
@@ -307,6 +309,18 @@ def eqconv_node_product_backward(plan: int, N: int, u, v, w, gy, du, dv, dw, wor
     _check(lib().eqconv_node_product_backward(plan, int(N), _ptr(u, f), _ptr(v, f), _ptr(w, f), _ptr(gy, f),
                                               _ptr(du, f), _ptr(dv, f), _ptr(dw, f), _ptr(workspace),
                                               int(workspace_bytes), _stream(stream)), "eqconv_node_product_backward")
+
+
+def eqconv_radial_workspace_bytes(plan: int, E: int) -> int:
+    return int(lib().eqconv_radial_workspace_bytes(plan, int(E)))
+
+
+def eqconv_radial_weights(plan: int, E: int, r, W1, W2, W3, n_basis: int, r_cut: float, w, workspace,
+                          workspace_bytes: int, stream=None) -> None:
+    f = _f32()
+    _check(lib().eqconv_radial_weights(plan, int(E), _ptr(r, f), _ptr(W1, f), _ptr(W2, f), _ptr(W3, f),
+                                       int(n_basis), float(r_cut), _ptr(w, f), _ptr(workspace),
+                                       int(workspace_bytes), _stream(stream)), "eqconv_radial_weights")
 
 
 def eqconv_spherical_harmonics(plan: int, E: int, r, Y, stream=None) -> None:

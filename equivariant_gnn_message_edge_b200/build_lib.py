@@ -5,6 +5,10 @@
 Each .cu under csrc/ is compiled to an object in _build/ (in parallel; objects
 newer than every source and header are reused) and linked into
 equivariant_gnn_message_edge_b200/libeqconv.so with the static CUDA runtime.
+
+The .cu files under csrc/testing/ are test-only builds of library kernels with
+changed constants (see each file's header); each becomes its own small
+library lib<name>.so beside libeqconv.so, used only by tests/.
 """
 from __future__ import annotations
 
@@ -22,6 +26,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libeqconv.so")
+TESTING = os.path.join(CSRC, "testing")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-std=c++17", "-O3", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
@@ -57,6 +62,8 @@ def _deps(path: str, seen=None) -> set:
 
 def _compile(src: str, force: bool, verbose: bool) -> str:
     obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+    if os.path.dirname(src) == TESTING:
+        obj = os.path.join(BUILD, "testing_" + os.path.basename(src)[:-3] + ".o")
     if not force and os.path.exists(obj):
         t = os.path.getmtime(obj)
         if all(t > os.path.getmtime(d) for d in _deps(src)):
@@ -86,7 +93,27 @@ def build(jobs: int | None = None, force: bool = False, verbose: bool = False) -
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
         os.replace(tmp, LIB)
+    build_testing(force, verbose)
     return LIB
+
+
+def build_testing(force: bool = False, verbose: bool = False) -> list:
+    """Test-only libraries: csrc/testing/<name>.cu + the tensor-map encoder ->
+    lib<name>.so in the package directory."""
+    out = []
+    tmap = _compile(os.path.join(CSRC, "eqc_tmap.cu"), False, verbose)
+    for src in sorted(glob.glob(os.path.join(TESTING, "*.cu"))):
+        obj = _compile(src, force, verbose)
+        lib = os.path.join(PKG, "lib" + os.path.basename(src)[:-3] + ".so")
+        if force or not os.path.exists(lib) or os.path.getmtime(lib) < max(os.path.getmtime(obj),
+                                                                             os.path.getmtime(tmap)):
+            tmp = lib + f".tmp{os.getpid()}"
+            r = subprocess.run([_nvcc()] + ARCH + ["-shared", "-o", tmp, obj, tmap], capture_output=True, text=True)
+            if r.returncode != 0:
+                raise RuntimeError(f"link failed ({lib}):\n{r.stdout}\n{r.stderr}")
+            os.replace(tmp, lib)
+        out.append(lib)
+    return out
 
 
 def main(argv=None):

@@ -25,6 +25,7 @@
 #include "eqc_nodeprod.cuh"
 #include "eqc_dispatch.h"
 #include "eqc_graph.h"
+#include "eqc_radial.h"
 #include "eqconv.h"
 
 namespace eqc {
@@ -73,38 +74,6 @@ cudaError_t launch_sh(int lsh, const float* r, float* Y, int E, cudaStream_t st)
         case 3: return sh_k<3>(r, Y, E, st);
         default: return cudaErrorInvalidValue;
     }
-}
-
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t count, int rows, int C, int tile_c) {
-    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-    if (!enc || !base || count == 0 || rows <= 0 || rows > 256 || tile_c > 256) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)rows, (cuuint64_t)count};
-    const cuuint64_t strides[2] = {(cuuint64_t)C * 4u, (cuuint64_t)rows * (cuuint64_t)C * 4u};
-    const cuuint32_t box[3] = {(cuuint32_t)tile_c, (cuuint32_t)rows, 1u};
-    const cuuint32_t estr[3] = {1u, 1u, 1u};
-    // promote L2 fills to the box row width at most: a wider promotion would
-    // fetch the neighbouring channel tile, which is not read until much later
-    const int row_bytes = tile_c * 4;
-    const CUtensorMapL2promotion promo = row_bytes >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
-                                         : row_bytes >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
-                                                            : CU_TENSOR_MAP_L2_PROMOTION_NONE;
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
-                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, promo,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 __global__ void k_zero_f4(float4* p, int64_t n4) {
@@ -671,6 +640,30 @@ int eqconv_node_product_backward(eqconv_plan_t plan, int N, const float* u, cons
     prm.N = N;
     prm.C = plan->C;
     return cuda_status(plan->np_ks->bwd(prm, (cudaStream_t)stream), "node product backward");
+}
+
+size_t eqconv_radial_workspace_bytes(eqconv_plan_t plan, int E) {
+    if (!plan || E < 0 || plan->node_product) return 0;
+    return eqc::radial::workspace_bytes(E, plan->P * plan->C);
+}
+
+int eqconv_radial_weights(eqconv_plan_t plan, int E, const float* r, const float* W1, const float* W2,
+                          const float* W3, int n_basis, float r_cut, float* w, void* workspace,
+                          size_t workspace_bytes, eqconv_stream_t stream) {
+    if (!plan || plan->node_product || E < 0) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_device(plan);
+    if (rc != EQCONV_OK) return rc;
+    if (n_basis < 1 || n_basis > eqc::radial::kMaxBasisHost || !(r_cut > 0.f)) return EQCONV_ERR_INVALID_ARG;
+    if (!W1 || !W2 || !W3 || (E > 0 && (!r || !w))) return EQCONV_ERR_INVALID_ARG;
+    if (plan->C % 32 != 0) return EQCONV_ERR_UNSUPPORTED;
+    const int PC = plan->P * plan->C;
+    const size_t need = eqc::radial::workspace_bytes(E, PC);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return EQCONV_ERR_WORKSPACE;
+    const cudaStream_t st = (cudaStream_t)stream;
+    const eqc::radial::Workspace ws = eqc::radial::carve(workspace, E, PC);
+    cudaError_t err = eqc::radial::prepare(ws, r, nullptr, E, W1, W2, W3, n_basis, r_cut, PC, st);
+    if (err != cudaSuccess) return cuda_status(err, "radial weights (hidden layers)");
+    return cuda_status(eqc::radial::weights(ws, E, PC, w, plan->d_status, st), "radial weights (last layer)");
 }
 
 int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y, eqconv_stream_t stream) {

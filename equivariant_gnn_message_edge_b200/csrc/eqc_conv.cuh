@@ -517,9 +517,23 @@ struct BwdParams {
 // mbarrier per stage counts the bytes of the bulk copies (cp.async.bulk, no
 // multicast) that fill it; the warp waits on the stage's phase before reading
 // it, and refills it S edges later.  Every wait is bounded: after
-// kWaitLimit polls the kernel sets status bit 4 and stops processing.
+// kWaitLimitNs the kernel sets status bit 4 and stops processing.
 
-constexpr uint32_t kWaitLimit = 1u << 24;
+// Every wait on a stage gives up after this much time (globaltimer ns); a
+// row copy that has not landed by then will not land.  Each poll may suspend
+// the thread for at most kWaitSuspendNs (the try_wait time hint), so the
+// bound holds whatever the hardware's own suspend limit is.
+#ifndef EQC_WAIT_LIMIT_NS
+#define EQC_WAIT_LIMIT_NS 200000000ull   // 0.2 s
+#endif
+constexpr uint64_t kWaitLimitNs = EQC_WAIT_LIMIT_NS;
+constexpr uint32_t kWaitSuspendNs = 1000;
+// Extra bytes every stage fill expects beyond what its copies carry.  Always 0
+// in the library; a test build sets it so that no fill can complete and the
+// bounded waits below must give up.
+#ifndef EQC_TEST_FILL_DEFICIT
+#define EQC_TEST_FILL_DEFICIT 0
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -538,21 +552,44 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                  : "memory");
 }
 
-// Returns false if the phase did not complete within the poll limit.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Warp-collective bounded wait on one phase of `bar`: every lane polls and
+// the warp leaves the loop together (the phase stays complete once it has
+// completed, so all lanes see it within one poll of each other; a timeout
+// seen by any lane ends the wait for all).  Returns false, on every lane, if
+// the phase did not complete within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     const uint32_t a = smem_addr(bar);
-    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(done)
-            : "r"(a), "r"(parity)
+            : "r"(a), "r"(parity), "r"(kWaitSuspendNs)
             : "memory");
-        if (done) return true;
+        if (__all_sync(0xffffffffu, done)) return true;
+        const uint64_t now = globaltimer_ns();
+        if (it == 0) t0 = now;
+        if (__any_sync(0xffffffffu, now - t0 > kWaitLimitNs)) return false;
     }
-    return false;
+}
+
+// After a wait gave up: wait (bounded again) for the fills still in flight,
+// those of edges [from, to) of the warp's staging sequence (edge u sits in
+// stage u % S and completes phase (u / S) & 1), so that no copy lands in
+// shared memory after the warp has left.  Stages without a fill in flight are
+// not waited on.
+template <int S>
+__device__ __forceinline__ void drain_fills(uint64_t* bars, uint32_t from, uint32_t to) {
+    for (uint32_t u = from; u < to; ++u) mbar_wait(&bars[2 * (u % S)], (u / S) & 1u);
 }
 
 __device__ __forceinline__ void fence_proxy_async() {
@@ -586,7 +623,7 @@ __device__ __forceinline__ void stage_fill(float* st, uint64_t* bar, const CUten
                                            int e, int o, int c0, uint64_t pol_w, uint64_t pol_g, int lane) {
     if (lane == 0) {
         fence_proxy_async();
-        mbar_expect_tx(bar, Stage<K, NG>::BYTES);
+        mbar_expect_tx(bar, Stage<K, NG>::BYTES + EQC_TEST_FILL_DEFICIT);
         tma_rows(st, tw, c0, e, bar, pol_w);
         tma_rows(st + K::NP * K::TILE_C, tg, c0, o, bar, pol_g);
     }
@@ -734,6 +771,7 @@ __global__ void __launch_bounds__(FwdShape<K>::WARPS * 32)
 
     uint32_t g = 0;        // edges staged so far by this warp (stage = g % S, phase = (g / S) & 1)
     bool ok_all = true;
+    uint32_t fill_from = 0, fill_to = 0;   // after a failed wait: staged edges whose fills are in flight
     int k = prm.ptr[node];
     const int ke = prm.ptr[node + 1];
     while (k < ke && ok_all) {
@@ -766,6 +804,8 @@ __global__ void __launch_bounds__(FwdShape<K>::WARPS * 32)
                 if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
                     if (lane == 0) atomicOr(prm.status, 4u);
                     ok_all = false;
+                    fill_from = gi;                       // fills of edges [gi, g + min(n, t + S)) are in flight
+                    fill_to = g + (uint32_t)min(n, t + S);
                     break;
                 }
                 // Lanes past C in a ragged tile read the tensor map's zero fill, so
@@ -803,8 +843,7 @@ __global__ void __launch_bounds__(FwdShape<K>::WARPS * 32)
         g += n;
     }
     if (!ok_all) {
-        // drain: wait (bounded) for copies still in flight before the warp exits
-        for (int s = 0; s < S; ++s) mbar_wait(&bars[2 * s], 0), mbar_wait(&bars[2 * s], 1);
+        drain_fills<S>(bars, fill_from, fill_to);
         return;
     }
     // a later band adds its sum; a band without edges for this node leaves y as it is
@@ -902,6 +941,7 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
 
     uint32_t g = 0;
     bool ok_all = true;
+    uint32_t fill_from = 0, fill_to = 0;   // after a failed wait: staged edges whose fills are in flight
     int k = prm.ptr[node];
     const int ke = prm.ptr[node + 1];
     while (k < ke && ok_all) {
@@ -940,6 +980,8 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
                 if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
                     if (lane == 0) atomicOr(prm.status, 4u);
                     ok_all = false;
+                    fill_from = gi;                       // fills of edges [gi, g + min(n, t + S)) are in flight
+                    fill_to = g + (uint32_t)min(n, t + S);
                     break;
                 }
                 const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_o, t);
@@ -1009,7 +1051,7 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
         g += n;
     }
     if (!ok_all) {
-        for (int s = 0; s < S; ++s) mbar_wait(&bars[2 * s], 0), mbar_wait(&bars[2 * s], 1);
+        drain_fills<S>(bars, fill_from, fill_to);
         return;
     }
     if constexpr (DET) {

@@ -9,7 +9,9 @@
 // Integer work only; the result is bit-exact and independent of scheduling
 // (integer atomics on counts, fixed-order ranks in the scatter).  No kernel
 // waits on another block: every dependency is a kernel boundary.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 #include <mutex>
@@ -290,6 +292,32 @@ cudaError_t graph_build(int N, int E, const int* senders, const int* receivers, 
 // once per device with cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_graph_scratch[kGraphScratchBytes];
 
+// Unique ID of the calling thread's current CUDA context (cuCtxGetId through
+// the runtime's driver entry points, so the library does not link libcuda);
+// 0 when there is no current context or the driver does not offer the call.
+static unsigned long long current_context_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
 cudaError_t graph_build_noalloc(int N, int E, const int* senders, const int* receivers, int* recv_ptr,
                                 int* recv_perm, int* send_ptr, int* send_perm, unsigned* status, cudaStream_t st,
                                 bool* too_large) {
@@ -300,6 +328,7 @@ cudaError_t graph_build_noalloc(int N, int E, const int* senders, const int* rec
     }
     static std::mutex mu;
     static void* addr[64] = {};
+    static unsigned long long ctx_id[64] = {};   // context the cached address belongs to (0: none)
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -307,12 +336,21 @@ cudaError_t graph_build_noalloc(int N, int E, const int* senders, const int* rec
     void* scratch = nullptr;
     {
         std::lock_guard<std::mutex> lock(mu);
-        if (!addr[dev]) {
-            err = cudaGetSymbolAddress(&addr[dev], g_graph_scratch);
+        // The address belongs to the device's current context: after
+        // cudaDeviceReset the primary context is a new one and the array has
+        // a new address, so the cache is keyed by the context's unique ID and
+        // looked up again when it changes (or when no ID can be read).
+        const unsigned long long id = current_context_id();
+        if (!addr[dev] || id == 0 || id != ctx_id[dev]) {
+            void* a = nullptr;
+            err = cudaGetSymbolAddress(&a, g_graph_scratch);
             if (err != cudaSuccess) {
                 addr[dev] = nullptr;
+                ctx_id[dev] = 0;
                 return err;
             }
+            addr[dev] = a;
+            ctx_id[dev] = current_context_id();   // the lookup made the device's context current
         }
         scratch = addr[dev];
     }

@@ -1,0 +1,41 @@
+// Host interface of the on-chip radial weights (no device code).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+
+namespace eqc {
+namespace radial {
+
+constexpr int kMaxBasisHost = 16;   // Bessel functions (eqc_radial.cuh kMaxBasis)
+
+// Pieces of the caller's workspace (all 256-byte aligned):
+//   a_hi, a_lo  [PC][64] fp16   W3^T split into fp16 pairs, scaled by 2^s_W3
+//   inv_scale   [1]             2^-s_W3
+//   h_hi, h_lo  [E][64]  fp16   h2 of every edge (or position) split, scaled per row
+//   uscale      [E]             u(d) * 2^-(s_W3 + s_h2)
+struct Workspace {
+    __half* a_hi;
+    __half* a_lo;
+    float* inv_scale;
+    __half* h_hi;
+    __half* h_lo;
+    float* uscale;
+    size_t bytes;
+};
+
+Workspace carve(void* ws, int E, int PC);
+size_t workspace_bytes(int E, int PC);
+
+// W3 split (one CTA) and the hidden layers of every edge, in the order of
+// `perm` (position k holds edge perm[k]; perm == nullptr: edge order).
+cudaError_t prepare(const Workspace& ws, const float* r, const int* perm, int E, const float* W1, const float* W2,
+                    const float* W3, int NB, float rc, int PC, cudaStream_t st);
+
+// w [E][PC] from a prepared workspace (edge order), on the tensor cores.
+cudaError_t weights(const Workspace& ws, int E, int PC, float* w, unsigned* status, cudaStream_t st);
+
+}  // namespace radial
+}  // namespace eqc

@@ -255,6 +255,20 @@ def water_box_graph():
     return _WATER_GRAPH
 
 
+def water_box_system():
+    """The water box as a function of positions: (pos [n][3] fp64, senders,
+    receivers, shift [E][3] fp64, is_dummy) with r = pos[s] - pos[rcv] + shift
+    for every edge (the minimum-image shift; (cutoff, 0, 0) on the dummy
+    i -> i edges, whose r then does not depend on the positions)."""
+    c = WATER_BOX
+    pos = random_sequential_packing(c["n_atoms"], c["box"], c["min_dist"])
+    s, rcv, r, is_dummy = water_box_graph()
+    d = pos[s] - pos[rcv]
+    shift = -c["box"] * np.round(d / c["box"])
+    shift[is_dummy] = [c["cutoff"], 0.0, 0.0]
+    return pos, s, rcv, shift, is_dummy
+
+
 def water_box_weights(P: int, C: int) -> np.ndarray:
     """Radial weights w[E, P, C] of the water box's edges (zero on dummies)."""
     _, _, r, is_dummy = water_box_graph()

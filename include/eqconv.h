@@ -82,8 +82,11 @@ enum {
 typedef struct eqconv_plan_s* eqconv_plan_t;
 
 /* Edge layout.  The caller fills N, E, senders and receivers and provides the
- * four output arrays; eqconv_graph_build fills them (FlashCart §4: receiver
- * sorted edges; sender order for deterministic sender gradients):
+ * four output arrays; eqconv_graph_build fills them (FlashCart, arXiv
+ * 2610.06409, §4 and App. D: the forward runs over receiver-sorted edges so
+ * that each program sums a receiver's incoming edges locally; the
+ * deterministic VJP walks the edges in sender order so that each sender's
+ * input gradient is summed by one program):
  *   recv_ptr[N+1]  = [0, cumsum(in-degree)]    recv_perm[E] = stable argsort(receivers)
  *   send_ptr[N+1]  = [0, cumsum(out-degree)]   send_perm[E] = stable argsort(senders)
  * All device pointers, caller-owned; the struct itself is read on the host. */
@@ -191,7 +194,11 @@ EQCONV_API int eqconv_cg_table(int l1, int l2, int l3, double* out, int out_len)
 EQCONV_API size_t eqconv_graph_workspace_bytes(int N, int E);
 
 /* Builds recv_ptr/recv_perm/send_ptr/send_perm on `stream` (stable LSD radix
- * sort + histogram + exclusive scan; bit-exact with a stable argsort).
+ * sort + histogram + exclusive scan; bit-exact with a stable argsort): the
+ * receiver-sorted and sender-sorted edge orders of FlashCart §4 / App. D.
+ * N, E, senders and receivers are read from *g (host struct, device arrays);
+ * the workspace is caller-owned device memory of at least
+ * eqconv_graph_workspace_bytes(N, E) bytes (EQCONV_ERR_WORKSPACE otherwise).
  * Out-of-range senders/receivers set the device status word and are counted
  * nowhere (the outputs are then unspecified but in-bounds). */
 EQCONV_API int eqconv_graph_build(eqconv_plan_t plan, const eqconv_graph_t* g, void* workspace,
@@ -210,7 +217,9 @@ EQCONV_API int eqconv_graph_build(eqconv_plan_t plan, const eqconv_graph_t* g, v
  *     eqconv_last_error then states the bytes needed.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is cached per device together
+ *     with the ID of the context it belongs to: after cudaDeviceReset the
+ *     next call sees a new context and looks the address up again.
  *   - Every call shares the one array: calls that overlap on the GPU (on two
  *     streams, or from two threads) race and corrupt each other's result.
  *     The scratch keeps the last call's contents; each call clears what it
@@ -218,8 +227,14 @@ EQCONV_API int eqconv_graph_build(eqconv_plan_t plan, const eqconv_graph_t* g, v
 EQCONV_API int eqconv_graph_build_noalloc(eqconv_plan_t plan, const eqconv_graph_t* g,
                                           eqconv_stream_t stream);
 
-/* Forward (one fused kernel; receiver-sorted, atomic-free, no per-edge
- * messages in memory; deterministic): writes y [N][D_out][C]. */
+/* Forward: y [N][D_out][C] by the formula at the top of this file (e3j,
+ * arXiv 2609.35099, abstract and Table 1: the convolution of MACE-style
+ * potentials; FlashCart, arXiv 2610.06409, App. B for the paths and §4 /
+ * App. D for the scheme: receiver-sorted, one program per receiver and
+ * channel tile summing its incoming edges locally and storing each output
+ * once, no atomics and no per-edge message tensor).  One fused kernel launch
+ * (more when gather bands are set); deterministic.  x, w and y must be
+ * 16-byte aligned; y is overwritten.  `flags` is reserved (pass 0). */
 EQCONV_API int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
                    const float* r, const float* w, float* y, unsigned flags,
                    eqconv_stream_t stream);
@@ -229,10 +244,21 @@ EQCONV_API int eqconv_forward(eqconv_plan_t plan, const eqconv_graph_t* g, const
  * in-kernel; otherwise per-tile partials of dr's harmonic gradient). */
 EQCONV_API size_t eqconv_backward_workspace_bytes(eqconv_plan_t plan, int E);
 
-/* Backward given gy: writes dx [N][D_in][C], dw [E][P][C], dr [E][3].
+/* Backward (vector-Jacobian product) given gy [N][D_out][C]: writes
+ *   dx[j, l1 m1, c] = sum_{e: send(e)=j} sum_p w[e,p,c] sum_{m2,m3} C_p Y_{l2 m2}(r_e) gy[recv(e), l3 m3, c]
+ *   dw[e, p, c]     = sum_{m1,m2,m3} C_p x[send(e), l1 m1, c] Y_{l2 m2}(r_e) gy[recv(e), l3 m3, c]
+ *   dr[e]           = (dY(r_e/|r_e|)/dr_e)^T gY[e],
+ *                     gY[e, l2 m2] = sum_c sum_{p with this l2} w[e,p,c] sum_{m1,m3} C_p x gy
+ * (FlashCart, arXiv 2610.06409, §2: forces are the gradient of the energy
+ * with respect to positions, so dr carries them; §4 and App. D: the VJP's
+ * shared input gradient dx is accumulated either with atomic adds in
+ * receiver order or, in sender order, deterministically; weight gradients
+ * are stored directly).
  * flags & EQCONV_DETERMINISTIC: one pass over the sender CSR, dx summed in
- * registers, no atomics; otherwise one pass over the receiver CSR with dx
- * accumulated by atomic adds (dx is zeroed by the library first). */
+ * registers, no atomics, bitwise reproducible; otherwise one pass over the
+ * receiver CSR with dx accumulated by atomic adds (dx is zeroed by the
+ * library first).  The workspace (eqconv_backward_workspace_bytes) is needed
+ * only when C spans several channel tiles.  All outputs are overwritten. */
 EQCONV_API int eqconv_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x,
                     const float* r, const float* w, const float* gy, float* dx, float* dw,
                     float* dr, void* workspace, size_t workspace_bytes, unsigned flags,
@@ -308,13 +334,43 @@ EQCONV_API int eqconv_node_product_backward(eqconv_plan_t plan, int N, const flo
                                             float* dw, void* workspace, size_t workspace_bytes,
                                             eqconv_stream_t stream);
 
+/* ---- Radial weights from edge lengths ------------------------------------
+ * FlashCart (arXiv 2610.06409) App. B: a radial envelope makes every edge's
+ * contribution vanish smoothly at the cutoff; App. E: the weights vanish with
+ * their first two derivatives there.  e3j (arXiv 2609.35099) Table 3: 8
+ * radial (Bessel) functions, 5 Angstrom cutoff.  With d = |r_e|,
+ * x = min(d / r_cut, 1) and no biases:
+ *   b_n(d)     = sqrt(2 / r_cut) sin(n pi d / r_cut) / max(d, 1e-12)   n = 1..n_basis
+ *   u(d)       = 1 - 28 x^6 + 48 x^7 - 21 x^8
+ *   w[e, p, c] = u(d) * sum_k h2[k] W3[k][p*C + c],
+ *   h2 = silu(silu(b W1) W2),   silu(z) = z / (1 + exp(-z))
+ * W1 [n_basis][64], W2 [64][64], W3 [64][P*C] fp32 row-major (hidden width
+ * EQCONV_RADIAL_HIDDEN); 1 <= n_basis <= 16; C % 32 == 0.  The last layer
+ * runs on the tensor cores with every operand split into two scaled fp16
+ * halves (about 22 bits of each operand kept; fp32 accumulation).
+ * The workspace (eqconv_radial_workspace_bytes, 16-byte aligned) holds the
+ * split W3, the edges' split h2 and per-edge factors; caller-owned. */
+#define EQCONV_RADIAL_HIDDEN 64
+
+EQCONV_API size_t eqconv_radial_workspace_bytes(eqconv_plan_t plan, int E);
+
+/* w [E][P][C] of the formula above, written to memory (the unfused radial
+ * path; eqconv_forward_radial keeps w on the chip instead).  Three launches
+ * on `stream`: the W3 split, the hidden layers, the last layer. */
+EQCONV_API int eqconv_radial_weights(eqconv_plan_t plan, int E, const float* r, const float* W1, const float* W2,
+                                     const float* W3, int n_basis, float r_cut, float* w, void* workspace,
+                                     size_t workspace_bytes, eqconv_stream_t stream);
+
 /* The spherical harmonics the kernels use, Y [E][(L_sh+1)^2] (a test hook
  * for the in-kernel harmonics; not on the hot path). */
 EQCONV_API int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y,
                                eqconv_stream_t stream);
 
 /* Synchronises `stream`, reads and clears the plan's device status word;
- * *status receives EQCONV_OK or EQCONV_ERR_DEVICE_CHECK. */
+ * *status receives EQCONV_OK or EQCONV_ERR_DEVICE_CHECK (the return value
+ * reports whether the query itself worked, so a failed synchronisation is
+ * not mistaken for a device check).  Status bits: 1 an out-of-range node
+ * index was skipped, 4 a bounded wait for a row copy gave up. */
 EQCONV_API int eqconv_get_device_error(eqconv_plan_t plan, eqconv_stream_t stream, int* status);
 
 EQCONV_API void eqconv_plan_destroy(eqconv_plan_t plan);

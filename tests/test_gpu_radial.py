@@ -1,0 +1,89 @@
+"""Radial weights on the tensor cores (eqconv_radial_weights) against the
+oracle's radial MLP (needs a B200).
+
+w[e, p, c] = u(|r_e|) * (silu(silu(b(|r_e|) W1) W2) W3)[p*C + c] with the
+Bessel basis b and the C2 polynomial envelope u (FlashCart App. B / App. E;
+e3j Table 3: 8 Bessel functions, 5 A cutoff).  The last layer runs as fp16
+hi/lo products with fp32 accumulation in tensor memory; the result must match
+the fp64 oracle within the convolution's tolerance, at sizes that span
+several 128-row and 64-edge tiles with ragged tails, for edges at, beyond and
+on zero length, and for weights of very different scales.
+"""
+import numpy as np
+import pytest
+import torch
+
+from equivariant_gnn_message_edge_b200 import binding as B
+from equivariant_gnn_message_edge_b200 import workloads as wl
+from equivariant_gnn_message_edge_b200.conv import EqConv
+from oracle import radial as orad
+from tests.gpu_common import assert_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _edges(E, rc, seed):
+    rng = np.random.default_rng(seed)
+    d = rng.standard_normal((E, 3))
+    d /= np.linalg.norm(d, axis=1, keepdims=True)
+    length = rng.uniform(0.3, 1.1 * rc, size=E)      # some beyond the cutoff
+    r = d * length[:, None]
+    if E >= 4:
+        r[0] = 0.0                                   # zero length
+        r[1] = [rc, 0.0, 0.0]                        # exactly at the cutoff: u = 0
+        r[2] = [0.0, 0.0, 1e-3]                      # very short
+    return r.astype(np.float32)
+
+
+def _gpu_weights(conv, r, params, n_basis, rc):
+    E = r.shape[0]
+    ws_n = B.eqconv_radial_workspace_bytes(conv.plan, E)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
+    w = torch.full((max(E, 1), conv.P, conv.C), float("nan"), device="cuda")
+    W1, W2, W3 = (to_dev(p) for p in params)
+    B.eqconv_radial_weights(conv.plan, E, to_dev(r), W1, W2, W3, n_basis, rc, w, ws, ws_n)
+    torch.cuda.synchronize()
+    assert B.eqconv_get_device_error(conv.plan) == B.EQCONV_OK
+    return w[:E].cpu().numpy()
+
+
+@pytest.mark.parametrize("L,C,E", [(1, 32, 1), (1, 32, 65), (2, 128, 1000), (2, 32, 333), (3, 64, 700),
+                                   (3, 128, 129)])
+def test_radial_weights_match_oracle(L, C, E):
+    ins = wl.natural_irreps(L)
+    conv = EqConv(ins, L, ins, C)
+    rc, nb = 5.0, 8
+    r = _edges(E, rc, seed=E + C)
+    params = wl.radial_mlp_params(conv.P, C, 64, nb, seed=7 + L)
+    got = _gpu_weights(conv, r, params, nb, rc)
+    want = orad.radial_weights(np.linalg.norm(r.astype(np.float64), axis=1), rc, params, conv.P, C)
+    assert_close(f"w L={L} C={C} E={E}", got, want)
+    d = np.linalg.norm(r.astype(np.float64), axis=1)
+    assert np.all(got[d >= rc * (1 + 1e-6)] == 0.0), "weights beyond the cutoff must be exactly zero"
+
+
+@pytest.mark.parametrize("scale", [1e-4, 1e3])
+def test_radial_weights_scale_robust(scale):
+    """The power-of-two scaling keeps the fp16 halves in range for weights
+    far from unit size."""
+    conv = EqConv("0e+1o+2e", 2, "0e+1o+2e", 64)
+    rc, nb = 5.0, 8
+    r = _edges(500, rc, seed=3)
+    params = wl.radial_mlp_params(conv.P, 64, 64, nb, seed=11)
+    params = [params[0], params[1] * np.float32(scale), params[2] * np.float32(1.0 / scale)]
+    got = _gpu_weights(conv, r, params, nb, rc)
+    want = orad.radial_weights(np.linalg.norm(r.astype(np.float64), axis=1), rc, params, conv.P, 64)
+    assert_close(f"w scale {scale}", got, want)
+
+
+def test_radial_weights_water_box():
+    """The water box's own edges and MLP (dummy edges at the cutoff get 0)."""
+    cfg = wl.WATER_BOX
+    ins = wl.natural_irreps(cfg["L"])
+    conv = EqConv(ins, cfg["L"], ins, cfg["C"])
+    s, rcv, r, dummy = wl.water_box_graph()
+    params = wl.radial_mlp_params(conv.P, cfg["C"], cfg["hidden"], cfg["n_bessel"])
+    got = _gpu_weights(conv, r, params, cfg["n_bessel"], cfg["cutoff"])
+    ref = orad.radial_weights(np.linalg.norm(r.astype(np.float64), axis=1), cfg["cutoff"], params, conv.P, cfg["C"])
+    assert_close("water box w", got, ref)
+    assert np.all(got[dummy] == 0.0)
