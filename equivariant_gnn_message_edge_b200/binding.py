@@ -38,6 +38,7 @@ ABI_FUNCTIONS = (
     "eqconv_double_backward_workspace_bytes", "eqconv_double_backward",
     "eqconv_node_product_plan_create", "eqconv_node_product", "eqconv_node_product_workspace_bytes",
     "eqconv_node_product_backward", "eqconv_radial_workspace_bytes", "eqconv_radial_weights",
+    "eqconv_forward_radial_workspace_bytes", "eqconv_forward_radial",
 )
 
 
@@ -89,6 +90,8 @@ _SIGS = {
     "eqconv_node_product_backward": (_ci, [_vp, _ci] + [_vp] * 8 + [_sz, _vp]),
     "eqconv_spherical_harmonics": (_ci, [_vp, _ci, _vp, _vp, _vp]),
     "eqconv_radial_workspace_bytes": (_sz, [_vp, _ci]),
+    "eqconv_forward_radial_workspace_bytes": (_sz, [_vp, _ci, _ci]),
+    "eqconv_forward_radial": (_ci, [_vp, _pg] + [_vp] * 5 + [_ci, ctypes.c_float, _vp, _vp, _sz, _vp]),
     "eqconv_radial_weights": (_ci, [_vp, _ci] + [_vp] * 4 + [_ci, ctypes.c_float, _vp, _vp, _sz, _vp]),
     "eqconv_get_device_error": (_ci, [_vp, _vp, _pi]),
     "eqconv_plan_destroy": (None, [_vp]),
@@ -321,6 +324,18 @@ def eqconv_radial_weights(plan: int, E: int, r, W1, W2, W3, n_basis: int, r_cut:
     _check(lib().eqconv_radial_weights(plan, int(E), _ptr(r, f), _ptr(W1, f), _ptr(W2, f), _ptr(W3, f),
                                        int(n_basis), float(r_cut), _ptr(w, f), _ptr(workspace),
                                        int(workspace_bytes), _stream(stream)), "eqconv_radial_weights")
+
+
+def eqconv_forward_radial_workspace_bytes(plan: int, N: int, E: int) -> int:
+    return int(lib().eqconv_forward_radial_workspace_bytes(plan, int(N), int(E)))
+
+
+def eqconv_forward_radial(plan: int, graph: eqconv_graph_t, x, r, W1, W2, W3, n_basis: int, r_cut: float, y,
+                          workspace, workspace_bytes: int, stream=None) -> None:
+    f = _f32()
+    _check(lib().eqconv_forward_radial(plan, ctypes.byref(graph), _ptr(x, f), _ptr(r, f), _ptr(W1, f), _ptr(W2, f),
+                                       _ptr(W3, f), int(n_basis), float(r_cut), _ptr(y, f), _ptr(workspace),
+                                       int(workspace_bytes), _stream(stream)), "eqconv_forward_radial")
 
 
 def eqconv_spherical_harmonics(plan: int, E: int, r, Y, stream=None) -> None:

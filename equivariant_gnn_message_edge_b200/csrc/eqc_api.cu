@@ -26,6 +26,7 @@
 #include "eqc_dispatch.h"
 #include "eqc_graph.h"
 #include "eqc_radial.h"
+#include "eqc_radial_conv.h"
 #include "eqconv.h"
 
 namespace eqc {
@@ -664,6 +665,55 @@ int eqconv_radial_weights(eqconv_plan_t plan, int E, const float* r, const float
     cudaError_t err = eqc::radial::prepare(ws, r, nullptr, E, W1, W2, W3, n_basis, r_cut, PC, st);
     if (err != cudaSuccess) return cuda_status(err, "radial weights (hidden layers)");
     return cuda_status(eqc::radial::weights(ws, E, PC, w, plan->d_status, st), "radial weights (last layer)");
+}
+
+static const eqc::radial::RadConvSet* radial_set(eqconv_plan_t plan) {
+    if (!plan || plan->node_product || (plan->mode & eqc::kModeAllParity)) return nullptr;
+    return eqc::radial::find_radial_conv(plan->lin, plan->lsh, plan->lout);
+}
+
+size_t eqconv_forward_radial_workspace_bytes(eqconv_plan_t plan, int N, int E) {
+    const eqc::radial::RadConvSet* rs = radial_set(plan);
+    if (!rs || N < 0 || E < 0) return 0;
+    return rs->fwd_workspace(N, E, plan->C, (plan->mode & eqc::kModePerPath) != 0);
+}
+
+int eqconv_forward_radial(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r,
+                          const float* W1, const float* W2, const float* W3, int n_basis, float r_cut, float* y,
+                          void* workspace, size_t workspace_bytes, eqconv_stream_t stream) {
+    if (!plan || plan->node_product) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_graph(g);
+    if (rc != EQCONV_OK) return rc;
+    if ((rc = check_device(plan)) != EQCONV_OK) return rc;
+    const eqc::radial::RadConvSet* rs = radial_set(plan);
+    if (!rs || plan->C % 32 != 0) return EQCONV_ERR_UNSUPPORTED;
+    if (n_basis < 1 || n_basis > eqc::radial::kMaxBasisHost || !(r_cut > 0.f)) return EQCONV_ERR_INVALID_ARG;
+    if (g->N == 0) return EQCONV_OK;
+    if (!x || !y || !W1 || !W2 || !W3 || (g->E > 0 && !r)) return EQCONV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return EQCONV_ERR_INVALID_ARG;
+    const bool per_path = (plan->mode & eqc::kModePerPath) != 0;
+    const size_t need = rs->fwd_workspace(g->N, g->E, plan->C, per_path);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return EQCONV_ERR_WORKSPACE;
+    eqc::radial::RadFwdArgs a{};
+    a.x = x;
+    a.r = r;
+    a.recv_ptr = g->recv_ptr;
+    a.recv_perm = g->recv_perm;
+    a.senders = g->senders;
+    a.W1 = W1;
+    a.W2 = W2;
+    a.W3 = W3;
+    a.NB = n_basis;
+    a.rc = r_cut;
+    a.y = y;
+    a.per_path = per_path;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    a.N = g->N;
+    a.E = g->E;
+    a.C = plan->C;
+    a.status = plan->d_status;
+    return cuda_status(rs->fwd(a, (cudaStream_t)stream), "forward (radial)");
 }
 
 int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y, eqconv_stream_t stream) {

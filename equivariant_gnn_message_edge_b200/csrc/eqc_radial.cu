@@ -17,6 +17,213 @@ void count_launch();
 
 namespace radial {
 
+// --------------------------------------------------------------- W3 prep
+
+// A_hi / A_lo [PC][64] fp16 = split(W3^T * 2^s), s for the largest |W3|;
+// inv_scale[0] = 2^-s.  One CTA of 1024 threads (W3 has 64 * P * C values).
+__global__ void __launch_bounds__(1024)
+    radial_prep_w3_kernel(const float* __restrict__ W3, int PC, __half* __restrict__ A_hi, __half* __restrict__ A_lo,
+                          float* __restrict__ inv_scale) {
+    __shared__ float red[32];
+    const int tid = threadIdx.x;
+    const int n = kH * PC;
+    float m = 0.f;
+    for (int i = tid; i < n; i += blockDim.x) m = fmaxf(m, fabsf(W3[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+    if (tid < 32) {
+        m = tid < (int)(blockDim.x >> 5) ? red[tid] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (tid == 0) red[0] = m;
+    }
+    __syncthreads();
+    const int s = pow2_exponent_for(red[0]);
+    const float sc = ldexpf(1.f, s);
+    for (int i = tid; i < n; i += blockDim.x) {
+        const int pc = i / kH, k = i - pc * kH;
+        __half hi, lo;
+        split_f16(W3[(size_t)k * PC + pc] * sc, hi, lo);
+        A_hi[i] = hi;
+        A_lo[i] = lo;
+    }
+    if (tid == 0) inv_scale[0] = ldexpf(1.f, -s);
+}
+
+// ------------------------------------------------------- hidden layers
+
+// For output position k (edge e = perm[k], or k without perm): the two
+// hidden layers on the CUDA cores, then h2 split into fp16 pairs with its own
+// power of two (H_hi / H_lo [E][64]), and uscale[k] = u(d) * 2^-(s_W3 +
+// s_h2).  One thread per edge; W1 and W2 are read from shared memory by all
+// threads at once (broadcast).
+__global__ void __launch_bounds__(128)
+    radial_hidden_kernel(const float* __restrict__ r, const int* __restrict__ perm, int E,
+                         const float* __restrict__ W1, const float* __restrict__ W2, int NB, float rc,
+                         const float* __restrict__ w3_inv_scale, __half* __restrict__ H_hi,
+                         __half* __restrict__ H_lo, float* __restrict__ uscale) {
+    __shared__ __align__(16) float sW1[kMaxBasis * kH];
+    __shared__ __align__(16) float sW2[kH * kH];
+    for (int i = threadIdx.x; i < NB * kH; i += blockDim.x) sW1[i] = W1[i];
+    for (int i = threadIdx.x; i < kH * kH; i += blockDim.x) sW2[i] = W2[i];
+    __syncthreads();
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= E) return;
+    const int e = perm ? perm[k] : k;
+    const float rx = r[(size_t)e * 3], ry = r[(size_t)e * 3 + 1], rz = r[(size_t)e * 3 + 2];
+    const float d = sqrtf(fmaf(rx, rx, fmaf(ry, ry, rz * rz)));
+    const float inv_d = 1.f / fmaxf(d, 1e-12f);
+    const float pref = sqrtf(2.f / rc);
+    const float kd = 3.14159265358979323846f * d / rc;
+    float h1[kH];
+#pragma unroll
+    for (int j = 0; j < kH; ++j) h1[j] = 0.f;
+    for (int nb = 0; nb < NB; ++nb) {
+        const float b = pref * sinf((float)(nb + 1) * kd) * inv_d;
+#pragma unroll
+        for (int j = 0; j < kH; ++j) h1[j] = fmaf(b, sW1[nb * kH + j], h1[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kH; ++j) h1[j] = silu(h1[j]);
+    float h2[kH];
+#pragma unroll
+    for (int j = 0; j < kH; ++j) h2[j] = 0.f;
+#pragma unroll 4
+    for (int q = 0; q < kH; ++q) {
+        const float a = h1[q];
+#pragma unroll
+        for (int j = 0; j < kH; j += 4) {
+            const float4 wv = *reinterpret_cast<const float4*>(&sW2[q * kH + j]);
+            h2[j] = fmaf(a, wv.x, h2[j]);
+            h2[j + 1] = fmaf(a, wv.y, h2[j + 1]);
+            h2[j + 2] = fmaf(a, wv.z, h2[j + 2]);
+            h2[j + 3] = fmaf(a, wv.w, h2[j + 3]);
+        }
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < kH; ++j) {
+        h2[j] = silu(h2[j]);
+        m = fmaxf(m, fabsf(h2[j]));
+    }
+    const int s = pow2_exponent_for(m);
+    const float sc = ldexpf(1.f, s);
+    uint4* dh = reinterpret_cast<uint4*>(H_hi + (size_t)k * kH);
+    uint4* dl = reinterpret_cast<uint4*>(H_lo + (size_t)k * kH);
+#pragma unroll
+    for (int q = 0; q < kH / 8; ++q) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            __half h0, l0, h1v, l1v;
+            split_f16(h2[8 * q + 2 * t] * sc, h0, l0);
+            split_f16(h2[8 * q + 2 * t + 1] * sc, h1v, l1v);
+            hw[t] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1v) << 16);
+            lw[t] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1v) << 16);
+        }
+        dh[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        dl[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    uscale[k] = envelope(d, rc) * ldexpf(1.f, -s) * w3_inv_scale[0];
+}
+
+// ------------------------------------------- last layer to w (standalone)
+
+// w[e, pc] = uscale[e] * sum_k A[pc, k] H[e, k] for one tile of 128 rows pc
+// of W3^T and 64 edges (edge = position; H and uscale in edge order): TMA
+// brings the four fp16 tiles, one thread issues the 12 MMAs (3 products x 4
+// K steps) into 64 columns of tensor memory, and each warp reads its 32 rows
+// back (row = lane) and stores them, 32 consecutive pc per edge (128 B).
+// This writes w to memory: the convolution's fused radial path keeps it on
+// the chip instead; this kernel is the unfused path and a check of the
+// tensor-core stage on its own.
+struct WSmem {
+    static constexpr int A_BYTES = kRowTile * kTileRowBytes;   // 16 KB
+    static constexpr int B_BYTES = kEdgeTile * kTileRowBytes;  // 8 KB
+    static constexpr int BYTES = 2 * A_BYTES + 2 * B_BYTES + 1024 /* barriers */ + 1024 /* alignment */;
+};
+
+__global__ void __launch_bounds__(128)
+    radial_w_kernel(const __grid_constant__ CUtensorMap map_a_hi, const __grid_constant__ CUtensorMap map_a_lo,
+                    const __grid_constant__ CUtensorMap map_h_hi, const __grid_constant__ CUtensorMap map_h_lo,
+                    const float* __restrict__ uscale, int E, int PC, float* __restrict__ w, unsigned* status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* a_hi = base;
+    uint8_t* a_lo = a_hi + WSmem::A_BYTES;
+    uint8_t* b_hi = a_lo + WSmem::A_BYTES;
+    uint8_t* b_lo = b_hi + WSmem::B_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(b_lo + WSmem::B_BYTES);   // [0] copies, [1] MMAs
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+    __shared__ int ok_shared;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int row0 = blockIdx.x * kRowTile, e0 = blockIdx.y * kEdgeTile;
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_fence_init();
+        ok_shared = 1;
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 64);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        mbar_expect_tx(&bars[0], 2 * WSmem::A_BYTES + 2 * WSmem::B_BYTES);
+        tma_2d(a_hi, &map_a_hi, 0, row0, &bars[0]);
+        tma_2d(a_lo, &map_a_lo, 0, row0, &bars[0]);
+        tma_2d(b_hi, &map_h_hi, 0, e0, &bars[0]);
+        tma_2d(b_lo, &map_h_lo, 0, e0, &bars[0]);
+        if (mbar_wait_one(&bars[0], 0)) {
+            tc_fence_after();
+            constexpr uint32_t id = idesc_f16(kRowTile, kEdgeTile);
+            const uint64_t dah = sw128_desc(smem_addr(a_hi)), dal = sw128_desc(smem_addr(a_lo));
+            const uint64_t dbh = sw128_desc(smem_addr(b_hi)), dbl = sw128_desc(smem_addr(b_lo));
+#pragma unroll
+            for (int kk = 0; kk < kH / 16; ++kk) {
+                const uint64_t adv = (uint64_t)(kk * 32) >> 4;   // 32 B per K step, in 16 B units
+                umma_f16(tmem, dah + adv, dbh + adv, id, kk > 0);
+                umma_f16(tmem, dah + adv, dbl + adv, id, 1);
+                umma_f16(tmem, dal + adv, dbh + adv, id, 1);
+            }
+            umma_commit(&bars[1]);
+        } else {
+            atomicOr(status, 4u);
+            ok_shared = 0;
+            // nothing was issued: complete the MMA barrier's phase so the
+            // other threads do not wait out their limit
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&bars[1])) : "memory");
+        }
+    }
+    __syncwarp();
+    const bool done = mbar_wait(&bars[1], 0);
+    tc_fence_after();
+    if (!done && lane == 0) atomicOr(status, 4u);
+    if (done && ok_shared) {
+        const int pc = row0 + warp * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll
+        for (int c0 = 0; c0 < kEdgeTile; c0 += 16) {
+            float v[16];
+            tmem_ld16(trow + c0, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int e = e0 + c0 + j;
+                if (e < E && pc < PC) w[(size_t)e * PC + pc] = v[j] * uscale[e];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+}
+
 static PFN_cuTensorMapEncodeTiled_v12000 encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;

@@ -1,0 +1,410 @@
+// The convolution with its radial weights produced on the chip (sm_100a):
+// w[e, p, c] never exists in global memory.
+//
+//   y[i, l3 m3, c] = sum_{e -> i} sum_p w[e, p, c] sum_{m1, m2} C_p[m1, m2, m3] x[s(e), l1 m1, c] Y_{l2 m2}(r_e)
+//   w[e, p, c]     = u(|r_e|) * (h2(|r_e|) . W3)[p*C + c]                     (eqc_radial.cuh)
+//
+// (e3j, arXiv 2609.35099, abstract and Table 3: the MACE convolution with 8
+// Bessel radial functions; FlashCart, arXiv 2610.06409, §4 / App. D for the
+// receiver-sorted scheme and App. B / App. E for the radial envelope.)
+//
+// One CTA takes a range of receivers (their in-edges are consecutive
+// positions of the receiver CSR), one slice of 32 channels and a group of up
+// to 12 paths.  Its 448 threads are 14 warps with fixed roles:
+//   * warp 12 (one thread): stages the group's W3^T rows (3 tiles of 4
+//     paths x 32 channels, fp16 hi/lo, resident for the whole CTA) and the
+//     h2 tiles of 64 positions (TMA, 2 stages), and issues the MMAs
+//       D[(path, channel), edge] = W3^T . h2^T      (M = 128, N = 64, K = 64)
+//     into one of two tensor-memory buffers (3 x 64 columns each);
+//   * warp 13 (one thread): copies each position's sender row x[s, :, slice]
+//     into a ring of shared-memory slots (TMA, one box of D_in x 32 floats);
+//   * warps 0..11 (the path warps): warp w owns path p = 12 g + w.  Its lanes
+//     are the slice's 32 channels, and tensor-memory lanes 32 (w % 4) .. +31
+//     of tile w / 4 hold exactly that path's 32 channels, so each lane reads
+//     its own w[e, p, c] with tcgen05.ld.  Per edge it forms the path's
+//     coupling A_p = C_p . Y(r_e) (lane t for edge t of a batch, into shared
+//     memory), reads its input block of the x slot and accumulates
+//       acc[m3] += w * sum_m1 A_p[m3][m1] x[m1]
+//     for the current receiver, writing the path's output block of a
+//     receiver when its edges end.
+// Outputs are per-path blocks (every path its own 2 l3 + 1 rows); a plan
+// that sums paths by output irrep adds the blocks afterwards in path order
+// (radial_sum_paths_kernel), so the result is deterministic.
+#pragma once
+
+#include "eqc_radial.cuh"
+
+namespace eqc {
+namespace radial {
+
+constexpr int kSlice = 32;         // channels per CTA: one per lane of a path warp
+constexpr int kGroupPaths = 12;    // paths per CTA: 3 MMA tiles of 4 paths x 32 channels
+constexpr int kGroupTiles = 3;
+constexpr int kPathWarps = 12;
+constexpr int kMmaWarp = 12, kXWarp = 13;
+constexpr int kConvThreads = 14 * 32;
+constexpr int kXSlots = 16;        // sender-row ring depth (positions in flight)
+constexpr int kBatch = 16;         // edges per harmonics / coupling batch of a path warp
+constexpr int kTmemCols = 512;     // 2 buffers x 3 tiles x 64 columns, rounded to a power of two
+
+struct RadFwdParams {
+    const float* x;      // [N][D_in][C]
+    const float* r;      // [E][3]
+    const int* ptr;      // recv_ptr [N+1]
+    const int* perm;     // recv_perm [E]
+    const int* senders;  // [E]
+    const float* uscale; // [E] by receiver position
+    float* y_pp;         // [N][D_pp][C] per-path output blocks
+    int N, C, E;
+    int nodes_per_cta;
+    unsigned* status;
+};
+
+template <class K>
+constexpr int max_coupling_floats() {
+    int m = 4;
+    for (int p = 0; p < K::NP; ++p) {
+        const int sz = ((2 * K::PL.l1[p] + 1) * (2 * K::PL.l3[p] + 1) + 3) & ~3;
+        if (sz > m) m = sz;
+    }
+    return m;
+}
+
+// Shared-memory layout of the fused forward (bytes; tiles 1024-aligned).
+template <class K>
+struct RadFwdSmem {
+    static constexpr int A_TILE = kRowTile * kTileRowBytes;                 // 16 KB: 128 rows of W3^T
+    static constexpr int H_TILE = kEdgeTile * kTileRowBytes;                // 8 KB: 64 rows of h2
+    static constexpr int W3_OFF = 0;                                        // [tile][hi, lo]
+    static constexpr int H_OFF = W3_OFF + kGroupTiles * 2 * A_TILE;         // [stage][hi, lo]
+    static constexpr int X_SLOT = K::D_IN * kSlice * 4;
+    static constexpr int X_OFF = H_OFF + 2 * 2 * H_TILE;
+    static constexpr int NA = max_coupling_floats<K>();
+    static constexpr int CPL_OFF = X_OFF + kXSlots * X_SLOT;
+    static constexpr int CPL_WARP = kBatch * NA * 4;
+    static constexpr int US_OFF = CPL_OFF + kPathWarps * CPL_WARP;          // per path warp: batch uscale
+    static constexpr int BAR_OFF = US_OFF + kPathWarps * kBatch * 4;
+    // barriers: w3, h_full[2], h_empty[2], t_full[2], t_empty[2], x_full[R], x_empty[R]
+    static constexpr int NBAR = 9 + 2 * kXSlots;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int END = MISC_OFF + 16;
+    static constexpr int BYTES = END + 1024;                               // + alignment slack
+};
+
+// Per-edge coupling of one path: Arow[m3 * d1 + m1] = sum_m2 C_p[m1,m2,m3] Y[l2^2 + m2].
+template <int L1, int L2, int L3>
+__device__ __forceinline__ void path_coupling(const float* Y, float* Arow) {
+    constexpr int d1 = 2 * L1 + 1, d2 = 2 * L2 + 1, d3 = 2 * L3 + 1, o2 = L2 * L2;
+    constexpr int n4 = (d1 * d3 + 3) / 4;
+    float a[n4 * 4];
+#pragma unroll
+    for (int q = d1 * d3; q < n4 * 4; ++q) a[q] = 0.f;
+    static_for<d3>([&](auto m3c) {
+        static_for<d1>([&](auto m1c) {
+            constexpr int m1 = EQC_CV(m1c), m3 = EQC_CV(m3c);
+            float s = 0.f;
+            static_for<d2>([&](auto m2c) {
+                constexpr int m2 = EQC_CV(m2c);
+                constexpr double c = RealCG<L1, L2, L3>::t.v[m1][m2][m3];
+                if constexpr (c != 0.0) s = fmaf((float)c, Y[o2 + m2], s);
+            });
+            a[m3 * d1 + m1] = s;
+        });
+    });
+#pragma unroll
+    for (int q = 0; q < n4; ++q)
+        reinterpret_cast<float4*>(Arow)[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+}
+
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+    uint32_t v;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(v) : : "memory");
+    return __uint_as_float(v);
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// The path warp's whole run for path P_ (compile-time), over the CTA's
+// positions [k0, k1) and receivers [n0, n1).
+template <class K, int P_>
+__device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* base, uint32_t tmem, int warp,
+                                              int lane, int n0, int n1, int k0, int k1, int c0,
+                                              volatile int* abort_flag) {
+    using S = RadFwdSmem<K>;
+    constexpr int l1 = K::PL.l1[P_], l2 = K::PL.l2[P_], l3 = K::PL.l3[P_];
+    constexpr int d1 = 2 * l1 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o3 = K::PL.o3[P_];
+    constexpr int NA = S::NA;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::BAR_OFF);
+    uint64_t* t_full = bars + 5;
+    uint64_t* t_empty = bars + 7;
+    uint64_t* x_full = bars + 9;
+    uint64_t* x_empty = bars + 9 + kXSlots;
+    float* cpl = reinterpret_cast<float*>(base + S::CPL_OFF + warp * S::CPL_WARP);
+    float* us_s = reinterpret_cast<float*>(base + S::US_OFF) + warp * kBatch;
+    const float* xring = reinterpret_cast<const float*>(base + S::X_OFF);
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tile_col = (uint32_t)(64 * (warp >> 2));
+    const int C = prm.C;
+
+    float acc[d3];
+#pragma unroll
+    for (int m = 0; m < d3; ++m) acc[m] = 0.f;
+    int cur = n0;
+    int cur_end = prm.ptr[n0 + 1];
+    auto flush = [&]() {
+        float* yo = prm.y_pp + ((size_t)cur * K::D_OUT + o3) * C + c0 + lane;
+#pragma unroll
+        for (int m = 0; m < d3; ++m) {
+            __stcs(yo + (size_t)m * C, acc[m]);
+            acc[m] = 0.f;
+        }
+    };
+
+    const int ntiles = (k1 - k0 + kEdgeTile - 1) / kEdgeTile;
+    for (int j = 0; j < ntiles; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&t_full[s], (uint32_t)(j >> 1) & 1u) || __any_sync(0xffffffffu, *abort_flag)) {
+            if (lane == 0) atomicOr(prm.status, 4u);
+            *abort_flag = 1;
+            return;
+        }
+        tc_fence_after();
+        const uint32_t tcol = tmem + lane_base + (uint32_t)(s * kGroupTiles * kEdgeTile) + tile_col;
+        const int kt = k0 + j * kEdgeTile;
+        const int kt_end = min(k1, kt + kEdgeTile);
+        for (int kb = kt; kb < kt_end; kb += kBatch) {
+            const int nb = min(kBatch, kt_end - kb);
+            if (lane < nb) {
+                const int k = kb + lane;
+                const int e = prm.perm[k];
+                float ux, uy, uz, il;
+                const bool ok = unit_dir(prm.r[(size_t)e * 3], prm.r[(size_t)e * 3 + 1], prm.r[(size_t)e * 3 + 2],
+                                         ux, uy, uz, il);
+                if constexpr (l2 > 0) {
+                    float Y[K::D_SH];
+                    sh_eval<K::LSH>(ok, ux, uy, uz, Y);
+                    path_coupling<l1, l2, l3>(Y, cpl + lane * NA);
+                }
+                us_s[lane] = prm.uscale[k];
+            }
+            __syncwarp();
+            for (int t = 0; t < nb; ++t) {
+                const int k = kb + t;
+                while (k >= cur_end) {   // the current receiver's edges are done (empty ones too)
+                    flush();
+                    ++cur;
+                    cur_end = prm.ptr[cur + 1];
+                }
+                const float w = tmem_ld1(tcol + (uint32_t)(k - kt)) * us_s[t];
+                const int q = k - k0;
+                const int slot = q % kXSlots;
+                if (!mbar_wait(&x_full[slot], (uint32_t)(q / kXSlots) & 1u) || __any_sync(0xffffffffu, *abort_flag)) {
+                    if (lane == 0) atomicOr(prm.status, 4u);
+                    *abort_flag = 1;
+                    return;
+                }
+                const float* xs = xring + slot * (S::X_SLOT / 4) + o1 * kSlice + lane;
+                float xv[d1];
+#pragma unroll
+                for (int m = 0; m < d1; ++m) xv[m] = xs[m * kSlice];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&x_empty[slot]);
+                if constexpr (l2 == 0) {
+#pragma unroll
+                    for (int m = 0; m < d1; ++m) acc[m] = fmaf(w, xv[m], acc[m]);
+                } else {
+                    const float* A = cpl + t * NA;
+#pragma unroll
+                    for (int m3 = 0; m3 < d3; ++m3) {
+                        float u = 0.f;
+#pragma unroll
+                        for (int m1 = 0; m1 < d1; ++m1) u = fmaf(A[m3 * d1 + m1], xv[m1], u);
+                        acc[m3] = fmaf(w, u, acc[m3]);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&t_empty[s]);
+    }
+    while (cur < n1) {   // the last receiver and any empty ones after it
+        flush();
+        ++cur;
+    }
+}
+
+template <class K>
+__global__ void __launch_bounds__(kConvThreads, 1)
+    radial_conv_fwd_kernel(const RadFwdParams prm, const __grid_constant__ CUtensorMap map_a_hi,
+                           const __grid_constant__ CUtensorMap map_a_lo, const __grid_constant__ CUtensorMap map_h_hi,
+                           const __grid_constant__ CUtensorMap map_h_lo, const __grid_constant__ CUtensorMap map_x) {
+    using S = RadFwdSmem<K>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::BAR_OFF);
+    uint64_t* w3_full = bars;
+    uint64_t* h_full = bars + 1;
+    uint64_t* h_empty = bars + 3;
+    uint64_t* t_full = bars + 5;
+    uint64_t* t_empty = bars + 7;
+    uint64_t* x_full = bars + 9;
+    uint64_t* x_empty = bars + 9 + kXSlots;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(base + S::MISC_OFF + 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const int n0 = blockIdx.x * prm.nodes_per_cta;
+    const int n1 = min(prm.N, n0 + prm.nodes_per_cta);
+    const int c0 = blockIdx.y * kSlice;
+    const int g0 = blockIdx.z * kGroupPaths;                       // first path of the group
+    const int gp = min(kGroupPaths, K::NP - g0);                   // paths in the group
+    const int gtiles = (gp + 3) / 4;
+    const int k0 = prm.ptr[n0], k1 = prm.ptr[n1];
+    const int ntiles = (k1 - k0 + kEdgeTile - 1) / kEdgeTile;
+
+    if (tid == 0) {
+        mbar_init(w3_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&h_full[s], 1);
+            mbar_init(&h_empty[s], 1);
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], gp);
+        }
+        for (int q = 0; q < kXSlots; ++q) {
+            mbar_init(&x_full[q], 1);
+            mbar_init(&x_empty[q], gp);
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < kPathWarps) {
+        const int p = g0 + warp;
+        if (warp < gp) {
+            static_for<K::NP>([&](auto pc) {
+                if (EQC_CV(pc) == p)
+                    path_warp_fwd<K, EQC_CV(pc)>(prm, base, tmem, warp, lane, n0, n1, k0, k1, c0, abort_flag);
+            });
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0 && ntiles > 0) {
+            // the group's W3^T rows: tile t, quarter q = path g0 + 4 t + q, channels [c0, c0 + 32)
+            mbar_expect_tx(w3_full, gtiles * 2 * S::A_TILE);
+            for (int t = 0; t < gtiles; ++t)
+                for (int q = 0; q < 4; ++q) {
+                    const int row = (g0 + 4 * t + q) * prm.C + c0;   // past P * C: zero fill
+                    uint8_t* dst = base + S::W3_OFF + t * 2 * S::A_TILE + q * 32 * kTileRowBytes;
+                    tma_2d(dst, &map_a_hi, 0, row, w3_full);
+                    tma_2d(dst + S::A_TILE, &map_a_lo, 0, row, w3_full);
+                }
+            auto load_h = [&](int j) {
+                const int s = j & 1;
+                uint8_t* dst = base + S::H_OFF + s * 2 * S::H_TILE;
+                mbar_expect_tx(&h_full[s], 2 * S::H_TILE);
+                tma_2d(dst, &map_h_hi, 0, k0 + j * kEdgeTile, &h_full[s]);
+                tma_2d(dst + S::H_TILE, &map_h_lo, 0, k0 + j * kEdgeTile, &h_full[s]);
+            };
+            load_h(0);
+            if (ntiles > 1) load_h(1);
+            bool ok = mbar_wait_one(w3_full, 0);
+            constexpr uint32_t id = idesc_f16(kRowTile, kEdgeTile);
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int s = j & 1;
+                ok = mbar_wait_one(&h_full[s], (uint32_t)(j >> 1) & 1u) &&
+                     (j < 2 || mbar_wait_one(&t_empty[s], (uint32_t)((j >> 1) - 1) & 1u));
+                if (!ok || *abort_flag) break;
+                tc_fence_after();
+                const uint8_t* hs = base + S::H_OFF + s * 2 * S::H_TILE;
+                const uint64_t dbh = sw128_desc(smem_addr(hs)), dbl = sw128_desc(smem_addr(hs + S::H_TILE));
+                for (int t = 0; t < gtiles; ++t) {
+                    const uint8_t* at = base + S::W3_OFF + t * 2 * S::A_TILE;
+                    const uint64_t dah = sw128_desc(smem_addr(at)), dal = sw128_desc(smem_addr(at + S::A_TILE));
+                    const uint32_t d = tmem + (uint32_t)(s * kGroupTiles * kEdgeTile + t * kEdgeTile);
+#pragma unroll
+                    for (int kk = 0; kk < kH / 16; ++kk) {
+                        const uint64_t adv = (uint64_t)(kk * 32) >> 4;
+                        umma_f16(d, dah + adv, dbh + adv, id, kk > 0);
+                        umma_f16(d, dah + adv, dbl + adv, id, 1);
+                        umma_f16(d, dal + adv, dbh + adv, id, 1);
+                    }
+                }
+                umma_commit(&t_full[s]);
+                umma_commit(&h_empty[s]);
+                if (j + 2 < ntiles) {
+                    ok = mbar_wait_one(&h_empty[s], (uint32_t)(j >> 1) & 1u);
+                    if (ok) load_h(j + 2);
+                }
+            }
+            if (!ok) {
+                atomicOr(prm.status, 4u);
+                *abort_flag = 1;
+            }
+        }
+    } else if (warp == kXWarp) {
+        if (lane == 0) {
+            for (int k = k0; k < k1; ++k) {
+                const int q = k - k0, slot = q % kXSlots;
+                if (q >= kXSlots && !mbar_wait_one(&x_empty[slot], (uint32_t)(q / kXSlots - 1) & 1u)) {
+                    atomicOr(prm.status, 4u);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                int sidx = prm.senders[prm.perm[k]];
+                if ((unsigned)sidx >= (unsigned)prm.N) {   // out of range: flagged, read as node 0
+                    atomicOr(prm.status, 1u);
+                    sidx = 0;
+                }
+                mbar_expect_tx(&x_full[slot], S::X_SLOT);
+                tma_rows(base + S::X_OFF + slot * S::X_SLOT, &map_x, c0, sidx, &x_full[slot],
+                         policy_evict_last());
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// y[i, l3^2 + m, c] = sum over paths p with that l3, in path order, of
+// y_pp[i, o3pp(p) + m, c]  (KS: the summed plan's Cfg; KP: its per-path Cfg).
+template <class KS, class KP>
+__global__ void radial_sum_paths_kernel(const float* __restrict__ y_pp, float* __restrict__ y, int N, int C) {
+    const int c4 = C / 4;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t total = (int64_t)N * KS::D_OUT * c4;
+    if (idx >= total) return;
+    const int cq = (int)(idx % c4);
+    const int row = (int)((idx / c4) % KS::D_OUT);
+    const int i = (int)(idx / ((int64_t)c4 * KS::D_OUT));
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    static_for<KP::NP>([&](auto pc) {
+        constexpr int p = EQC_CV(pc);
+        constexpr int l3 = KP::PL.l3[p];
+        if (row >= l3 * l3 && row < (l3 + 1) * (l3 + 1)) {
+            const float4 v = __ldcs(reinterpret_cast<const float4*>(
+                y_pp + ((size_t)i * KP::D_OUT + KP::PL.o3[p] + (row - l3 * l3)) * C) + cq);
+            s.x += v.x;
+            s.y += v.y;
+            s.z += v.z;
+            s.w += v.w;
+        }
+    });
+    __stcs(reinterpret_cast<float4*>(y + ((size_t)i * KS::D_OUT + row) * C) + cq, s);
+}
+
+}  // namespace radial
+}  // namespace eqc

@@ -361,6 +361,29 @@ EQCONV_API int eqconv_radial_weights(eqconv_plan_t plan, int E, const float* r, 
                                      const float* W3, int n_basis, float r_cut, float* w, void* workspace,
                                      size_t workspace_bytes, eqconv_stream_t stream);
 
+/* Device workspace bytes eqconv_forward_radial needs for (N, E); 0 when the
+ * plan has no fused radial path. */
+EQCONV_API size_t eqconv_forward_radial_workspace_bytes(eqconv_plan_t plan, int N, int E);
+
+/* The convolution's forward with w[e, p, c] produced on the chip from the
+ * edge lengths by the radial MLP above (W1, W2, W3, n_basis, r_cut as in
+ * eqconv_radial_weights): y = forward(x, r, w(|r|)) without w ever in
+ * memory (e3j Table 3 / FlashCart App. B, App. E for the weights; FlashCart
+ * §4 / App. D for the receiver-sorted scheme).  Plans: natural-parity
+ * prefixes with (L_in, L_sh, L_out) = (1,1,1), (1,2,2), (2,2,2) or (3,3,3),
+ * summed or EQCONV_OUT_PER_PATH layout, C % 32 == 0; others return
+ * EQCONV_ERR_UNSUPPORTED.  Launches on `stream`: the W3 split, the hidden
+ * layers (by receiver position), the fused kernel (one CTA per receiver
+ * range, 32-channel slice and group of up to 12 paths: tensor-core last
+ * layer into tensor memory, read there by one warp per path) and, for a
+ * summed plan, the sum of the per-path blocks in path order.  Deterministic.
+ * Out-of-range senders set the status word; the result is then unspecified
+ * (reads stay in bounds).  The workspace
+ * (eqconv_forward_radial_workspace_bytes) is caller-owned device memory. */
+EQCONV_API int eqconv_forward_radial(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r,
+                                     const float* W1, const float* W2, const float* W3, int n_basis, float r_cut,
+                                     float* y, void* workspace, size_t workspace_bytes, eqconv_stream_t stream);
+
 /* The spherical harmonics the kernels use, Y [E][(L_sh+1)^2] (a test hook
  * for the in-kernel harmonics; not on the hot path). */
 EQCONV_API int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y,

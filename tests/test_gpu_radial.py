@@ -87,3 +87,75 @@ def test_radial_weights_water_box():
     ref = orad.radial_weights(np.linalg.norm(r.astype(np.float64), axis=1), cfg["cutoff"], params, conv.P, cfg["C"])
     assert_close("water box w", got, ref)
     assert np.all(got[dummy] == 0.0)
+
+
+# ------------------------------------------------ fused forward (radial on chip)
+
+def _poisson_case(N, mean_deg, seed):
+    rng = np.random.default_rng(seed)
+    deg = rng.poisson(mean_deg, size=N)
+    deg[::7] = 0                                         # receivers with no in-edges
+    rcv = np.repeat(np.arange(N, dtype=np.int32), deg)
+    snd = rng.integers(0, N, size=rcv.size).astype(np.int32)
+    r = _edges(rcv.size, 5.0, seed + 1)
+    return snd, rcv, r
+
+
+def _fused_forward(conv, N, s, rcv, r, x, params, nb, rc):
+    g = conv.graph(to_dev(s), to_dev(rcv), N)
+    ws_n = B.eqconv_forward_radial_workspace_bytes(conv.plan, N, len(s))
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device="cuda")
+    y = torch.full((N, conv.D_out, conv.C), float("nan"), device="cuda")
+    W1, W2, W3 = (to_dev(p) for p in params)
+    B.eqconv_forward_radial(conv.plan, g.c, to_dev(x), to_dev(r), W1, W2, W3, nb, rc, y, ws, ws_n)
+    torch.cuda.synchronize()
+    assert B.eqconv_get_device_error(conv.plan) == B.EQCONV_OK
+    return y.cpu().numpy()
+
+
+def test_forward_radial_tiny_box_against_bruteforce():
+    """The tiny box (0e+1o -> 0e+1o+2e, L_sh = 2) against the oracle's
+    composition of the radial MLP with the per-edge message brute force."""
+    from oracle import conv as oconv
+    W = wl.WORKLOADS["tiny"]
+    s, rcv, r = wl.make_graph(W)
+    conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    x = wl.features(W.N, prob.D_in, W.C, wl.SEED_X)
+    params = wl.radial_mlp_params(prob.P, W.C, 64, 8, seed=21)
+    got = _fused_forward(conv, W.N, s, rcv, r, x, params, 8, 3.5)
+    want = orad.conv_with_radial(prob, W.N, s, rcv, r, x, 3.5, params)
+    assert_close("y (fused radial, tiny box)", got, want)
+
+
+@pytest.mark.parametrize("L,C,N,per_path", [(1, 32, 300, False), (2, 64, 700, False), (2, 128, 517, True),
+                                            (3, 64, 400, False), (3, 32, 129, True)])
+def test_forward_radial_matches_oracle(L, C, N, per_path):
+    """Several channel slices, one or two path groups (L = 3: 23 paths),
+    ragged receiver ranges, receivers without edges, edges beyond the cutoff
+    and of zero length; summed and per-path output layouts."""
+    from oracle import conv as oconv
+    ins = wl.natural_irreps(L)
+    conv = EqConv(ins, L, ins, C, per_path=per_path)
+    prob = oconv.Problem(ins, L, ins, C, per_path=per_path)
+    s, rcv, r = _poisson_case(N, 12.0, seed=N + C)
+    x = wl.features(N, prob.D_in, C, wl.SEED_X)
+    rc, nb = 5.0, 8
+    params = wl.radial_mlp_params(prob.P, C, 64, nb, seed=31 + L)
+    got = _fused_forward(conv, N, s, rcv, r, x, params, nb, rc)
+    w = orad.radial_weights(np.linalg.norm(r.astype(np.float64), axis=1), rc, params, prob.P, C).astype(np.float32)
+    want = oconv.full(prob, N, s, rcv, r, x, w)
+    assert_close(f"y (fused radial L={L} C={C} N={N} per_path={per_path})", got, want)
+
+
+def test_forward_radial_no_edges_and_unsupported():
+    conv = EqConv("0e+1o+2e", 2, "0e+1o+2e", 32)
+    x = np.ones((5, 9, 32), np.float32)
+    params = wl.radial_mlp_params(conv.P, 32, 64, 8)
+    got = _fused_forward(conv, 5, np.zeros(0, np.int32), np.zeros(0, np.int32), np.zeros((0, 3), np.float32), x,
+                         params, 8, 5.0)
+    assert np.all(got == 0.0)
+    odd = EqConv("0e+1o", 1, "0e+1o", 32)          # (1, 1, 1) is compiled; (2, 1, 2) is not
+    assert B.eqconv_forward_radial_workspace_bytes(odd.plan, 10, 10) > 0
+    other = EqConv("0e+1o+2e", 1, "0e+1o+2e", 32)
+    assert B.eqconv_forward_radial_workspace_bytes(other.plan, 10, 10) == 0
