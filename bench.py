@@ -250,7 +250,7 @@ def waterbox_leg(dev, stream, reps, reduce, warmup=3):
     import torch
 
     from equivariant_gnn_message_edge_b200 import binding as B
-    from equivariant_gnn_message_edge_b200.conv import EqConv
+    from equivariant_gnn_message_edge_b200.conv import EqConv, RadialEqConv
     cfg = wl.WATER_BOX
     ins = wl.natural_irreps(cfg["L"])
     C, N, rc = cfg["C"], cfg["n_atoms"], cfg["cutoff"]
@@ -271,35 +271,152 @@ def waterbox_leg(dev, stream, reps, reduce, warmup=3):
         readout = to(wl.features(N, conv.D_out, C, wl.SEED_GY))
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    def step():
+    rconv = RadialEqConv(ins, cfg["L"], ins, C, n_basis=cfg["n_bessel"], r_cut=rc)
+
+    def step_unfused():
         p = pos_d.detach().requires_grad_(True)
         Ws = [[t.detach().requires_grad_(True) for t in ps] for ps in params]
         r = p[s_l] - p[r_l] + shift_d
         y1 = conv(g, x1, r, radial_weights_torch(r, rc, Ws[0], P, C))
         y2 = conv(g, y1 / avg, r, radial_weights_torch(r, rc, Ws[1], P, C))
         e = (y2 * readout).sum()
-        grads = torch.autograd.grad(e, [p] + Ws[0] + Ws[1])
-        return grads
+        return torch.autograd.grad(e, [p] + Ws[0] + Ws[1])
 
-    ms = []
-    with torch.cuda.stream(stream):
-        for k in range(warmup + reps):
-            flush.fill_(k & 0xFF)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            step()
-            b.record(stream)
-            if k >= warmup:
-                ms.append((a, b))
-    stream.synchronize()
-    assert B.eqconv_get_device_error(conv.plan, stream.cuda_stream) == B.EQCONV_OK
-    t = reduce(statistics.median([a.elapsed_time(b) for a, b in ms]))
+    def step_fused():
+        p = pos_d.detach().requires_grad_(True)
+        Ws = [[t.detach().requires_grad_(True) for t in ps] for ps in params]
+        r = p[s_l] - p[r_l] + shift_d
+        y1 = rconv(g, x1, r, *Ws[0])
+        y2 = rconv(g, y1 / avg, r, *Ws[1])
+        e = (y2 * readout).sum()
+        return torch.autograd.grad(e, [p] + Ws[0] + Ws[1])
+
+    def timed(fn):
+        ms = []
+        launches0 = B.eqconv_launch_count()
+        with torch.cuda.stream(stream):
+            for k in range(warmup + reps):
+                flush.fill_(k & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                if k >= warmup:
+                    ms.append((a, b))
+        stream.synchronize()
+        assert B.eqconv_get_device_error(conv.plan, stream.cuda_stream) == B.EQCONV_OK
+        launches = (B.eqconv_launch_count() - launches0) // (warmup + reps)
+        return reduce(statistics.median([a.elapsed_time(b) for a, b in ms])), launches
+
+    t_u, _ = timed(step_unfused)
+    t_f, l_f = timed(step_fused)
     return {"atoms": N, "edges": int(len(s)), "dummy_edges": int(dummy.sum()), "C": C, "L": cfg["L"], "P": P,
-            "unfused_ms_per_step": round(t, 4),
+            "ms_per_step": round(t_f, 4), "unfused_ms_per_step": round(t_u, 4),
+            "speedup_vs_unfused": round(t_u / t_f, 2), "libeqconv_launches_per_step": int(l_f),
+            "fused": "libeqconv eqconv_forward_radial / eqconv_backward_radial per layer (radial MLP on the "
+                     "chip: w and dw never in memory) + torch autograd for positions -> edge vectors and the "
+                     "readout",
             "unfused": "radial MLP in fp32 torch ops (cuBLAS GEMMs, TF32 off) writing w [E][P][C] to HBM per "
                        "layer + libeqconv forward/backward (deterministic) + torch autograd glue",
             "step": "2 conv layers forward + gradient of <gy, y2> w.r.t. positions (forces) and MLP weights; "
                     "L2 flushed between steps"}
+
+
+def radial_leg(name, dev, stream, reps, reduce, warmup=3):
+    """The convolution of workload `name` with radial-MLP weights (8 Bessel
+    functions, 8 -> 64 -> 64 -> P*C SiLU MLP, 5 A cutoff): the fused path
+    (eqconv_forward_radial / eqconv_backward_radial: w and dw never in
+    memory) against the unfused one (the same MLP in fp32 torch ops writing
+    w to memory, libeqconv's forward and backward, torch autograd for the
+    MLP), each forward and forward+backward."""
+    import torch
+
+    from equivariant_gnn_message_edge_b200 import binding as B
+    from equivariant_gnn_message_edge_b200.conv import EqConv, RadialEqConv
+    W = wl.WORKLOADS[name]
+    rc, nb = 5.0, 8
+    rconv = RadialEqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C, n_basis=nb, r_cut=rc)
+    conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    P, D_in, D_out, C = conv.P, conv.D_in, conv.D_out, W.C
+    torch.backends.cuda.matmul.allow_tf32 = False
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    with torch.cuda.stream(stream):
+        s, rcv, r = wl.make_graph(W)
+        E = len(s)
+        s_d, r_d, rv = to(s), to(rcv), to(r)
+        g = conv.graph(s_d, r_d, W.N, stream=stream)
+        gen = torch.Generator(device=dev).manual_seed(wl.SEED_X + 200)
+        x = torch.randn((W.N, D_in, C), generator=gen, device=dev)
+        gy = torch.randn((W.N, D_out, C), generator=gen, device=dev)
+        params = [to(p) for p in wl.radial_mlp_params(P, C, 64, nb)]
+        y = torch.empty((W.N, D_out, C), device=dev)
+        fws_n = B.eqconv_forward_radial_workspace_bytes(rconv.plan, W.N, E)
+        bws_n = B.eqconv_backward_radial_workspace_bytes(rconv.plan, W.N, E)
+        fws = torch.empty(fws_n, dtype=torch.uint8, device=dev)
+        bws = torch.empty(bws_n, dtype=torch.uint8, device=dev)
+        dx, dr = torch.empty_like(x), torch.empty_like(rv)
+        gW = [torch.empty_like(p) for p in params]
+    h = stream.cuda_stream
+
+    def fused_fwd():
+        B.eqconv_forward_radial(rconv.plan, g.c, x, rv, *params, nb, rc, y, fws, fws_n, h)
+
+    def fused_bwd():
+        B.eqconv_backward_radial(rconv.plan, g.c, x, rv, *params, nb, rc, gy, dx, dr, *gW, bws, bws_n, h)
+
+    def unfused_fwd():
+        w = radial_weights_torch(rv, rc, params, P, C)
+        B.eqconv_forward(conv.plan, g.c, x, rv, w, y, 0, h)
+
+    def unfused_fwd_bwd():
+        xr = x.detach().requires_grad_(True)
+        rr = rv.detach().requires_grad_(True)
+        Ws = [p.detach().requires_grad_(True) for p in params]
+        yy = conv(g, xr, rr, radial_weights_torch(rr, rc, Ws, P, C))
+        return torch.autograd.grad(yy, [xr, rr] + Ws, gy)
+
+    def timed(fn):
+        out = []
+        with torch.cuda.stream(stream):
+            for k in range(warmup + reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                if k >= warmup:
+                    out.append((a, b))
+        stream.synchronize()
+        return reduce(statistics.median([a.elapsed_time(b) for a, b in out]))
+
+    t_ff, t_fb = timed(fused_fwd), timed(fused_bwd)
+    t_uf, t_ufb = timed(unfused_fwd), timed(unfused_fwd_bwd)
+    assert B.eqconv_get_device_error(rconv.plan, h) == B.EQCONV_OK
+    flop = 6.0 * E * 64 * P * C          # 3 fp16 products, 2 flop per multiply-add, per forward GEMM
+    peak_tc = measured_tensor_peak()
+    out = {"N": W.N, "E": E, "C": C, "P": P, "radial": "8 Bessel, 8 -> 64 -> 64 -> P*C SiLU MLP, 5 A cutoff",
+           "fused_ms": {"fwd": round(t_ff, 4), "bwd": round(t_fb, 4), "fwd_bwd": round(t_ff + t_fb, 4)},
+           "unfused_ms": {"fwd": round(t_uf, 4), "fwd_bwd": round(t_ufb, 4)},
+           "speedup_fwd": round(t_uf / t_ff, 2), "speedup_fwd_bwd": round(t_ufb / (t_ff + t_fb), 2),
+           "roofline_fwd_tensor": {"bound": "tensor", "achieved": round(flop / (t_ff * 1e-3) / 1e12, 1),
+                                   "peak": peak_tc[0], "unit": "TFLOP/s",
+                                   "frac": round(flop / (t_ff * 1e-3) / 1e12 / peak_tc[0], 4),
+                                   "flop": "6 E 64 P C: the last layer's three fp16 products (the whole fused "
+                                           "forward timed)", "peak_kind": peak_tc[1]},
+           "unfused": "radial MLP in fp32 torch ops (cuBLAS, TF32 off) writing w to memory + libeqconv "
+                      "forward/backward + torch autograd for the MLP"}
+    del fws, bws, x, gy, y, dx, dr
+    torch.cuda.empty_cache()
+    return out
+
+
+def measured_tensor_peak():
+    """Dense f16 / bf16 tensor peak (TFLOP/s): the measured cuBLAS bf16 burst
+    figure (f16 runs at the bf16 rate), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (bf16 burst; f16 has the same rate)"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def dbl_bytes(N, E, C, D_in, D_out, P, part_bytes):
@@ -659,6 +776,8 @@ def run_native(args, rank, world, local_rank):
                           for c in (64, 128, 256, 512, 1024)]
     if "waterbox" in want:
         legs["waterbox"] = waterbox_leg(dev, stream, reps, red)
+    if "radial" in want:
+        legs["radial_lmax2"] = radial_leg("lmax2", dev, stream, reps, red)
 
     peak, peak_kind = measured_peak()
     ms_step = t_max / args.steps
@@ -868,9 +987,9 @@ def main():
     ap.add_argument("--no-node-product", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
-    ap.add_argument("--legs", default="lmax3,sweep,waterbox",
+    ap.add_argument("--legs", default="lmax3,sweep,waterbox,radial",
                     help="other stated workloads to time after the main step (comma list of lmax3, sweep, "
-                         "waterbox; empty for none)")
+                         "waterbox, radial; empty for none)")
     ap.add_argument("--nodes", type=int, default=None,
                     help="override the workload's node count (smaller profiling captures)")
     args = ap.parse_args()

@@ -39,6 +39,9 @@ ABI_FUNCTIONS = (
     "eqconv_node_product_plan_create", "eqconv_node_product", "eqconv_node_product_workspace_bytes",
     "eqconv_node_product_backward", "eqconv_radial_workspace_bytes", "eqconv_radial_weights",
     "eqconv_forward_radial_workspace_bytes", "eqconv_forward_radial",
+    "eqconv_backward_radial_workspace_bytes", "eqconv_backward_radial",
+    "eqconv_symmetric_contraction_plan_create", "eqconv_symmetric_contraction",
+    "eqconv_symmetric_contraction_workspace_bytes", "eqconv_symmetric_contraction_backward",
 )
 
 
@@ -91,6 +94,13 @@ _SIGS = {
     "eqconv_spherical_harmonics": (_ci, [_vp, _ci, _vp, _vp, _vp]),
     "eqconv_radial_workspace_bytes": (_sz, [_vp, _ci]),
     "eqconv_forward_radial_workspace_bytes": (_sz, [_vp, _ci, _ci]),
+    "eqconv_symmetric_contraction_plan_create": (_ci, [ctypes.POINTER(_vp), ctypes.c_char_p, ctypes.c_char_p, _ci,
+                                                       _ci]),
+    "eqconv_symmetric_contraction": (_ci, [_vp, _ci] + [_vp] * 5 + [_vp]),
+    "eqconv_symmetric_contraction_workspace_bytes": (_sz, [_vp, _ci]),
+    "eqconv_symmetric_contraction_backward": (_ci, [_vp, _ci] + [_vp] * 9 + [_sz, _vp]),
+    "eqconv_backward_radial_workspace_bytes": (_sz, [_vp, _ci, _ci]),
+    "eqconv_backward_radial": (_ci, [_vp, _pg] + [_vp] * 5 + [_ci, ctypes.c_float] + [_vp] * 7 + [_sz, _vp]),
     "eqconv_forward_radial": (_ci, [_vp, _pg] + [_vp] * 5 + [_ci, ctypes.c_float, _vp, _vp, _sz, _vp]),
     "eqconv_radial_weights": (_ci, [_vp, _ci] + [_vp] * 4 + [_ci, ctypes.c_float, _vp, _vp, _sz, _vp]),
     "eqconv_get_device_error": (_ci, [_vp, _vp, _pi]),
@@ -336,6 +346,48 @@ def eqconv_forward_radial(plan: int, graph: eqconv_graph_t, x, r, W1, W2, W3, n_
     _check(lib().eqconv_forward_radial(plan, ctypes.byref(graph), _ptr(x, f), _ptr(r, f), _ptr(W1, f), _ptr(W2, f),
                                        _ptr(W3, f), int(n_basis), float(r_cut), _ptr(y, f), _ptr(workspace),
                                        int(workspace_bytes), _stream(stream)), "eqconv_forward_radial")
+
+
+def eqconv_backward_radial_workspace_bytes(plan: int, N: int, E: int) -> int:
+    return int(lib().eqconv_backward_radial_workspace_bytes(plan, int(N), int(E)))
+
+
+def eqconv_backward_radial(plan: int, graph: eqconv_graph_t, x, r, W1, W2, W3, n_basis: int, r_cut: float, gy,
+                           dx, dr, gW1, gW2, gW3, workspace, workspace_bytes: int, stream=None) -> None:
+    f = _f32()
+    _check(lib().eqconv_backward_radial(plan, ctypes.byref(graph), _ptr(x, f), _ptr(r, f), _ptr(W1, f), _ptr(W2, f),
+                                        _ptr(W3, f), int(n_basis), float(r_cut), _ptr(gy, f), _ptr(dx, f),
+                                        _ptr(dr, f), _ptr(gW1, f), _ptr(gW2, f), _ptr(gW3, f), _ptr(workspace),
+                                        int(workspace_bytes), _stream(stream)), "eqconv_backward_radial")
+
+
+def eqconv_symmetric_contraction_plan_create(irreps_A: str, irreps_out: str, C: int, n_species: int) -> int:
+    h = _vp()
+    _check(lib().eqconv_symmetric_contraction_plan_create(ctypes.byref(h), irreps_A.encode(), irreps_out.encode(),
+                                                          int(C), int(n_species)),
+           "eqconv_symmetric_contraction_plan_create")
+    return h.value
+
+
+def eqconv_symmetric_contraction(plan: int, N: int, A, species, W1, W2, B_out, stream=None) -> None:
+    f = _f32()
+    _check(lib().eqconv_symmetric_contraction(plan, int(N), _ptr(A, f), _ptr(species, _i32()), _ptr(W1, f),
+                                              _ptr(W2, f), _ptr(B_out, f), _stream(stream)),
+           "eqconv_symmetric_contraction")
+
+
+def eqconv_symmetric_contraction_workspace_bytes(plan: int, N: int) -> int:
+    return int(lib().eqconv_symmetric_contraction_workspace_bytes(plan, int(N)))
+
+
+def eqconv_symmetric_contraction_backward(plan: int, N: int, A, species, W1, W2, gB, dA, dW1, dW2, workspace,
+                                          workspace_bytes: int, stream=None) -> None:
+    f = _f32()
+    _check(lib().eqconv_symmetric_contraction_backward(plan, int(N), _ptr(A, f), _ptr(species, _i32()), _ptr(W1, f),
+                                                       _ptr(W2, f), _ptr(gB, f), _ptr(dA, f), _ptr(dW1, f),
+                                                       _ptr(dW2, f), _ptr(workspace), int(workspace_bytes),
+                                                       _stream(stream)),
+           "eqconv_symmetric_contraction_backward")
 
 
 def eqconv_spherical_harmonics(plan: int, E: int, r, Y, stream=None) -> None:

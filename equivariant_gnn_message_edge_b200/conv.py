@@ -148,6 +148,65 @@ class _EqConvBwdFn(torch.autograd.Function):
         return None, None, None, g_x, g_r, g_w, g_gy
 
 
+class RadialEqConv:
+    """The convolution with its weights produced on the chip from the edge
+    lengths by the radial MLP (Bessel basis, C2 envelope, 2 SiLU layers of
+    width 64; see include/eqconv.h, eqconv_forward_radial):
+
+        conv = RadialEqConv("0e+1o+2e+3o", 3, "0e+1o+2e+3o", C=128, n_basis=8, r_cut=5.0)
+        y = conv(g, x, r, W1, W2, W3)       # differentiable in x, r, W1, W2, W3
+
+    The backward runs eqconv_backward_radial (deterministic; w and dw never
+    in memory); it is not twice differentiable."""
+
+    def __init__(self, irreps_in: str, L_sh: int, irreps_out: str, C: int, n_basis: int = 8, r_cut: float = 5.0,
+                 per_path: bool = False):
+        self.conv = EqConv(irreps_in, L_sh, irreps_out, C, per_path=per_path)
+        self.plan, self.P, self.D_in, self.D_out, self.C = (self.conv.plan, self.conv.P, self.conv.D_in,
+                                                            self.conv.D_out, C)
+        self.n_basis, self.r_cut = int(n_basis), float(r_cut)
+        if B.eqconv_forward_radial_workspace_bytes(self.plan, 1, 1) == 0:
+            raise B.EqconvError("RadialEqConv: no fused radial path for this plan", B.EQCONV_ERR_UNSUPPORTED)
+
+    def graph(self, senders, receivers, N, stream=None) -> Graph:
+        return self.conv.graph(senders, receivers, N, stream)
+
+    def forward_raw(self, g: Graph, x, r, W1, W2, W3, y=None, stream=None):
+        if y is None:
+            y = torch.empty((g.N, self.D_out, self.C), dtype=torch.float32, device=x.device)
+        nbytes = B.eqconv_forward_radial_workspace_bytes(self.plan, g.N, g.E)
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+        B.eqconv_forward_radial(self.plan, g.c, x, r, W1, W2, W3, self.n_basis, self.r_cut, y, ws, nbytes, stream)
+        return y
+
+    def backward_raw(self, g: Graph, x, r, W1, W2, W3, gy, stream=None):
+        dx, dr = torch.empty_like(x), torch.empty_like(r)
+        gW1, gW2, gW3 = torch.empty_like(W1), torch.empty_like(W2), torch.empty_like(W3)
+        nbytes = B.eqconv_backward_radial_workspace_bytes(self.plan, g.N, g.E)
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+        B.eqconv_backward_radial(self.plan, g.c, x, r, W1, W2, W3, self.n_basis, self.r_cut, gy, dx, dr, gW1, gW2,
+                                 gW3, ws, nbytes, stream)
+        return dx, dr, gW1, gW2, gW3
+
+    def __call__(self, g: Graph, x, r, W1, W2, W3):
+        return _RadialEqConvFn.apply(self, g, x, r, W1, W2, W3)
+
+
+class _RadialEqConvFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, op: RadialEqConv, g: Graph, x, r, W1, W2, W3):
+        args = [t.contiguous() for t in (x, r, W1, W2, W3)]
+        ctx.op, ctx.g = op, g
+        ctx.save_for_backward(*args)
+        return op.forward_raw(g, *args)
+
+    @staticmethod
+    def backward(ctx, gy):
+        x, r, W1, W2, W3 = ctx.saved_tensors
+        dx, dr, gW1, gW2, gW3 = ctx.op.backward_raw(ctx.g, x, r, W1, W2, W3, gy.contiguous())
+        return None, None, dx, dr, gW1, gW2, gW3
+
+
 class NodeProduct:
     """Node-local channel-diagonal product of two node features (see
     include/eqconv.h): y = sum_p w_p C_p u_l1 v_l2, summed per output irrep or
@@ -205,3 +264,63 @@ class _NodeProductFn(torch.autograd.Function):
         need_dw = ctx.has_w and ctx.needs_input_grad[3]
         du, dv, dw = ctx.op.backward_raw(u, v, w, gy.contiguous(), need_dw=need_dw)
         return None, du, dv, dw
+
+
+class SymmetricContraction:
+    """Symmetric contraction of correlation order 2 with per-species weights
+    (the MACE product basis; see include/eqconv.h):
+
+        sc = SymmetricContraction("0e+1o+2e+3o", "0e+1o", C=128, n_species=2)
+        B = sc(A, species, W1, W2)           # differentiable in A, W1, W2
+
+    W1 [S][min(L_A, L_out)+1][C], W2 [S][P][C] with P = len(sc.paths)."""
+
+    def __init__(self, irreps_A: str, irreps_out: str, C: int, n_species: int):
+        self.C, self.S = C, n_species
+        self.plan = B.eqconv_symmetric_contraction_plan_create(irreps_A, irreps_out, C, n_species)
+        info = B.eqconv_plan_info(self.plan)
+        self.P, self.D_A, self.D_out, self.paths = info["P"], info["D_in"], info["D_out"], info["paths"]
+        L_A = int(round(self.D_A ** 0.5)) - 1
+        L_out = int(round(self.D_out ** 0.5)) - 1
+        self.L1N = min(L_A, L_out) + 1
+
+    def __del__(self):
+        try:
+            B.eqconv_plan_destroy(self.plan)
+        except Exception:
+            pass
+
+    def forward_raw(self, A, species, W1, W2, out=None, stream=None):
+        N = A.shape[0]
+        if out is None:
+            out = torch.empty((N, self.D_out, self.C), dtype=torch.float32, device=A.device)
+        B.eqconv_symmetric_contraction(self.plan, N, A, species, W1, W2, out, stream)
+        return out
+
+    def backward_raw(self, A, species, W1, W2, gB, stream=None):
+        N = A.shape[0]
+        dA, dW1, dW2 = torch.empty_like(A), torch.empty_like(W1), torch.empty_like(W2)
+        nbytes = B.eqconv_symmetric_contraction_workspace_bytes(self.plan, N)
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=A.device)
+        B.eqconv_symmetric_contraction_backward(self.plan, N, A, species, W1, W2, gB, dA, dW1, dW2, ws, nbytes,
+                                                stream)
+        return dA, dW1, dW2
+
+    def __call__(self, A, species, W1, W2):
+        return _SymContractionFn.apply(self, A, species, W1, W2)
+
+
+class _SymContractionFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, op: SymmetricContraction, A, species, W1, W2):
+        A, W1, W2 = A.contiguous(), W1.contiguous(), W2.contiguous()
+        ctx.op = op
+        ctx.save_for_backward(A, species, W1, W2)
+        return op.forward_raw(A, species, W1, W2)
+
+    @staticmethod
+    def backward(ctx, gB):
+        A, species, W1, W2 = ctx.saved_tensors
+        dA, dW1, dW2 = ctx.op.backward_raw(A, species, W1, W2, gB.contiguous())
+        return None, dA, None, dW1, dW2
+

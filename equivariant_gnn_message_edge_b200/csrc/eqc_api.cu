@@ -27,6 +27,8 @@
 #include "eqc_graph.h"
 #include "eqc_radial.h"
 #include "eqc_radial_conv.h"
+#include "eqc_symc.cuh"
+#include "eqc_symc.h"
 #include "eqconv.h"
 
 namespace eqc {
@@ -101,6 +103,8 @@ struct eqconv_plan_s {
     const eqc::DblKernelSet* dbl_ks;   // double backward (summed natural-parity outputs only)
     bool node_product;                 // a node-local product plan (no convolution)
     const eqc::NpKernelSet* np_ks;     // node-local product
+    const eqc::SymKernelSet* symc_ks;  // symmetric contraction (then node_product is true too)
+    int n_species;
 };
 
 namespace {
@@ -590,6 +594,110 @@ int eqconv_double_backward(eqconv_plan_t plan, const eqconv_graph_t* g, const fl
     return cuda_status(plan->dbl_ks->run(recv, send, (cudaStream_t)stream), "double backward");
 }
 
+int eqconv_symmetric_contraction_plan_create(eqconv_plan_t* out, const char* irreps_A, const char* irreps_out, int C,
+                                             int n_species) {
+    if (!out) return EQCONV_ERR_INVALID_ARG;
+    *out = nullptr;
+    const int la = parse_natural_prefix(irreps_A), lout = parse_natural_prefix(irreps_out);
+    if (la == -1 || lout == -1 || C <= 0 || n_species < 1) return EQCONV_ERR_INVALID_ARG;
+    if (la == -2 || lout == -2 || C % 4 != 0 || C > 4096 || n_species > eqc::kSymMaxSpecies)
+        return EQCONV_ERR_UNSUPPORTED;
+    const eqc::SymKernelSet* ks = eqc::find_symc(la, lout);
+    if (!ks || ks->np == 0) return EQCONV_ERR_UNSUPPORTED;
+    eqconv_plan_s* p = new (std::nothrow) eqconv_plan_s();
+    if (!p) return EQCONV_ERR_CUDA;
+    p->lin = la;
+    p->lsh = la;
+    p->lout = lout;
+    p->C = C;
+    p->mode = 0;
+    p->P = ks->np;
+    p->D_in = ks->d_a;
+    p->D_sh = ks->d_a;
+    p->D_out = ks->d_out;
+    for (int i = 0; i < ks->np; ++i) {
+        for (int k = 0; k < 3; ++k) p->paths[i][k] = ks->paths[i][k];
+        p->path_rows[i] = ks->paths[i][2] * ks->paths[i][2];
+    }
+    p->node_product = true;   // not a convolution plan
+    p->symc_ks = ks;
+    p->n_species = n_species;
+    if (cudaGetDevice(&p->device) != cudaSuccess || cudaMalloc(&p->d_status, sizeof(unsigned)) != cudaSuccess) {
+        delete p;
+        return EQCONV_ERR_CUDA;
+    }
+    if (cudaMemset(p->d_status, 0, sizeof(unsigned)) != cudaSuccess) {
+        cudaFree(p->d_status);
+        delete p;
+        return EQCONV_ERR_CUDA;
+    }
+    *out = p;
+    return EQCONV_OK;
+}
+
+int eqconv_symmetric_contraction(eqconv_plan_t plan, int N, const float* A, const int32_t* species, const float* W1,
+                                 const float* W2, float* B, eqconv_stream_t stream) {
+    if (!plan || N < 0) return EQCONV_ERR_INVALID_ARG;
+    if (!plan->symc_ks) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_device(plan);
+    if (rc != EQCONV_OK) return rc;
+    if (N == 0) return EQCONV_OK;
+    if (!A || !species || !W1 || !W2 || !B || !aligned16(A) || !aligned16(B) || !aligned16(W1) || !aligned16(W2))
+        return EQCONV_ERR_INVALID_ARG;
+    eqc::SymParams prm{};
+    prm.A = A;
+    prm.species = species;
+    prm.W1 = W1;
+    prm.W2 = W2;
+    prm.B = B;
+    prm.N = N;
+    prm.C = plan->C;
+    prm.S = plan->n_species;
+    prm.status = plan->d_status;
+    return cuda_status(plan->symc_ks->fwd(prm, (cudaStream_t)stream), "symmetric contraction");
+}
+
+size_t eqconv_symmetric_contraction_workspace_bytes(eqconv_plan_t plan, int N) {
+    if (!plan || !plan->symc_ks || N < 0) return 0;
+    return plan->symc_ks->workspace(N, plan->C, plan->n_species);
+}
+
+int eqconv_symmetric_contraction_backward(eqconv_plan_t plan, int N, const float* A, const int32_t* species,
+                                          const float* W1, const float* W2, const float* gB, float* dA, float* dW1,
+                                          float* dW2, void* workspace, size_t workspace_bytes,
+                                          eqconv_stream_t stream) {
+    if (!plan || N < 0) return EQCONV_ERR_INVALID_ARG;
+    if (!plan->symc_ks) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_device(plan);
+    if (rc != EQCONV_OK) return rc;
+    if (!W1 || !W2 || !dW1 || !dW2) return EQCONV_ERR_INVALID_ARG;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if (N == 0) {
+        const size_t s = (size_t)plan->n_species * plan->C * sizeof(float);
+        cudaError_t e = cudaMemsetAsync(dW1, 0, s * plan->symc_ks->l1n, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dW2, 0, s * plan->symc_ks->np, st);
+        return cuda_status(e, "symmetric contraction backward, no nodes");
+    }
+    if (!A || !species || !gB || !dA || !aligned16(A) || !aligned16(gB) || !aligned16(dA) || !aligned16(W1) ||
+        !aligned16(W2))
+        return EQCONV_ERR_INVALID_ARG;
+    const size_t need = plan->symc_ks->workspace(N, plan->C, plan->n_species);
+    if (!workspace || workspace_bytes < need) return EQCONV_ERR_WORKSPACE;
+    eqc::SymParams prm{};
+    prm.A = A;
+    prm.species = species;
+    prm.W1 = W1;
+    prm.W2 = W2;
+    prm.gB = gB;
+    prm.dA = dA;
+    prm.dw_part = static_cast<float*>(workspace);
+    prm.N = N;
+    prm.C = plan->C;
+    prm.S = plan->n_species;
+    prm.status = plan->d_status;
+    return cuda_status(plan->symc_ks->bwd(prm, dW1, dW2, st), "symmetric contraction backward");
+}
+
 size_t eqconv_node_product_workspace_bytes(eqconv_plan_t plan, int N) {
     if (!plan || N < 0 || !plan->np_ks) return 0;
     const int need = (N + eqc::kNpWarps - 1) / eqc::kNpWarps;
@@ -714,6 +822,62 @@ int eqconv_forward_radial(eqconv_plan_t plan, const eqconv_graph_t* g, const flo
     a.C = plan->C;
     a.status = plan->d_status;
     return cuda_status(rs->fwd(a, (cudaStream_t)stream), "forward (radial)");
+}
+
+size_t eqconv_backward_radial_workspace_bytes(eqconv_plan_t plan, int N, int E) {
+    const eqc::radial::RadConvSet* rs = radial_set(plan);
+    if (!rs || N < 0 || E < 0 || plan->C % 32 != 0) return 0;
+    return rs->bwd_workspace(N, E, plan->C);
+}
+
+int eqconv_backward_radial(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r,
+                           const float* W1, const float* W2, const float* W3, int n_basis, float r_cut,
+                           const float* gy, float* dx, float* dr, float* gW1, float* gW2, float* gW3,
+                           void* workspace, size_t workspace_bytes, eqconv_stream_t stream) {
+    if (!plan || plan->node_product) return EQCONV_ERR_INVALID_ARG;
+    int rc = check_graph(g);
+    if (rc != EQCONV_OK) return rc;
+    if ((rc = check_device(plan)) != EQCONV_OK) return rc;
+    const eqc::radial::RadConvSet* rs = radial_set(plan);
+    if (!rs || plan->C % 32 != 0) return EQCONV_ERR_UNSUPPORTED;
+    if (n_basis < 1 || n_basis > eqc::radial::kMaxBasisHost || !(r_cut > 0.f)) return EQCONV_ERR_INVALID_ARG;
+    if (!W1 || !W2 || !W3 || !gW1 || !gW2 || !gW3) return EQCONV_ERR_INVALID_ARG;
+    if (g->N == 0) {
+        const cudaStream_t st = (cudaStream_t)stream;
+        cudaError_t e = cudaMemsetAsync(gW1, 0, (size_t)n_basis * 64 * 4, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(gW2, 0, (size_t)64 * 64 * 4, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(gW3, 0, (size_t)64 * plan->P * plan->C * 4, st);
+        return cuda_status(e, "backward (radial), no nodes");
+    }
+    if (!x || !gy || !dx || (g->E > 0 && (!r || !dr))) return EQCONV_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gy) || !aligned16(dx)) return EQCONV_ERR_INVALID_ARG;
+    const size_t need = rs->bwd_workspace(g->N, g->E, plan->C);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return EQCONV_ERR_WORKSPACE;
+    eqc::radial::RadBwdArgs a{};
+    a.x = x;
+    a.r = r;
+    a.gy = gy;
+    a.send_ptr = g->send_ptr;
+    a.send_perm = g->send_perm;
+    a.receivers = g->receivers;
+    a.W1 = W1;
+    a.W2 = W2;
+    a.W3 = W3;
+    a.NB = n_basis;
+    a.rc = r_cut;
+    a.dx = dx;
+    a.dr = dr;
+    a.gW1 = gW1;
+    a.gW2 = gW2;
+    a.gW3 = gW3;
+    a.per_path = (plan->mode & eqc::kModePerPath) != 0;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    a.N = g->N;
+    a.E = g->E;
+    a.C = plan->C;
+    a.status = plan->d_status;
+    return cuda_status(rs->bwd(a, (cudaStream_t)stream), "backward (radial)");
 }
 
 int eqconv_spherical_harmonics(eqconv_plan_t plan, int E, const float* r, float* Y, eqconv_stream_t stream) {

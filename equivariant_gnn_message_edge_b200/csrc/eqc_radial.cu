@@ -56,77 +56,88 @@ __global__ void __launch_bounds__(1024)
 
 // For output position k (edge e = perm[k], or k without perm): the two
 // hidden layers on the CUDA cores, then h2 split into fp16 pairs with its own
-// power of two (H_hi / H_lo [E][64]), and uscale[k] = u(d) * 2^-(s_W3 +
-// s_h2).  One thread per edge; W1 and W2 are read from shared memory by all
-// threads at once (broadcast).
+// power of two s (H_hi / H_lo [E][64]), uscale[k] = u(d) 2^-(s_W3 + s) (so
+// that w = D * uscale) and zscale[k] = 2^-(s_W3 + s) (may be null).  hmax
+// (may be null) receives the largest |h2| of all edges (as the bits of a
+// non-negative float, by atomicMax).  One thread per edge; W1 and W2 are read
+// from shared memory by all threads at once.
 __global__ void __launch_bounds__(128)
     radial_hidden_kernel(const float* __restrict__ r, const int* __restrict__ perm, int E,
                          const float* __restrict__ W1, const float* __restrict__ W2, int NB, float rc,
                          const float* __restrict__ w3_inv_scale, __half* __restrict__ H_hi,
-                         __half* __restrict__ H_lo, float* __restrict__ uscale) {
+                         __half* __restrict__ H_lo, float* __restrict__ uscale, float* __restrict__ zscale,
+                         unsigned* __restrict__ hmax) {
     __shared__ __align__(16) float sW1[kMaxBasis * kH];
     __shared__ __align__(16) float sW2[kH * kH];
     for (int i = threadIdx.x; i < NB * kH; i += blockDim.x) sW1[i] = W1[i];
     for (int i = threadIdx.x; i < kH * kH; i += blockDim.x) sW2[i] = W2[i];
     __syncthreads();
     const int k = blockIdx.x * blockDim.x + threadIdx.x;
-    if (k >= E) return;
-    const int e = perm ? perm[k] : k;
-    const float rx = r[(size_t)e * 3], ry = r[(size_t)e * 3 + 1], rz = r[(size_t)e * 3 + 2];
-    const float d = sqrtf(fmaf(rx, rx, fmaf(ry, ry, rz * rz)));
-    const float inv_d = 1.f / fmaxf(d, 1e-12f);
-    const float pref = sqrtf(2.f / rc);
-    const float kd = 3.14159265358979323846f * d / rc;
-    float h1[kH];
+    float m = 0.f;   // largest |h2| of this thread's edge
+    if (k < E) {
+        const int e = perm ? perm[k] : k;
+        const float rx = r[(size_t)e * 3], ry = r[(size_t)e * 3 + 1], rz = r[(size_t)e * 3 + 2];
+        const float d = sqrtf(fmaf(rx, rx, fmaf(ry, ry, rz * rz)));
+        const float inv_d = 1.f / fmaxf(d, 1e-12f);
+        const float pref = sqrtf(2.f / rc);
+        const float kd = 3.14159265358979323846f * d / rc;
+        float h1[kH];
 #pragma unroll
-    for (int j = 0; j < kH; ++j) h1[j] = 0.f;
-    for (int nb = 0; nb < NB; ++nb) {
-        const float b = pref * sinf((float)(nb + 1) * kd) * inv_d;
+        for (int j = 0; j < kH; ++j) h1[j] = 0.f;
+        for (int nb = 0; nb < NB; ++nb) {
+            const float b = pref * sinf((float)(nb + 1) * kd) * inv_d;
 #pragma unroll
-        for (int j = 0; j < kH; ++j) h1[j] = fmaf(b, sW1[nb * kH + j], h1[j]);
-    }
+            for (int j = 0; j < kH; ++j) h1[j] = fmaf(b, sW1[nb * kH + j], h1[j]);
+        }
 #pragma unroll
-    for (int j = 0; j < kH; ++j) h1[j] = silu(h1[j]);
-    float h2[kH];
+        for (int j = 0; j < kH; ++j) h1[j] = silu(h1[j]);
+        float h2[kH];
 #pragma unroll
-    for (int j = 0; j < kH; ++j) h2[j] = 0.f;
+        for (int j = 0; j < kH; ++j) h2[j] = 0.f;
 #pragma unroll 4
-    for (int q = 0; q < kH; ++q) {
-        const float a = h1[q];
+        for (int q = 0; q < kH; ++q) {
+            const float a = h1[q];
 #pragma unroll
-        for (int j = 0; j < kH; j += 4) {
-            const float4 wv = *reinterpret_cast<const float4*>(&sW2[q * kH + j]);
-            h2[j] = fmaf(a, wv.x, h2[j]);
-            h2[j + 1] = fmaf(a, wv.y, h2[j + 1]);
-            h2[j + 2] = fmaf(a, wv.z, h2[j + 2]);
-            h2[j + 3] = fmaf(a, wv.w, h2[j + 3]);
+            for (int j = 0; j < kH; j += 4) {
+                const float4 wv = *reinterpret_cast<const float4*>(&sW2[q * kH + j]);
+                h2[j] = fmaf(a, wv.x, h2[j]);
+                h2[j + 1] = fmaf(a, wv.y, h2[j + 1]);
+                h2[j + 2] = fmaf(a, wv.z, h2[j + 2]);
+                h2[j + 3] = fmaf(a, wv.w, h2[j + 3]);
+            }
         }
-    }
-    float m = 0.f;
 #pragma unroll
-    for (int j = 0; j < kH; ++j) {
-        h2[j] = silu(h2[j]);
-        m = fmaxf(m, fabsf(h2[j]));
-    }
-    const int s = pow2_exponent_for(m);
-    const float sc = ldexpf(1.f, s);
-    uint4* dh = reinterpret_cast<uint4*>(H_hi + (size_t)k * kH);
-    uint4* dl = reinterpret_cast<uint4*>(H_lo + (size_t)k * kH);
-#pragma unroll
-    for (int q = 0; q < kH / 8; ++q) {
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            __half h0, l0, h1v, l1v;
-            split_f16(h2[8 * q + 2 * t] * sc, h0, l0);
-            split_f16(h2[8 * q + 2 * t + 1] * sc, h1v, l1v);
-            hw[t] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1v) << 16);
-            lw[t] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1v) << 16);
+        for (int j = 0; j < kH; ++j) {
+            h2[j] = silu(h2[j]);
+            m = fmaxf(m, fabsf(h2[j]));
         }
-        dh[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        dl[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        const int s = pow2_exponent_for(m);
+        const float sc = ldexpf(1.f, s);
+        uint4* dh = reinterpret_cast<uint4*>(H_hi + (size_t)k * kH);
+        uint4* dl = reinterpret_cast<uint4*>(H_lo + (size_t)k * kH);
+#pragma unroll
+        for (int q = 0; q < kH / 8; ++q) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                __half h0, l0, h1v, l1v;
+                split_f16(h2[8 * q + 2 * t] * sc, h0, l0);
+                split_f16(h2[8 * q + 2 * t + 1] * sc, h1v, l1v);
+                hw[t] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1v) << 16);
+                lw[t] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1v) << 16);
+            }
+            dh[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            dl[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+        const float z = ldexpf(1.f, -s) * w3_inv_scale[0];
+        uscale[k] = envelope(d, rc) * z;
+        if (zscale) zscale[k] = z;
     }
-    uscale[k] = envelope(d, rc) * ldexpf(1.f, -s) * w3_inv_scale[0];
+    if (hmax) {   // blockDim is a multiple of 32: every lane of the warp is here
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(hmax, __float_as_uint(m));
+    }
 }
 
 // ------------------------------------------- last layer to w (standalone)
@@ -269,6 +280,8 @@ Workspace carve(void* ws, int E, int PC) {
     p += h;
     w.uscale = reinterpret_cast<float*>(p);
     p += up256((size_t)(E > 0 ? E : 1) * 4);
+    w.zscale = reinterpret_cast<float*>(p);
+    p += up256((size_t)(E > 0 ? E : 1) * 4);
     w.bytes = (size_t)(p - static_cast<char*>(ws));
     return w;
 }
@@ -276,13 +289,13 @@ Workspace carve(void* ws, int E, int PC) {
 size_t workspace_bytes(int E, int PC) { return carve(nullptr, E, PC).bytes; }
 
 cudaError_t prepare(const Workspace& ws, const float* r, const int* perm, int E, const float* W1, const float* W2,
-                    const float* W3, int NB, float rc, int PC, cudaStream_t st) {
+                    const float* W3, int NB, float rc, int PC, cudaStream_t st, unsigned* hmax) {
     radial_prep_w3_kernel<<<1, 1024, 0, st>>>(W3, PC, ws.a_hi, ws.a_lo, ws.inv_scale);
     count_launch();
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess || E == 0) return err;
     radial_hidden_kernel<<<(E + 127) / 128, 128, 0, st>>>(r, perm, E, W1, W2, NB, rc, ws.inv_scale, ws.h_hi,
-                                                          ws.h_lo, ws.uscale);
+                                                          ws.h_lo, ws.uscale, ws.zscale, hmax);
     count_launch();
     return cudaGetLastError();
 }

@@ -21,7 +21,8 @@
 //   D = A_hi B_hi + A_hi B_lo + A_lo B_hi
 // (the dropped A_lo B_lo is below 2^-22 of the product).  The powers of two
 // put every operand's largest magnitude in [2^13, 2^14): one for all of W3,
-// one per edge for h2; they are undone exactly in the per-edge factor
+// one per edge for h2; they are undone exactly, with the envelope, in the
+// per-edge factor
 //   uscale[e] = u(d) * 2^-(s_W3 + s_h2(e)),   w = D * uscale.
 #pragma once
 

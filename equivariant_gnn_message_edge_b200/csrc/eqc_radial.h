@@ -15,7 +15,8 @@ constexpr int kMaxBasisHost = 16;   // Bessel functions (eqc_radial.cuh kMaxBasi
 //   a_hi, a_lo  [PC][64] fp16   W3^T split into fp16 pairs, scaled by 2^s_W3
 //   inv_scale   [1]             2^-s_W3
 //   h_hi, h_lo  [E][64]  fp16   h2 of every edge (or position) split, scaled per row
-//   uscale      [E]             u(d) * 2^-(s_W3 + s_h2)
+//   uscale      [E]             u(d) 2^-(s_W3 + s_h2)
+//   zscale      [E]             2^-(s_W3 + s_h2)
 struct Workspace {
     __half* a_hi;
     __half* a_lo;
@@ -23,6 +24,7 @@ struct Workspace {
     __half* h_hi;
     __half* h_lo;
     float* uscale;
+    float* zscale;
     size_t bytes;
 };
 
@@ -30,9 +32,12 @@ Workspace carve(void* ws, int E, int PC);
 size_t workspace_bytes(int E, int PC);
 
 // W3 split (one CTA) and the hidden layers of every edge, in the order of
-// `perm` (position k holds edge perm[k]; perm == nullptr: edge order).
+// `perm` (position k holds edge perm[k]; perm == nullptr: edge order):
+// H = split(h2 * 2^s), uscale = u(d) 2^-(s_W3 + s), so w = (W3^T H^T) * uscale;
+// zscale = 2^-(s_W3 + s).  hmax (may be null; zeroed by the caller) receives
+// max |h2| as float bits.
 cudaError_t prepare(const Workspace& ws, const float* r, const int* perm, int E, const float* W1, const float* W2,
-                    const float* W3, int NB, float rc, int PC, cudaStream_t st);
+                    const float* W3, int NB, float rc, int PC, cudaStream_t st, unsigned* hmax = nullptr);
 
 // w [E][PC] from a prepared workspace (edge order), on the tensor cores.
 cudaError_t weights(const Workspace& ws, int E, int PC, float* w, unsigned* status, cudaStream_t st);

@@ -1,0 +1,863 @@
+// Backward of the convolution with on-chip radial weights (sm_100a): dx, the
+// MLP weight gradients and dr through both routes of r, with w and dw never
+// in global memory.
+//
+// With w = u(d) z3, z3 = h2 . W3, and dw the weight gradient of the
+// convolution's VJP (FlashCart, arXiv 2610.06409, §4 / App. D: a
+// sender-ordered pass sums each sender's input gradient deterministically):
+//   g_W3[k, pc] = sum_e h2[e, k] u dw[e, pc]                   (tensor cores)
+//   g_h2[e, k]  = sum_pc W3[k, pc] u dw[e, pc]                 (tensor cores)
+//   g_u[e]      = sum_pc dw[e, pc] z3[e, pc]                   (lane sums)
+//   then the small MLP backward per edge
+//   dr_e = (dY/dr)^T gY[e] + g_d(|r_e|) r_e / |r_e|
+// (FlashCart §2: forces are the energy's gradient in the positions, so both
+// routes of r count).
+//
+// radial_conv_bwd_kernel: one CTA per sender range x 32-channel slice x
+// group of up to 8 paths (2 MMA tiles of 4 paths x 32 channels).  Warps:
+//   * 0..7 (path warps): warp w owns path 8 g + w, its lanes the 32 channels.
+//     For every out-edge of the current sender (positions of the sender
+//     CSR) it reads w from tensor memory, the receiver's gy rows from the
+//     ring, the edge's harmonics, and with h[m1][m2] = sum_m3 C_p gy[m3]:
+//       t[m1] = sum_m2 Y[m2] h,  dw = x . t,  dx += w t,
+//       gY[m2] += w sum_m1 x[m1] h      (summed over the 32 lanes)
+//     u dw goes, scaled and split into fp16 halves, into the G tile
+//     [(path, channel) rows][64 edges] in shared memory;
+//   * 8..11 (reader warps, one per tensor-memory subpartition): copy Gd of
+//     every tile and, at the end, the CTA's g_W3 rows out of tensor memory;
+//   * 12 (one thread): stages W3^T and h2 tiles with TMA and issues the
+//     MMAs: w = W3^T . h2^T, then per tile g_W3 += G . h2 and Gd = W3 . G
+//     (K over the tile's edges / the group's rows), G the tile of u dw;
+//   * 13 (one thread): copies each position's receiver row gy[i, :, slice].
+// Per-path dx blocks, per-edge gY partials, Gd partials and g_W3 partials go
+// to the workspace; radial_bwd_epilogue_kernel and the reductions finish dr,
+// dx and the weight gradients in a fixed order (deterministic).
+//
+// Scaling of u dw for fp16: G = u dw 2^sG 2^-sB(e) (sB(e) the power of two of
+// the edge's h2), with sG chosen from a bound of |dw| (49 max|x| max|gy|:
+// |dw| <= |x_l1| |A_p| |gy_l3| and |A_p|_F <= sqrt((2 l2 + 1)(2 l3 + 1))) and
+// of |h2| so that |G| < 2^14; the per-edge powers of two cancel against those
+// of h2 in g_W3.  g_u = sum_pc dw z3 is summed over the lanes with the
+// harmonic gradient, from z3 in tensor memory, so it needs no division by u.
+#pragma once
+
+#include "eqc_radial_conv.cuh"
+
+namespace eqc {
+namespace radial {
+
+constexpr int kBwdGroupPaths = 8;
+constexpr int kBwdGroupTiles = 2;
+constexpr int kBwdPathWarps = 8;
+constexpr int kBwdReaderWarp0 = 8;
+constexpr int kBwdMmaWarp = 12, kBwdGyWarp = 13;
+constexpr int kBwdThreads = 14 * 32;
+constexpr int kGySlots = 16;
+constexpr uint32_t kColW = 0;       // w: [2 buffers][2 tiles][64]
+constexpr uint32_t kColGW = 256;    // g_W3 accumulators: [2 tiles][64 (k)]
+constexpr uint32_t kColGD = 384;    // Gd: 64 columns (M = 64 layout)
+
+struct RadBwdParams {
+    const float* x;        // [N][D_in][C]
+    const float* r;        // [E][3]
+    const float* gy;       // [N][D_out][C] (the plan's output layout)
+    const int* ptr;        // send_ptr [N+1]
+    const int* perm;       // send_perm [E]
+    const int* receivers;  // [E]
+    const float* uscale;   // [E] by sender position
+    const float* scal;     // [0] 2^-sA; [1..3] bits of max|x|, max|gy|, max|u h2|
+    float* dx_pp;          // [N][DX_PP][C] per-path dx blocks
+    float* gy_part;        // [E][slices][SD2] per-path harmonic-gradient partials
+    float* gd_part;        // [slices * groups][E][64] Gd partials (scaled)
+    float* gw3_part;       // [ranges][P * C][64] g_W3 partials (scaled)
+    int N, C, E, nodes_per_cta;
+    unsigned* status;
+};
+
+// per-path dx rows (2 l1 + 1 each, in path order) and per-edge partial
+// offsets (1 + (2 l2 + 1 if l2 > 0) per path)
+template <class K>
+struct BwdRows {
+    static constexpr int dx_off(int p) {
+        int o = 0;
+        for (int q = 0; q < p; ++q) o += 2 * K::PL.l1[q] + 1;
+        return o;
+    }
+    // per path: [sum of dw z3 (for g_u), then the 2 l2 + 1 harmonic-gradient values if l2 > 0]
+    static constexpr int gy_off(int p) {
+        int o = 0;
+        for (int q = 0; q < p; ++q) o += 1 + (K::PL.l2[q] > 0 ? 2 * K::PL.l2[q] + 1 : 0);
+        return o;
+    }
+    static constexpr int DX_PP = dx_off(K::NP);
+    static constexpr int SD2 = gy_off(K::NP);
+};
+
+__device__ __forceinline__ int inv_pow2_exponent(float v) {   // v = 2^-s -> s
+    int e;
+    frexpf(v, &e);   // v = 0.5 * 2^e
+    return 1 - e;
+}
+
+// Exponent g = sG + sA of the G tile: G = dw * 2^g * uscale_e = u dw 2^sG
+// 2^-sB(e), with sG from the bounds |dw| <= 49 max|x| max|gy|, u <= 1 and
+// 2^-sB(e) <= 2^-13 max|h2|, so that |G| < 2^14.  Computed on the device
+// from the maxima (scal[1..3]) and 2^-sA (scal[0]).
+__device__ __forceinline__ int g_scale_exponent(const float* scal) {
+    const float mx = __uint_as_float(reinterpret_cast<const unsigned*>(scal)[1]);
+    const float mg = __uint_as_float(reinterpret_cast<const unsigned*>(scal)[2]);
+    const float mh = __uint_as_float(reinterpret_cast<const unsigned*>(scal)[3]);
+    const float bound = 49.f * mx * mg * mh;
+    int e = 0;
+    if (bound > 0.f) frexpf(bound, &e);   // bound < 2^e
+    return (27 - e) + inv_pow2_exponent(scal[0]);
+}
+
+template <class K>
+struct RadBwdSmem {
+    static constexpr int A_TILE = kRowTile * kTileRowBytes;               // 16 KB
+    static constexpr int H_TILE = kEdgeTile * kTileRowBytes;              // 8 KB
+    static constexpr int G_TILE = kRowTile * kEdgeTile * 2;               // 16 KB: 128 rows x 64 edges fp16
+    static constexpr int W3_OFF = 0;                                      // [tile][hi, lo]
+    static constexpr int H_OFF = W3_OFF + kBwdGroupTiles * 2 * A_TILE;    // [stage][hi, lo]
+    static constexpr int G_OFF = H_OFF + 2 * 2 * H_TILE;                  // [tile][hi, lo]
+    static constexpr int GY_SLOT = K::D_OUT * kSlice * 4;
+    static constexpr int GY_OFF = G_OFF + kBwdGroupTiles * 2 * G_TILE;
+    static constexpr int YS = (K::D_SH + 3) & ~3;                         // harmonics row (floats)
+    static constexpr int Y_WARP = kBatch * (YS + 4) * 4;                  // + the batch's edge factor
+    // gy ring depth: what fits beside the rest (2 .. kGySlots)
+    static constexpr int FIXED = GY_OFF + kBwdPathWarps * Y_WARP + (14 + 2 * kGySlots) * 8 + 16 + 1024;
+    static constexpr int FIT = (227 * 1024 - FIXED) / GY_SLOT;
+    static constexpr int GYS = FIT > kGySlots ? kGySlots : (FIT < 2 ? 2 : FIT);
+    static constexpr int Y_OFF = GY_OFF + GYS * GY_SLOT;
+    static constexpr int BAR_OFF = Y_OFF + kBwdPathWarps * Y_WARP;
+    // w3, h_full[2], h_empty[2], t_full[2], t_empty[2], g_full, g_empty, gd_full, gd_empty, gw_full,
+    // gy_full[GYS], gy_empty[GYS]
+    static constexpr int NBAR = 14 + 2 * GYS;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int END = MISC_OFF + 16;
+    static constexpr int BYTES = END + 1024;
+    static_assert(BYTES <= 227 * 1024, "fused radial backward: shared memory");
+};
+
+// One fp16 chunk of 8 edges for G row `row` at edge chunk `q8` of a 128 x 64
+// swizzled tile (rows of 128 B, 8-row groups of 1024 B).
+__device__ __forceinline__ uint32_t g_chunk_offset(int row, int q8) {
+    return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((q8 ^ (row & 7)) << 4));
+}
+
+template <class K, int P_>
+__device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* base, uint32_t tmem, int warp,
+                                              int lane, int n0, int n1, int k0, int k1, int c0, int slice,
+                                              int slices, int gexp, volatile int* abort_flag) {
+    using S = RadBwdSmem<K>;
+    using R = BwdRows<K>;
+    constexpr int l1 = K::PL.l1[P_], l2 = K::PL.l2[P_], l3 = K::PL.l3[P_];
+    constexpr int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
+    constexpr int o1 = l1 * l1, o3 = K::PL.o3[P_], o2 = l2 * l2;
+    constexpr int oxp = R::dx_off(P_), ogp = R::gy_off(P_);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::BAR_OFF);
+    uint64_t* t_full = bars + 5;
+    uint64_t* t_empty = bars + 7;
+    uint64_t* g_full = bars + 9;
+    uint64_t* g_empty = bars + 10;
+    uint64_t* gy_full = bars + 14;
+    uint64_t* gy_empty = bars + 14 + S::GYS;
+    float* ys = reinterpret_cast<float*>(base + S::Y_OFF + warp * S::Y_WARP);   // [kBatch][YS + 4]
+    const float* gring = reinterpret_cast<const float*>(base + S::GY_OFF);
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const int tile = warp >> 2;                    // MMA tile of this path
+    const int grow = 32 * (warp & 3) + lane;       // G row (path, channel) inside the tile
+    uint8_t* g_hi = base + S::G_OFF + tile * 2 * S::G_TILE;
+    uint8_t* g_lo = g_hi + S::G_TILE;
+    const float gscale0 = ldexpf(1.f, gexp);       // G / dw = 2^gexp * uscale_e
+    const int C = prm.C;
+    const size_t cl = (size_t)c0 + lane;
+
+    float xv[d1], dxa[d1];
+    int cur = n0;
+    int cur_end = prm.ptr[n0 + 1];
+    auto load_x = [&]() {
+        const float* xs = prm.x + ((size_t)cur * K::D_IN + o1) * C + cl;
+#pragma unroll
+        for (int m = 0; m < d1; ++m) {
+            xv[m] = __ldg(xs + (size_t)m * C);
+            dxa[m] = 0.f;
+        }
+    };
+    auto flush = [&]() {
+        float* dxo = prm.dx_pp + ((size_t)cur * R::DX_PP + oxp) * C + cl;
+#pragma unroll
+        for (int m = 0; m < d1; ++m) __stcs(dxo + (size_t)m * C, dxa[m]);
+    };
+    load_x();
+
+    uint32_t ghi[4], glo[4];   // 8 edges of fp16 G values, packed in pairs
+    const int ntiles = (k1 - k0 + kEdgeTile - 1) / kEdgeTile;
+    for (int j = 0; j < ntiles; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&t_full[s], (uint32_t)(j >> 1) & 1u) || __any_sync(0xffffffffu, *abort_flag)) {
+            if (lane == 0) atomicOr(prm.status, 4u);
+            *abort_flag = 1;
+            return;
+        }
+        tc_fence_after();
+        // the G tile of the previous tile has been read by the MMAs
+        if (j > 0 && !mbar_wait(g_empty, (uint32_t)(j - 1) & 1u)) {
+            if (lane == 0) atomicOr(prm.status, 4u);
+            *abort_flag = 1;
+            return;
+        }
+        const uint32_t tcol = tmem + lane_base + kColW + (uint32_t)((s * kBwdGroupTiles + tile) * kEdgeTile);
+        const int kt = k0 + j * kEdgeTile;
+        const int kt_end = min(k1, kt + kEdgeTile);
+        for (int kb = kt; kb < kt + kEdgeTile; kb += kBatch) {
+            const int nb = max(0, min(kBatch, kt_end - kb));
+            if (lane < nb) {
+                const int k = kb + lane;
+                const int e = prm.perm[k];
+                float ux, uy, uz, il;
+                const bool ok = unit_dir(prm.r[(size_t)e * 3], prm.r[(size_t)e * 3 + 1], prm.r[(size_t)e * 3 + 2],
+                                         ux, uy, uz, il);
+                float Y[K::D_SH];
+                sh_eval<K::LSH>(ok, ux, uy, uz, Y);
+                float* yrow = ys + lane * (S::YS + 4);
+#pragma unroll
+                for (int q = 0; q < K::D_SH; ++q) yrow[q] = Y[q];
+                yrow[S::YS] = prm.uscale[k];
+            }
+            __syncwarp();
+            for (int t = 0; t < kBatch; ++t) {
+                const int k = kb + t;
+                float gval = 0.f;
+                if (t < nb) {
+                    while (k >= cur_end) {   // the current sender's edges are done (empty ones too)
+                        flush();
+                        ++cur;
+                        cur_end = prm.ptr[cur + 1];
+                        load_x();
+                    }
+                    const float* yrow = ys + t * (S::YS + 4);
+                    const float us = yrow[S::YS];
+                    const float Dv = tmem_ld1(tcol + (uint32_t)(k - kt));   // z3 * 2^(sA + sB)
+                    const float w = Dv * us;
+                    const int q = k - k0;
+                    const int slot = q % S::GYS;
+                    if (!mbar_wait(&gy_full[slot], (uint32_t)(q / S::GYS) & 1u) ||
+                        __any_sync(0xffffffffu, *abort_flag)) {
+                        if (lane == 0) atomicOr(prm.status, 4u);
+                        *abort_flag = 1;
+                        return;
+                    }
+                    const float* gs = gring + slot * (S::GY_SLOT / 4) + o3 * kSlice + lane;
+                    float gv[d3];
+#pragma unroll
+                    for (int m = 0; m < d3; ++m) gv[m] = gs[m * kSlice];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&gy_empty[slot]);
+                    float tv[d1];
+                    [[maybe_unused]] float hG[d2];
+                    if constexpr (l2 == 0) {
+#pragma unroll
+                        for (int m = 0; m < d1; ++m) tv[m] = gv[m];
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < d1; ++m) tv[m] = 0.f;
+#pragma unroll
+                        for (int m = 0; m < d2; ++m) hG[m] = 0.f;
+                        static_for<d2>([&](auto m2c) {
+                            constexpr int m2 = EQC_CV(m2c);
+                            const float y2 = yrow[o2 + m2];
+                            static_for<d1>([&](auto m1c) {
+                                constexpr int m1 = EQC_CV(m1c);
+                                if constexpr (cg_row_nonzero<l1, l2, l3>(m1, m2)) {
+                                    float h = 0.f;
+                                    static_for<d3>([&](auto m3c) {
+                                        constexpr int m3 = EQC_CV(m3c);
+                                        constexpr double c = RealCG<l1, l2, l3>::t.v[m1][m2][m3];
+                                        if constexpr (c != 0.0) h = fmaf((float)c, gv[m3], h);
+                                    });
+                                    tv[m1] = fmaf(y2, h, tv[m1]);
+                                    hG[m2] = fmaf(xv[m1], h, hG[m2]);
+                                }
+                            });
+                        });
+                    }
+                    float dw = xv[0] * tv[0];
+#pragma unroll
+                    for (int m = 1; m < d1; ++m) dw = fmaf(xv[m], tv[m], dw);
+#pragma unroll
+                    for (int m = 0; m < d1; ++m) dxa[m] = fmaf(w, tv[m], dxa[m]);
+                    gval = dw * gscale0 * us;
+                    // this path's partials of the edge, summed over the 32 channels:
+                    // sum dw z3 (scaled; for g_u) and the harmonic gradient
+                    float gu = dw * Dv;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) gu += __shfl_xor_sync(0xffffffffu, gu, o);
+                    if constexpr (l2 > 0) {
+#pragma unroll
+                        for (int m = 0; m < d2; ++m) {
+                            float v = w * hG[m];
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                            hG[m] = v;
+                        }
+                    }
+                    if (lane == 0) {
+                        float* gp = prm.gy_part + ((size_t)k * slices + slice) * R::SD2 + ogp;
+                        gp[0] = gu;
+                        if constexpr (l2 > 0) {
+#pragma unroll
+                            for (int m = 0; m < d2; ++m) gp[1 + m] = hG[m];
+                        }
+                    }
+                }
+                // pack G (zero for edges past the range) and store every 8 edges
+                __half gh, gl;
+                split_f16(gval, gh, gl);
+                const int pr = t & 7;
+                const uint32_t bh = __half_as_ushort(gh), bl = __half_as_ushort(gl);
+                if ((pr & 1) == 0) {
+                    ghi[pr >> 1] = bh;
+                    glo[pr >> 1] = bl;
+                } else {
+                    ghi[pr >> 1] |= bh << 16;
+                    glo[pr >> 1] |= bl << 16;
+                }
+                if (pr == 7) {
+                    const uint32_t off = g_chunk_offset(grow, (kb - kt + t) >> 3);
+                    *reinterpret_cast<uint4*>(g_hi + off) = make_uint4(ghi[0], ghi[1], ghi[2], ghi[3]);
+                    *reinterpret_cast<uint4*>(g_lo + off) = make_uint4(glo[0], glo[1], glo[2], glo[3]);
+                }
+            }
+            __syncwarp();
+        }
+        // G written (generic proxy) -> visible to the tensor cores (async proxy)
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(g_full);
+            mbar_arrive(&t_empty[s]);
+        }
+    }
+    // the last sender and any empty ones after it
+    while (true) {
+        flush();
+        if (++cur >= n1) break;
+        load_x();
+    }
+}
+
+template <class K>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    radial_conv_bwd_kernel(const RadBwdParams prm, const __grid_constant__ CUtensorMap map_a_hi,
+                           const __grid_constant__ CUtensorMap map_a_lo, const __grid_constant__ CUtensorMap map_h_hi,
+                           const __grid_constant__ CUtensorMap map_h_lo, const __grid_constant__ CUtensorMap map_gy) {
+    using S = RadBwdSmem<K>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::BAR_OFF);
+    uint64_t* w3_full = bars;
+    uint64_t* h_full = bars + 1;
+    uint64_t* h_empty = bars + 3;
+    uint64_t* t_full = bars + 5;
+    uint64_t* t_empty = bars + 7;
+    uint64_t* g_full = bars + 9;
+    uint64_t* g_empty = bars + 10;
+    uint64_t* gd_full = bars + 11;
+    uint64_t* gd_empty = bars + 12;
+    uint64_t* gw_full = bars + 13;
+    uint64_t* gy_full = bars + 14;
+    uint64_t* gy_empty = bars + 14 + S::GYS;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(base + S::MISC_OFF + 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const int n0 = blockIdx.x * prm.nodes_per_cta;
+    const int n1 = min(prm.N, n0 + prm.nodes_per_cta);
+    const int slice = blockIdx.y, slices = gridDim.y;
+    const int c0 = slice * kSlice;
+    const int g0 = blockIdx.z * kBwdGroupPaths;
+    const int gp = min(kBwdGroupPaths, K::NP - g0);
+    const int gtiles = (gp + 3) / 4;
+    const int k0 = prm.ptr[n0], k1 = prm.ptr[n1];
+    const int ntiles = (k1 - k0 + kEdgeTile - 1) / kEdgeTile;
+    const int sg = blockIdx.z * slices + slice;     // this CTA's (slice, group) partial index
+    const int gexp = g_scale_exponent(prm.scal);
+
+    if (tid == 0) {
+        mbar_init(w3_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&h_full[s], 1);
+            mbar_init(&h_empty[s], 1);
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], gp);
+        }
+        mbar_init(g_full, gp);
+        mbar_init(g_empty, 1);
+        mbar_init(gd_full, 1);
+        mbar_init(gd_empty, 4);
+        mbar_init(gw_full, 1);
+        for (int q = 0; q < S::GYS; ++q) {
+            mbar_init(&gy_full[q], 1);
+            mbar_init(&gy_empty[q], gp);
+        }
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    // G rows of absent paths (gp < 8) and of a missing second tile stay zero
+    for (int i = tid; i < kBwdGroupTiles * 2 * S::G_TILE / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(base + S::G_OFF)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async();
+    if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < kBwdPathWarps) {
+        const int p = g0 + warp;
+        if (warp < gp) {
+            static_for<K::NP>([&](auto pc) {
+                if (EQC_CV(pc) == p)
+                    path_warp_bwd<K, EQC_CV(pc)>(prm, base, tmem, warp, lane, n0, n1, k0, k1, c0, slice, slices,
+                                                 gexp, abort_flag);
+            });
+        }
+    } else if (warp < kBwdMmaWarp) {
+        // reader warp of subpartition q: Gd rows k = 16 q + lane (lanes < 16) of every tile
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        for (int j = 0; j < ntiles; ++j) {
+            if (!mbar_wait(gd_full, (uint32_t)j & 1u) || __any_sync(0xffffffffu, *abort_flag)) {
+                if (lane == 0) atomicOr(prm.status, 4u);
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const int kt = k0 + j * kEdgeTile;
+            const int kk = 16 * q + lane;
+#pragma unroll
+            for (int c16 = 0; c16 < kEdgeTile; c16 += 16) {
+                float v[16];
+                tmem_ld16(tmem + lane_base + kColGD + (uint32_t)c16, v);
+                if (lane < 16) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int k = kt + c16 + i;
+                        if (k < k1) prm.gd_part[((size_t)sg * prm.E + k) * kH + kk] = v[i];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(gd_empty);
+        }
+        // the CTA's g_W3 rows: tile t, row 32 q + lane = (path g0 + 4 t + q, channel c0 + lane);
+        // a range without edges contributes zeros
+        if (ntiles == 0) {
+            for (int t = 0; t < gtiles; ++t) {
+                const int p = g0 + 4 * t + q;
+                if (p < K::NP) {
+                    float* dst = prm.gw3_part +
+                                 ((size_t)blockIdx.x * K::NP * prm.C + (size_t)p * prm.C + c0 + lane) * kH;
+                    for (int i = 0; i < kH; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+        } else if (!*abort_flag) {
+            if (mbar_wait(gw_full, 0)) {
+                tc_fence_after();
+                for (int t = 0; t < gtiles; ++t) {
+                    const int p = g0 + 4 * t + q;
+                    float* dst = prm.gw3_part + ((size_t)blockIdx.x * K::NP * prm.C + (size_t)p * prm.C + c0 + lane) * kH;
+#pragma unroll
+                    for (int c16 = 0; c16 < kH; c16 += 16) {
+                        float v[16];
+                        tmem_ld16(tmem + lane_base + kColGW + (uint32_t)(t * kH + c16), v);
+                        if (p < K::NP)
+#pragma unroll
+                            for (int i = 0; i < 16; i += 4)
+                                *reinterpret_cast<float4*>(dst + c16 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    }
+                }
+            } else if (lane == 0) {
+                atomicOr(prm.status, 4u);
+            }
+        }
+    } else if (warp == kBwdMmaWarp) {
+        if (lane == 0 && ntiles > 0) {
+            mbar_expect_tx(w3_full, gtiles * 2 * S::A_TILE);
+            for (int t = 0; t < gtiles; ++t)
+                for (int q = 0; q < 4; ++q) {
+                    const int row = (g0 + 4 * t + q) * prm.C + c0;
+                    uint8_t* dst = base + S::W3_OFF + t * 2 * S::A_TILE + q * 32 * kTileRowBytes;
+                    tma_2d(dst, &map_a_hi, 0, row, w3_full);
+                    tma_2d(dst + S::A_TILE, &map_a_lo, 0, row, w3_full);
+                }
+            auto load_h = [&](int j) {
+                const int s = j & 1;
+                uint8_t* dst = base + S::H_OFF + s * 2 * S::H_TILE;
+                mbar_expect_tx(&h_full[s], 2 * S::H_TILE);
+                tma_2d(dst, &map_h_hi, 0, k0 + j * kEdgeTile, &h_full[s]);
+                tma_2d(dst + S::H_TILE, &map_h_lo, 0, k0 + j * kEdgeTile, &h_full[s]);
+            };
+            load_h(0);
+            if (ntiles > 1) load_h(1);
+            bool ok = mbar_wait_one(w3_full, 0);
+            constexpr uint32_t id_w = idesc_f16(kRowTile, kEdgeTile);                 // W3^T . H^T
+            constexpr uint32_t id_gw = idesc_f16(kRowTile, kH, false, true);          // G . H (B MN-major)
+            constexpr uint32_t id_gd = idesc_f16(kH, kEdgeTile, true, true);          // W3 . G (both MN-major)
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int s = j & 1;
+                ok = mbar_wait_one(&h_full[s], (uint32_t)(j >> 1) & 1u) &&
+                     (j < 2 || mbar_wait_one(&t_empty[s], (uint32_t)((j >> 1) - 1) & 1u));
+                if (!ok || *abort_flag) break;
+                tc_fence_after();
+                const uint8_t* hs = base + S::H_OFF + s * 2 * S::H_TILE;
+                const uint64_t dbh = sw128_desc(smem_addr(hs)), dbl = sw128_desc(smem_addr(hs + S::H_TILE));
+                // w of this tile
+                for (int t = 0; t < gtiles; ++t) {
+                    const uint8_t* at = base + S::W3_OFF + t * 2 * S::A_TILE;
+                    const uint64_t dah = sw128_desc(smem_addr(at)), dal = sw128_desc(smem_addr(at + S::A_TILE));
+                    const uint32_t d = tmem + kColW + (uint32_t)((s * kBwdGroupTiles + t) * kEdgeTile);
+#pragma unroll
+                    for (int kk = 0; kk < kH / 16; ++kk) {
+                        const uint64_t adv = (uint64_t)(kk * 32) >> 4;
+                        umma_f16(d, dah + adv, dbh + adv, id_w, kk > 0);
+                        umma_f16(d, dah + adv, dbl + adv, id_w, 1);
+                        umma_f16(d, dal + adv, dbh + adv, id_w, 1);
+                    }
+                }
+                umma_commit(&t_full[s]);
+                // the path warps' G tile of this tile, then g_W3 += G . H and Gd = W3 . G
+                ok = mbar_wait_one(g_full, (uint32_t)j & 1u) &&
+                     (j == 0 || mbar_wait_one(gd_empty, (uint32_t)(j - 1) & 1u));
+                if (!ok || *abort_flag) break;
+                tc_fence_after();
+                for (int t = 0; t < gtiles; ++t) {
+                    const uint8_t* gt = base + S::G_OFF + t * 2 * S::G_TILE;
+                    const uint64_t dgh = sw128_desc(smem_addr(gt)), dgl = sw128_desc(smem_addr(gt + S::G_TILE));
+                    const uint32_t d = tmem + kColGW + (uint32_t)(t * kH);
+#pragma unroll
+                    for (int kk = 0; kk < kEdgeTile / 16; ++kk) {
+                        const uint64_t a_adv = (uint64_t)(kk * 32) >> 4;      // G: K-major, 16 edges = 32 B
+                        const uint64_t b_adv = (uint64_t)(kk * 2048) >> 4;    // H: MN-major, 16 edge rows
+                        umma_f16(d, dgh + a_adv, dbh + b_adv, id_gw, (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16(d, dgh + a_adv, dbl + b_adv, id_gw, 1);
+                        umma_f16(d, dgl + a_adv, dbh + b_adv, id_gw, 1);
+                    }
+                }
+                for (int t = 0; t < gtiles; ++t) {
+                    const uint8_t* at = base + S::W3_OFF + t * 2 * S::A_TILE;
+                    const uint8_t* gt = base + S::G_OFF + t * 2 * S::G_TILE;
+                    const uint64_t dah = sw128_desc(smem_addr(at)), dal = sw128_desc(smem_addr(at + S::A_TILE));
+                    const uint64_t dgh = sw128_desc(smem_addr(gt)), dgl = sw128_desc(smem_addr(gt + S::G_TILE));
+#pragma unroll
+                    for (int kk = 0; kk < kRowTile / 16; ++kk) {
+                        const uint64_t adv = (uint64_t)(kk * 2048) >> 4;      // 16 (path, channel) rows
+                        umma_f16(tmem + kColGD, dah + adv, dgh + adv, id_gd, (t > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16(tmem + kColGD, dah + adv, dgl + adv, id_gd, 1);
+                        umma_f16(tmem + kColGD, dal + adv, dgh + adv, id_gd, 1);
+                    }
+                }
+                umma_commit(g_empty);
+                umma_commit(gd_full);
+                umma_commit(&h_empty[s]);
+                if (j + 2 < ntiles) {
+                    ok = mbar_wait_one(&h_empty[s], (uint32_t)(j >> 1) & 1u);
+                    if (ok) load_h(j + 2);
+                }
+            }
+            if (ok && !*abort_flag) {
+                umma_commit(gw_full);
+            } else {
+                atomicOr(prm.status, 4u);
+                *abort_flag = 1;
+            }
+        }
+    } else if (warp == kBwdGyWarp) {
+        if (lane == 0) {
+            for (int k = k0; k < k1; ++k) {
+                const int q = k - k0, slot = q % S::GYS;
+                if (q >= S::GYS && !mbar_wait_one(&gy_empty[slot], (uint32_t)(q / S::GYS - 1) & 1u)) {
+                    atomicOr(prm.status, 4u);
+                    *abort_flag = 1;
+                    break;
+                }
+                if (*abort_flag) break;
+                int ridx = prm.receivers[prm.perm[k]];
+                if ((unsigned)ridx >= (unsigned)prm.N) {
+                    atomicOr(prm.status, 1u);
+                    ridx = 0;
+                }
+                mbar_expect_tx(&gy_full[slot], S::GY_SLOT);
+                tma_rows(base + S::GY_OFF + slot * S::GY_SLOT, &map_gy, c0, ridx, &gy_full[slot],
+                         policy_evict_last());
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace radial
+}  // namespace eqc
+
+namespace eqc {
+namespace radial {
+
+// ---------------------------------------------------------------- helpers
+
+// out[0] = max |a| over n floats (as the bits of a non-negative float);
+// out must be zeroed first.  Grid-stride, float4 loads (n % 4 == 0).
+__global__ void radial_absmax_kernel(const float* __restrict__ a, int64_t n4, unsigned* __restrict__ out) {
+    float m = 0.f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(a) + i);
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(out, __float_as_uint(m));
+}
+
+__device__ __forceinline__ float silu_grad(float z) {
+    const float s = 1.f / (1.f + expf(-z));
+    return s * (1.f + z * (1.f - s));
+}
+
+// dx[j, l1^2 + m, c] = sum over paths p with that l1, in path order, of
+// dx_pp[j, dx_off(p) + m, c].
+template <class K>
+__global__ void radial_sum_dx_kernel(const float* __restrict__ dx_pp, float* __restrict__ dx, int N, int C) {
+    using R = BwdRows<K>;
+    const int c4 = C / 4;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)N * K::D_IN * c4) return;
+    const int cq = (int)(idx % c4);
+    const int row = (int)((idx / c4) % K::D_IN);
+    const int j = (int)(idx / ((int64_t)c4 * K::D_IN));
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    static_for<K::NP>([&](auto pc) {
+        constexpr int p = EQC_CV(pc);
+        constexpr int l1 = K::PL.l1[p];
+        if (row >= l1 * l1 && row < (l1 + 1) * (l1 + 1)) {
+            const float4 v = __ldcs(reinterpret_cast<const float4*>(
+                dx_pp + ((size_t)j * R::DX_PP + R::dx_off(p) + (row - l1 * l1)) * C) + cq);
+            s.x += v.x;
+            s.y += v.y;
+            s.z += v.z;
+            s.w += v.w;
+        }
+    });
+    __stcs(reinterpret_cast<float4*>(dx + ((size_t)j * K::D_IN + row) * C) + cq, s);
+}
+
+// Per sender position k (edge e = perm[k]), one thread each, 64 per CTA, the
+// CTA walking `chunks` chunks of 64 positions:
+//   Gd = sum of the (slice, group) partials, unscaled;  g_h2 = u Gd,
+//   g_u = h2 . Gd;  back through the two SiLU layers (recomputed) to g_b;
+//   g_d = g_b . b'(d) + g_u u'(d);  gY = sum of the per-path partials;
+//   dr[e] = (dY/dr)^T gY + g_d r / d.
+// The CTA's partial sums of g_W2 = sum_e h1 (x) g_z2 and g_W1 = sum_e b (x)
+// g_z1 are accumulated in a fixed order (thread t owns row t) and written to
+// gw2_part / gw1_part [CTA].
+constexpr int kEpiThreads = 64;
+constexpr int kEpiStride = kH + 1;   // thread-private smem rows (conflict-free)
+constexpr int kEpiSmemBytes =
+    (kMaxBasis * kH + kH * kH + 3 * kEpiThreads * kEpiStride + kEpiThreads * (kMaxBasis + 1)) * 4;
+
+template <class K>
+__global__ void __launch_bounds__(kEpiThreads)
+    radial_bwd_epilogue_kernel(const float* __restrict__ r, const int* __restrict__ perm, int E,
+                               const float* __restrict__ W1, const float* __restrict__ W2, int NB, float rc,
+                               const float* __restrict__ scal, const float* __restrict__ zscale,
+                               const float* __restrict__ gy_part, int slices, const float* __restrict__ gd_part,
+                               int SG, int chunks, float* __restrict__ dr, float* __restrict__ gw1_part,
+                               float* __restrict__ gw2_part) {
+    using R = BwdRows<K>;
+    extern __shared__ __align__(16) float epi_smem[];   // kEpiSmemBytes
+    float* sW1 = epi_smem;                               // [kMaxBasis][kH]
+    float* sW2 = sW1 + kMaxBasis * kH;                   // [kH][kH]
+    float* sz1 = sW2 + kH * kH;                          // z1, then g_z1 (rows of kEpiStride)
+    float* sh1 = sz1 + kEpiThreads * kEpiStride;         // h1
+    float* sg2 = sh1 + kEpiThreads * kEpiStride;         // g_z2
+    float* sb = sg2 + kEpiThreads * kEpiStride;          // Bessel values (rows of kMaxBasis + 1)
+    const int t = threadIdx.x;
+    for (int i = t; i < NB * kH; i += kEpiThreads) sW1[i] = W1[i];
+    for (int i = t; i < kH * kH; i += kEpiThreads) sW2[i] = W2[i];
+    const int sA = inv_pow2_exponent(scal[0]);
+    const int gexp = g_scale_exponent(scal);
+    float acc2[kH];                       // g_W2 row t
+    float acc1[kMaxBasis];                // g_W1 column t
+#pragma unroll
+    for (int i = 0; i < kH; ++i) acc2[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxBasis; ++i) acc1[i] = 0.f;
+    float* z1 = sz1 + t * kEpiStride;
+    float* h1 = sh1 + t * kEpiStride;
+    float* g2 = sg2 + t * kEpiStride;
+    float* bb = sb + t * (kMaxBasis + 1);
+
+    for (int ch = 0; ch < chunks; ++ch) {
+        __syncthreads();   // weights loaded / previous chunk's rows consumed
+        const int k = (blockIdx.x * chunks + ch) * kEpiThreads + t;
+        const bool live = k < E;
+        if (live) {
+            const int e = perm[k];
+            const float rx = r[(size_t)e * 3], ry = r[(size_t)e * 3 + 1], rz = r[(size_t)e * 3 + 2];
+            const float d = sqrtf(fmaf(rx, rx, fmaf(ry, ry, rz * rz)));
+            const float inv_d = 1.f / fmaxf(d, 1e-12f);
+            const float pref = sqrtf(2.f / rc);
+            const float kd = 3.14159265358979323846f * d / rc;
+            // forward of the MLP, recomputed
+            for (int j = 0; j < kH; ++j) z1[j] = 0.f;
+            float gbd[kMaxBasis];   // b'_n(d)
+            for (int n = 0; n < NB; ++n) {
+                float sn, cn;
+                sincosf((float)(n + 1) * kd, &sn, &cn);
+                const float kn = (float)(n + 1) * 3.14159265358979323846f / rc;
+                const float b = pref * sn * inv_d;
+                bb[n] = b;
+                gbd[n] = pref * (kn * cn * inv_d - sn * inv_d * inv_d);
+                for (int j = 0; j < kH; ++j) z1[j] = fmaf(b, sW1[n * kH + j], z1[j]);
+            }
+            for (int j = 0; j < kH; ++j) h1[j] = silu(z1[j]);
+            float z2[kH];
+#pragma unroll
+            for (int j = 0; j < kH; ++j) z2[j] = 0.f;
+            for (int q = 0; q < kH; ++q) {
+                const float a = h1[q];
+#pragma unroll
+                for (int j = 0; j < kH; j += 4) {
+                    const float4 wv = *reinterpret_cast<const float4*>(&sW2[q * kH + j]);
+                    z2[j] = fmaf(a, wv.x, z2[j]);
+                    z2[j + 1] = fmaf(a, wv.y, z2[j + 1]);
+                    z2[j + 2] = fmaf(a, wv.z, z2[j + 2]);
+                    z2[j + 3] = fmaf(a, wv.w, z2[j + 3]);
+                }
+            }
+            const float x = fminf(d / rc, 1.f);
+            // u'(d) = (-168 x^5 + 336 x^6 - 168 x^7) / rc, zero from the cutoff on
+            const float x2 = x * x, x5 = x2 * x2 * x;
+            const float du = d < rc ? x5 * fmaf(x, fmaf(-168.f, x, 336.f), -168.f) / rc : 0.f;
+            // g_h2 = u W3 . dw: with G = dw 2^gexp uscale_e = u dw 2^gexp zscale_e,
+            // D = sum_pc (W3 2^sA) G = 2^(sA + gexp) zscale_e g_h2
+            const float zs = zscale[k];
+            const float fac = ldexpf(1.f, -(sA + gexp)) / zs;
+#pragma unroll
+            for (int j = 0; j < kH; ++j) {
+                float s = 0.f;
+                for (int q = 0; q < SG; ++q) s += gd_part[((size_t)q * E + k) * kH + j];
+                g2[j] = s * fac * silu_grad(z2[j]);
+            }
+            // g_u = sum_pc dw z3: the paths' partials (each sum dw D, D = z3 2^(sA + sB) = z3 / zscale)
+            float gu = 0.f;
+            for (int s = 0; s < slices; ++s) {
+                const float* gp = gy_part + ((size_t)k * slices + s) * R::SD2;
+                static_for<K::NP>([&](auto pc) { gu += gp[R::gy_off(EQC_CV(pc))]; });
+            }
+            gu *= zs;
+            // g_h1 = W2 g_z2, g_z1 = g_h1 silu'(z1)  (z1 row then holds g_z1)
+            for (int q = 0; q < kH; ++q) {
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < kH; j += 4) {
+                    const float4 wv = *reinterpret_cast<const float4*>(&sW2[q * kH + j]);
+                    s = fmaf(wv.x, g2[j], s);
+                    s = fmaf(wv.y, g2[j + 1], s);
+                    s = fmaf(wv.z, g2[j + 2], s);
+                    s = fmaf(wv.w, g2[j + 3], s);
+                }
+                z1[q] = s * silu_grad(z1[q]);
+            }
+            float gd_len = gu * du;
+            for (int n = 0; n < NB; ++n) {
+                float s = 0.f;
+                for (int j = 0; j < kH; ++j) s = fmaf(sW1[n * kH + j], z1[j], s);
+                gd_len = fmaf(s, gbd[n], gd_len);
+            }
+            // harmonic gradient: the per-path partials, in (slice, path) order
+            float ux, uy, uz, il;
+            const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
+            float d0 = 0.f, d1v = 0.f, d2v = 0.f;
+            if constexpr (K::G > 0) {
+                float gY[K::G];
+#pragma unroll
+                for (int q = 0; q < K::G; ++q) gY[q] = 0.f;
+                for (int s = 0; s < slices; ++s) {
+                    const float* gp = gy_part + ((size_t)k * slices + s) * R::SD2;
+                    static_for<K::NP>([&](auto pc) {
+                        constexpr int p = EQC_CV(pc);
+                        constexpr int l2 = K::PL.l2[p];
+                        if constexpr (l2 > 0) {
+#pragma unroll
+                            for (int m = 0; m < 2 * l2 + 1; ++m) gY[l2 * l2 - 1 + m] += gp[R::gy_off(p) + 1 + m];
+                        }
+                    });
+                }
+                sh_grad_contract<K::LSH>(ok, ux, uy, uz, il, gY, d0, d1v, d2v);
+            }
+            if (d > 1e-12f) {
+                d0 = fmaf(gd_len, rx * inv_d, d0);
+                d1v = fmaf(gd_len, ry * inv_d, d1v);
+                d2v = fmaf(gd_len, rz * inv_d, d2v);
+            }
+            dr[(size_t)e * 3] = d0;
+            dr[(size_t)e * 3 + 1] = d1v;
+            dr[(size_t)e * 3 + 2] = d2v;
+        } else {
+            for (int j = 0; j < kH; ++j) {
+                h1[j] = 0.f;
+                g2[j] = 0.f;
+                z1[j] = 0.f;
+            }
+            for (int n = 0; n < NB; ++n) bb[n] = 0.f;
+        }
+        __syncthreads();
+        // this chunk's terms of the weight gradients, edges in order
+        for (int i = 0; i < kEpiThreads; ++i) {
+            const float h = sh1[i * kEpiStride + t];
+            const float* gz2 = sg2 + i * kEpiStride;
+#pragma unroll
+            for (int j = 0; j < kH; ++j) acc2[j] = fmaf(h, gz2[j], acc2[j]);
+            const float gz1 = sz1[i * kEpiStride + t];
+            const float* bi = sb + i * (kMaxBasis + 1);
+            for (int n = 0; n < NB; ++n) acc1[n] = fmaf(bi[n], gz1, acc1[n]);
+        }
+    }
+    float* o2 = gw2_part + ((size_t)blockIdx.x * kH + t) * kH;
+#pragma unroll
+    for (int j = 0; j < kH; ++j) o2[j] = acc2[j];
+    float* o1 = gw1_part + (size_t)blockIdx.x * kMaxBasis * kH;
+    for (int n = 0; n < NB; ++n) o1[n * kH + t] = acc1[n];
+}
+
+// out[i] = sum_{b < nb} part[b * stride + i], in order of b (i < n).
+__global__ void radial_sum_parts_kernel(const float* __restrict__ part, int nb, int64_t stride, int64_t n,
+                                        float* __restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float s = 0.f;
+    for (int b = 0; b < nb; ++b) s += part[(size_t)b * stride + i];
+    out[i] = s;
+}
+
+// g_W3[k][pc] = 2^(sA - gexp) * sum over ranges of gw3_part[range][pc][k].
+__global__ void radial_sum_gw3_kernel(const float* __restrict__ part, int nranges, int PC,
+                                      const float* __restrict__ scal, float* __restrict__ gw3) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // over pc * 64 + k
+    if (i >= (int64_t)PC * kH) return;
+    const int pc = (int)(i / kH), k = (int)(i % kH);
+    float s = 0.f;
+    for (int b = 0; b < nranges; ++b) s += part[((size_t)b * PC + pc) * kH + k];
+    gw3[(size_t)k * PC + pc] = s * ldexpf(1.f, inv_pow2_exponent(scal[0]) - g_scale_exponent(scal));
+}
+
+}  // namespace radial
+}  // namespace eqc

@@ -199,6 +199,28 @@ constexpr PathList make_paths(int LIN, int LSH, int LOUT, int MODE = 0) {
     return P;
 }
 
+// Paths of the symmetric product of one natural-parity feature with itself
+// (correlation order 2): unordered pairs l1 <= l2 <= LA, outputs L <= LOUT,
+// triangle rule, l1 + l2 + L even (the odd couplings of equal inputs vanish
+// and (l2, l1, L) equals (l1, l2, L) on the symmetric product), ordered by
+// (l1, l2, L); o3 = L^2 (outputs summed by irrep).
+constexpr PathList make_sym_paths(int LA, int LOUT) {
+    PathList P{};
+    P.n = 0;
+    for (int a = 0; a <= LA; ++a)
+        for (int b = a; b <= LA; ++b)
+            for (int c = 0; c <= LOUT; ++c) {
+                if (c < iabs(a - b) || c > a + b || ((a + b + c) & 1)) continue;
+                P.l1[P.n] = a;
+                P.l2[P.n] = b;
+                P.l3[P.n] = c;
+                P.o3[P.n] = c * c;
+                ++P.n;
+            }
+    P.dout = (LOUT + 1) * (LOUT + 1);
+    return P;
+}
+
 // Offsets of each path's per-edge coupling matrix A_p[m3][m1] (paths with
 // l2 > 0 only), each padded to a multiple of 4 floats.
 struct AOffsets {

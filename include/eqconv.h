@@ -334,6 +334,44 @@ EQCONV_API int eqconv_node_product_backward(eqconv_plan_t plan, int N, const flo
                                             float* dw, void* workspace, size_t workspace_bytes,
                                             eqconv_stream_t stream);
 
+/* ---- Symmetric contraction, correlation order 2 ---------------------------
+ * e3j (arXiv 2609.35099), abstract and Table 3: MACE(a)'s product basis has
+ * correlation order 2; FlashCart (arXiv 2610.06409) §5 / App. B: the
+ * correlation ladder of channel-diagonal products of an atom's own
+ * features, weighted per path, channel and element.  For A [N][(L_A+1)^2][C]
+ * (irreps_A a natural-parity prefix) and species [N] (int32, 0..S-1):
+ *   B[i, L M, c] = W1[z_i, L, c] A[i, L M, c]                          (L <= min(L_A, L_out))
+ *                + sum_q W2[z_i, q, c] sum_{m1,m2} C_q[m1,m2,M] A[i,l1 m1,c] A[i,l2 m2,c]
+ * with q = (l1, l2, L) over l1 <= l2 <= L_A, L <= L_out, the triangle rule
+ * and l1 + l2 + L even, ordered by (l1, l2, L) (eqconv_plan_info gives them:
+ * P = their count, D_in = (L_A+1)^2, D_out = (L_out+1)^2).
+ * W1 [S][min(L_A, L_out)+1][C], W2 [S][P][C], B [N][D_out][C], fp32.
+ * L_A, L_out <= 3; 1 <= S <= 16; C % 4 == 0.  A symmetric-contraction plan
+ * is not a convolution plan.  Out-of-range species set the status word (bit
+ * 1); those nodes get B = 0. */
+EQCONV_API int eqconv_symmetric_contraction_plan_create(eqconv_plan_t* out, const char* irreps_A,
+                                                        const char* irreps_out, int C, int n_species);
+
+/* B = the contraction above; one launch on `stream`.  Pointers 16-byte aligned. */
+EQCONV_API int eqconv_symmetric_contraction(eqconv_plan_t plan, int N, const float* A, const int32_t* species,
+                                            const float* W1, const float* W2, float* B, eqconv_stream_t stream);
+
+/* Device workspace bytes eqconv_symmetric_contraction_backward needs (the
+ * per-warp weight-gradient partials). */
+EQCONV_API size_t eqconv_symmetric_contraction_workspace_bytes(eqconv_plan_t plan, int N);
+
+/* Backward given gB [N][D_out][C]:
+ *   dA = W1 gB + sum_q W2 (C_q A_l2 gB on block l1 + C_q A_l1 gB on block l2)
+ *   dW1[s, L, c] = sum over nodes of species s of A_L . gB_L
+ *   dW2[s, q, c] = sum over nodes of species s of C_q A A gB
+ * Deterministic: each warp sums its fixed node set per species in shared
+ * memory, a second launch adds the warps' partials in order.  All outputs
+ * overwritten. */
+EQCONV_API int eqconv_symmetric_contraction_backward(eqconv_plan_t plan, int N, const float* A, const int32_t* species,
+                                                     const float* W1, const float* W2, const float* gB, float* dA,
+                                                     float* dW1, float* dW2, void* workspace, size_t workspace_bytes,
+                                                     eqconv_stream_t stream);
+
 /* ---- Radial weights from edge lengths ------------------------------------
  * FlashCart (arXiv 2610.06409) App. B: a radial envelope makes every edge's
  * contribution vanish smoothly at the cutoff; App. E: the weights vanish with
@@ -383,6 +421,30 @@ EQCONV_API size_t eqconv_forward_radial_workspace_bytes(eqconv_plan_t plan, int 
 EQCONV_API int eqconv_forward_radial(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r,
                                      const float* W1, const float* W2, const float* W3, int n_basis, float r_cut,
                                      float* y, void* workspace, size_t workspace_bytes, eqconv_stream_t stream);
+
+/* Device workspace bytes eqconv_backward_radial needs for (N, E); 0 when
+ * the plan has no fused radial path. */
+EQCONV_API size_t eqconv_backward_radial_workspace_bytes(eqconv_plan_t plan, int N, int E);
+
+/* Backward of eqconv_forward_radial given gy (the plan's output layout):
+ *   dx  [N][D_in][C]   as eqconv_backward's, with w = w(|r|)
+ *   dr  [E][3]         (dY/dr)^T gY + (d/dd <dw, w(d)>) r / |r|: both routes
+ *                      of the edge vector (FlashCart §2: forces are the
+ *                      energy's gradient in the positions)
+ *   gW1 [n_basis][64], gW2 [64][64], gW3 [64][P*C]: gradients of <gy, y>
+ *                      with respect to the MLP weights
+ * w and dw never exist in memory: w is recomputed on the tensor cores, the
+ * sender-ordered pass (deterministic) keeps dw on the chip and feeds it to
+ * two tensor-core contractions (sum over edges of (u h2) x dw for gW3; W3 .
+ * dw per edge for the MLP's backward); a per-edge epilogue finishes the MLP
+ * backward and dr; the weight gradients are summed in a fixed order.
+ * Same plans and arguments as eqconv_forward_radial; outputs overwritten;
+ * bitwise reproducible run to run.  The workspace
+ * (eqconv_backward_radial_workspace_bytes) is caller-owned device memory. */
+EQCONV_API int eqconv_backward_radial(eqconv_plan_t plan, const eqconv_graph_t* g, const float* x, const float* r,
+                                      const float* W1, const float* W2, const float* W3, int n_basis, float r_cut,
+                                      const float* gy, float* dx, float* dr, float* gW1, float* gW2, float* gW3,
+                                      void* workspace, size_t workspace_bytes, eqconv_stream_t stream);
 
 /* The spherical harmonics the kernels use, Y [E][(L_sh+1)^2] (a test hook
  * for the in-kernel harmonics; not on the hot path). */

@@ -159,3 +159,88 @@ def test_forward_radial_no_edges_and_unsupported():
     assert B.eqconv_forward_radial_workspace_bytes(odd.plan, 10, 10) > 0
     other = EqConv("0e+1o+2e", 1, "0e+1o+2e", 32)
     assert B.eqconv_forward_radial_workspace_bytes(other.plan, 10, 10) == 0
+
+
+# ----------------------------------------------- fused backward (radial on chip)
+
+def _fused_backward(conv, N, s, rcv, r, x, params, nb, rc, gy):
+    g = conv.graph(to_dev(s), to_dev(rcv), N)
+    E = len(s)
+    ws_n = B.eqconv_backward_radial_workspace_bytes(conv.plan, N, E)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device="cuda")
+    nan = float("nan")
+    dx = torch.full((N, conv.D_in, conv.C), nan, device="cuda")
+    dr = torch.full((max(E, 1), 3), nan, device="cuda")
+    gW = [torch.full(tuple(p.shape), nan, device="cuda") for p in params]
+    W1, W2, W3 = (to_dev(p) for p in params)
+    B.eqconv_backward_radial(conv.plan, g.c, to_dev(x), to_dev(r), W1, W2, W3, nb, rc, to_dev(gy), dx, dr,
+                             gW[0], gW[1], gW[2], ws, ws_n)
+    torch.cuda.synchronize()
+    assert B.eqconv_get_device_error(conv.plan) == B.EQCONV_OK
+    return dx.cpu().numpy(), dr[:E].cpu().numpy(), [t.cpu().numpy() for t in gW]
+
+
+def _oracle_backward(prob, N, s, rcv, r, x, params, rc, gy):
+    """dx, dr (both routes of r) and the MLP weight gradients: the oracle's
+    C-loop backward with w from the radial MLP, then the MLP's VJP."""
+    from oracle import conv as oconv
+    d = np.linalg.norm(r.astype(np.float64), axis=1)
+    w = orad.radial_weights(d, rc, params, prob.P, prob.C).astype(np.float32)
+    _, dx, dw, dr_ang = oconv.full(prob, N, s, rcv, r, x, w, gy)
+    g_d, g_W = orad.radial_weights_vjp(d, rc, params, dw)
+    safe = np.where(d > 0, d, 1.0)
+    dr = dr_ang + (g_d / safe)[:, None] * r.astype(np.float64) * (d > 0)[:, None]
+    return dx, dr, g_W
+
+
+def test_backward_radial_tiny_box_against_bruteforce():
+    from oracle import conv as oconv
+    W = wl.WORKLOADS["tiny"]
+    s, rcv, r = wl.make_graph(W)
+    conv = EqConv(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    prob = oconv.Problem(W.irreps_in, W.L_sh, W.irreps_out, W.C)
+    x = wl.features(W.N, prob.D_in, W.C, wl.SEED_X)
+    gy = wl.features(W.N, prob.D_out, W.C, wl.SEED_GY)
+    params = wl.radial_mlp_params(prob.P, W.C, 64, 8, seed=21)
+    dx, dr, gW = _fused_backward(conv, W.N, s, rcv, r, x, params, 8, 3.5, gy)
+    _, dxr, drr, gWr = orad.conv_with_radial(prob, W.N, s, rcv, r, x, 3.5, params, gy=gy)
+    assert_close("dx (fused radial, tiny box)", dx, dxr)
+    assert_close("dr (fused radial, tiny box)", dr, drr)
+    for i in range(3):
+        assert_close(f"g_W{i + 1} (fused radial, tiny box)", gW[i], gWr[i])
+
+
+@pytest.mark.parametrize("L,C,N,per_path", [(1, 32, 300, False), (2, 64, 700, False), (2, 128, 517, True),
+                                            (3, 64, 400, False), (3, 32, 129, True)])
+def test_backward_radial_matches_oracle(L, C, N, per_path):
+    from oracle import conv as oconv
+    ins = wl.natural_irreps(L)
+    conv = EqConv(ins, L, ins, C, per_path=per_path)
+    prob = oconv.Problem(ins, L, ins, C, per_path=per_path)
+    s, rcv, r = _poisson_case(N, 12.0, seed=N + C + 5)
+    x = wl.features(N, prob.D_in, C, wl.SEED_X)
+    gy = wl.features(N, prob.D_out, C, wl.SEED_GY)
+    rc, nb = 5.0, 8
+    params = wl.radial_mlp_params(prob.P, C, 64, nb, seed=41 + L)
+    dx, dr, gW = _fused_backward(conv, N, s, rcv, r, x, params, nb, rc, gy)
+    dxr, drr, gWr = _oracle_backward(prob, N, s, rcv, r, x, params, rc, gy)
+    tag = f"L={L} C={C} N={N} per_path={per_path}"
+    assert_close(f"dx ({tag})", dx, dxr)
+    assert_close(f"dr ({tag})", dr, drr)
+    for i in range(3):
+        assert_close(f"g_W{i + 1} ({tag})", gW[i], gWr[i])
+
+
+def test_backward_radial_is_bitwise_reproducible():
+    ins = "0e+1o+2e"
+    conv = EqConv(ins, 2, ins, 64)
+    N = 600
+    s, rcv, r = _poisson_case(N, 20.0, seed=9)
+    x = wl.features(N, 9, 64, wl.SEED_X)
+    gy = wl.features(N, 9, 64, wl.SEED_GY)
+    params = wl.radial_mlp_params(conv.P, 64, 64, 8, seed=3)
+    a = _fused_backward(conv, N, s, rcv, r, x, params, 8, 5.0, gy)
+    b = _fused_backward(conv, N, s, rcv, r, x, params, 8, 5.0, gy)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    for i in range(3):
+        assert np.array_equal(a[2][i], b[2][i])
