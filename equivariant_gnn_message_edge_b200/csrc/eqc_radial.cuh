@@ -46,12 +46,16 @@ constexpr int kTileRowBytes = kH * 2;   // one fp16 row of 64 values: 128 B, one
 
 __device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
 
-// 2^s with s such that m * 2^s lies in [2^13, 2^14) (s = 0 for m = 0).
+// s such that m * 2^s lies in [2^13, 2^14), capped at 60; 60 for m = 0.  A
+// row of zeros (or of values below 2^-46) gets the largest scale, so that
+// the factor 2^-s, which the backward's dw tile carries for that row, stays
+// within its bound (2^-s <= 2^-13 max|h2|) and 2^-s itself stays a normal
+// float.
 __device__ __forceinline__ int pow2_exponent_for(float m) {
-    if (!(m > 0.f)) return 0;
+    if (!(m > 0.f)) return 60;
     int e;
     frexpf(m, &e);   // m = f * 2^e, f in [0.5, 1)
-    return 14 - e;
+    return 14 - e < 60 ? 14 - e : 60;
 }
 
 __device__ __forceinline__ void split_f16(float v, __half& hi, __half& lo) {
