@@ -808,6 +808,7 @@ int eqconv_forward_radial(eqconv_plan_t plan, const eqconv_graph_t* g, const flo
     a.recv_ptr = g->recv_ptr;
     a.recv_perm = g->recv_perm;
     a.senders = g->senders;
+    a.receivers = g->receivers;
     a.W1 = W1;
     a.W2 = W2;
     a.W3 = W3;
@@ -859,6 +860,7 @@ int eqconv_backward_radial(eqconv_plan_t plan, const eqconv_graph_t* g, const fl
     a.gy = gy;
     a.send_ptr = g->send_ptr;
     a.send_perm = g->send_perm;
+    a.senders = g->senders;
     a.receivers = g->receivers;
     a.W1 = W1;
     a.W2 = W2;

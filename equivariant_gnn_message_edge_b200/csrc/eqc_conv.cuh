@@ -864,6 +864,32 @@ __global__ void __launch_bounds__(FwdShape<K>::WARPS * 32)
 
 // --------------------------------------------------------------- backward
 
+// Sums NV values (a power of two <= 32) over the warp's 32 lanes at once:
+// each halving step trades half of the values with the partner lane, so the
+// cost is NV - 1 + 5 - log2(NV) shuffles instead of 5 NV.  Lane L returns the
+// sum of value L >> (5 - log2 NV).  The order of the additions is fixed
+// (bitwise reproducible).
+template <int NV>
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[NV], int lane) {
+    static_assert(NV >= 1 && NV <= 32 && (NV & (NV - 1)) == 0, "NV: a power of two <= 32");
+    constexpr int LOG = NV >= 32 ? 5 : NV >= 16 ? 4 : NV >= 8 ? 3 : NV >= 4 ? 2 : NV >= 2 ? 1 : 0;
+#pragma unroll
+    for (int st = 0; st < LOG; ++st) {
+        const int n = NV >> (st + 1), o = 16 >> st;
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+            const float send = upper ? v[i] : v[i + n];
+            const float keep = upper ? v[i + n] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    float r = v[0];
+#pragma unroll
+    for (int st = LOG; st < 5; ++st) r += __shfl_xor_sync(0xffffffffu, r, 16 >> st);
+    return r;
+}
+
 // Butterfly sum across the warp (fixed order: bitwise reproducible).
 template <int G>
 __device__ __forceinline__ void warp_sum(float (&v)[G]) {
@@ -872,6 +898,11 @@ __device__ __forceinline__ void warp_sum(float (&v)[G]) {
 #pragma unroll
         for (int k = 0; k < G; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], o);
 }
+
+// The smallest power of two >= n (n <= 32), for warp_transpose_sum.
+constexpr int pow2_at_least(int n) { return n <= 1 ? 1 : n <= 2 ? 2 : n <= 4 ? 4 : n <= 8 ? 8 : n <= 16 ? 16 : 32; }
+// log2 of the lanes that share one result of warp_transpose_sum<NV>.
+constexpr int transpose_sum_shift(int nv) { return nv >= 32 ? 0 : nv >= 16 ? 1 : nv >= 8 ? 2 : nv >= 4 ? 3 : nv >= 2 ? 4 : 5; }
 
 // DET: node = sender j, resident x_j, dx_j summed in registers in send_perm order.
 // !DET: node = receiver i, resident gy_i, dx scattered with atomic adds.
@@ -1012,7 +1043,22 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
                                        RegRows<V, K::D_OUT>{gres}, Wr, dxacc, sink,
                                        gyl, store_dw);
                 }
-                if constexpr (K::G > 0) {
+                if constexpr (K::G > 0 && V == 1) {
+                    // value q of the warp's sum lands on lanes q << SH .. (q + 1) << SH
+                    constexpr int NV = pow2_at_least(K::G), SH = transpose_sum_shift(NV);
+                    float tv[NV];
+#pragma unroll
+                    for (int q = 0; q < NV; ++q) tv[q] = q < K::G ? gyl[q] : 0.f;
+                    const float sum = warp_transpose_sum<NV>(tv, lane);
+                    const int q = lane >> SH;
+                    if ((lane & ((1 << SH) - 1)) == 0 && q < K::G) {
+                        if constexpr (FUSED)
+                            gYs[(t - b0) * K::GS + q] = sum;
+                        else
+                            prm.gy_part[((size_t)e * prm.T + tile) * K::G + q] = sum;
+                    }
+                } else if constexpr (K::G > 0) {
+                    // wider channel tiles are held by registers: the plain butterfly needs fewer
                     warp_sum<K::G>(gyl);
                     if (lane == 0) {
                         if constexpr (FUSED) {

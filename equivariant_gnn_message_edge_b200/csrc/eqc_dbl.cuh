@@ -27,9 +27,10 @@
 //     each edge's Y and rho, not its coupling matrices;
 //   * r epilogue (one thread per edge): sums the tiles in order and applies
 //     the gradient and the Hessian-vector product of the harmonics.
-// Rows are read with plain vector loads (no staging ring): the double
-// backward is a training-time op with twice the streamed bytes of the
-// backward (w and b).
+// Each warp stages its edges' rows through a ring of shared-memory stages
+// filled by tensor-map copies (as the first-order kernels do), K::STAGES
+// edges ahead: the receiver pass copies w_e, b_e, x_s and a_s per edge, the
+// sender pass w_e, b_e and gy_i.
 #pragma once
 
 #include "eqc_conv.cuh"
@@ -56,20 +57,9 @@ struct DblParams {
     unsigned* status;
 };
 
-#ifndef EQC_DBL_PREFETCH
-#define EQC_DBL_PREFETCH 1   // load the next edge's rows while the current edge is computed
-#endif
-
 template <class K>
 struct DblShape {
-    // prefetching doubles the row registers: it paid at lmax 2 (17.3 -> 16.7 ms)
-    // and cost at lmax 3 (41.6 -> 46.8 ms), where the per-edge code is larger
-    static constexpr bool PF = EQC_DBL_PREFETCH && K::NA_PAD <= 128;
     static constexpr int CH = K::NA_PAD > 128 ? 4 : 8;        // edges per coupling batch
-    // receiver pass: A(Y) and A(rho); sender pass: Y and rho
-    static constexpr int WARP_FLOATS = 2 * CH * (K::NA_PAD > K::D_SH ? K::NA_PAD : K::D_SH);
-    static constexpr int WARPS = 4;
-    static constexpr int SMEM = WARPS * WARP_FLOATS * 4;
 };
 
 template <int V>
@@ -100,38 +90,6 @@ __device__ __forceinline__ void load_rows(float (&d)[R][V], const float* base, i
 #pragma unroll
             for (int v = 0; v < V; ++v) d[k][v] = 0.f;
         }
-    }
-}
-
-// Lane t of the warp: harmonics, their derivative along q, and the coupling
-// matrices A(Y), A(rho) of edge e into shared memory.
-template <class K>
-__device__ __forceinline__ void dbl_couplings(const float* r, const float* q, int e, float* AY, float* AR) {
-    const float rx = r[3 * (size_t)e], ry = r[3 * (size_t)e + 1], rz = r[3 * (size_t)e + 2];
-    float ux, uy, uz, il;
-    const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
-    float Y[K::D_SH], rho[K::D_SH];
-    sh_eval<K::LSH>(ok, ux, uy, uz, Y);
-    sh_jvp<K::LSH>(rx, ry, rz, q[3 * (size_t)e], q[3 * (size_t)e + 1], q[3 * (size_t)e + 2], rho);
-    compute_A<K>(Y, AY);
-    compute_A<K>(rho, AR);
-}
-
-// Lane t of the warp: the harmonics Y and rho = (dY/dr) q of edge e into
-// shared memory (rows of K::YS floats: Y first, then rho), for the sender
-// pass, which needs no coupling matrices.
-template <class K>
-__device__ __forceinline__ void dbl_harmonics(const float* r, const float* q, int e, float* Yrow) {
-    const float rx = r[3 * (size_t)e], ry = r[3 * (size_t)e + 1], rz = r[3 * (size_t)e + 2];
-    float ux, uy, uz, il;
-    const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
-    float Y[K::D_SH], rho[K::D_SH];
-    sh_eval<K::LSH>(ok, ux, uy, uz, Y);
-    sh_jvp<K::LSH>(rx, ry, rz, q[3 * (size_t)e], q[3 * (size_t)e + 1], q[3 * (size_t)e + 2], rho);
-#pragma unroll
-    for (int k = 0; k < K::D_SH; ++k) {
-        Yrow[k] = Y[k];
-        Yrow[K::D_SH + k] = rho[k];
     }
 }
 
@@ -256,73 +214,141 @@ __device__ __forceinline__ void dbl_send_edge(const float* Yrow, const float (&x
     });
 }
 
-// Rows of one edge for the receiver pass (weights, weight cotangent, sender
-// features and their cotangent) and for the sender pass (weights, weight
-// cotangent, receiver output gradient), this lane's channels.
-template <class K>
-struct RecvRows {
-    float w[K::NP][K::VEC], b[K::NP][K::VEC], x[K::D_IN][K::VEC], a[K::D_IN][K::VEC];
-};
-template <class K>
-struct SendRows {
-    float w[K::NP][K::VEC], b[K::NP][K::VEC], g[K::D_OUT][K::VEC];
+// Per-warp shared memory of the two passes (floats, regions 128-byte
+// aligned): [stages: S x ROWS x TILE_C] [mbarriers] [per-batch rows].
+// Receiver pass: rows w (NP), b (NP), x (D_IN), a (D_IN) per stage and the
+// batch's coupling matrices A(Y), A(rho); sender pass: rows w, b, gy (D_OUT)
+// and the batch's harmonics Y, rho.
+template <class K, bool RECV>
+struct DblRing {
+    static constexpr int S = K::STAGES;
+    static constexpr int CH = DblShape<K>::CH;
+    static constexpr int up32(int f) { return (f + 31) & ~31; }
+    static constexpr int ROWS = RECV ? 2 * K::NP + 2 * K::D_IN : 2 * K::NP + K::D_OUT;
+    static constexpr int SF = ROWS * K::TILE_C;                       // floats per stage
+    static constexpr uint32_t STAGE_BYTES = SF * 4;
+    static constexpr int ST_F = S * SF;
+    static constexpr int BAR_F = up32(4 * S);
+    static constexpr int ROW_F = up32(RECV ? 2 * CH * K::NA_PAD : CH * 2 * K::D_SH);
+    static constexpr int TOTAL_F = ST_F + BAR_F + ROW_F;
+    static constexpr int WARPS = best_warps(TOTAL_F * 4);
+    static constexpr int SMEM = WARPS * TOTAL_F * 4;
 };
 
-// Receiver pass: g_gy.
+// Fill stage `st` for edge e and its other end o: the edge's w and b rows,
+// then the node rows of the two node maps (a null second map: one node map).
+template <class K, bool RECV>
+__device__ __forceinline__ void dbl_fill(float* st, uint64_t* bar, const CUtensorMap* tw, const CUtensorMap* tb,
+                                         const CUtensorMap* tn0, const CUtensorMap* tn1, int e, int o, int c0,
+                                         uint64_t pol_e, uint64_t pol_n, int lane) {
+    if (lane == 0) {
+        constexpr int DN = RECV ? K::D_IN : K::D_OUT;
+        fence_proxy_async();
+        mbar_expect_tx(bar, DblRing<K, RECV>::STAGE_BYTES + EQC_TEST_FILL_DEFICIT);
+        tma_rows(st, tw, c0, e, bar, pol_e);
+        tma_rows(st + K::NP * K::TILE_C, tb, c0, e, bar, pol_e);
+        tma_rows(st + 2 * K::NP * K::TILE_C, tn0, c0, o, bar, pol_n);
+        if constexpr (RECV) tma_rows(st + (2 * K::NP + DN) * K::TILE_C, tn1, c0, o, bar, pol_n);
+    }
+}
+
+// Receiver pass: g_gy.  One warp per receiver and channel tile.
 template <class K>
-__global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_recv_kernel(const DblParams prm) {
-    constexpr int V = K::VEC, CH = DblShape<K>::CH, W = DblShape<K>::WARPS;
+__global__ void __launch_bounds__(DblRing<K, true>::WARPS * 32)
+    eqconv_dbl_recv_kernel(const DblParams prm, const __grid_constant__ CUtensorMap tmap_w,
+                           const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_x,
+                           const __grid_constant__ CUtensorMap tmap_a) {
+    using L = DblRing<K, true>;
+    constexpr int V = K::VEC, S = L::S, CH = L::CH, W = L::WARPS, SF = L::SF;
     extern __shared__ __align__(128) float4 smem4[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int node = blockIdx.x * W + warp;
     if (node >= prm.N) return;
-    float* AY = reinterpret_cast<float*>(smem4) + warp * DblShape<K>::WARP_FLOATS;
+    float* stages = reinterpret_cast<float*>(smem4) + warp * L::TOTAL_F;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + L::ST_F);
+    float* AY = stages + L::ST_F + L::BAR_F;
     float* AR = AY + CH * K::NA_PAD;
     const int C = prm.C;
     const int c0 = blockIdx.y * K::TILE_C, cl = lane * V;
     const bool on = c0 + cl < C;
+    const uint64_t pol_e = policy_evict_first(), pol_n = policy_evict_last();
+    if (lane == 0) {
+        for (int q = 0; q < S; ++q) mbar_init(&bars[2 * q], 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
     float acc[K::D_OUT][V];
 #pragma unroll
     for (int d = 0; d < K::D_OUT; ++d)
 #pragma unroll
         for (int v = 0; v < V; ++v) acc[d][v] = 0.f;
-    const int kb = prm.ptr[node], ke = prm.ptr[node + 1];
-    for (int k0 = kb; k0 < ke; k0 += CH) {
-        const int nb = min(CH, ke - k0);
-        int my_e = 0, my_s = -1;
-        if (lane < nb) {
-            my_e = prm.perm[k0 + lane];
-            if ((unsigned)my_e < (unsigned)prm.E) my_s = prm.other[my_e];
-            if ((unsigned)my_s >= (unsigned)prm.N) {
-                atomicOr(prm.status, 1u);
-                my_s = -1;
-            } else {
-                dbl_couplings<K>(prm.r, prm.q, my_e, AY + lane * K::NA_PAD, AR + lane * K::NA_PAD);
-            }
+    uint32_t g = 0;   // edges staged so far (stage g % S, phase (g / S) & 1)
+    bool ok_all = true;
+    uint32_t fill_from = 0, fill_to = 0;
+    int k = prm.ptr[node];
+    const int ke = prm.ptr[node + 1];
+    while (k < ke && ok_all) {
+        int my_e, my_s;
+        float rx, ry, rz;
+        const int n = gather_window(prm.perm, prm.other, prm.r, prm.N, 0, prm.N, k, ke, prm.status, lane, my_e,
+                                    my_s, rx, ry, rz);
+        if (n == 0) continue;
+        const int pre = min(S, n);
+        for (int t = 0; t < pre; ++t) {
+            const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_s, t);
+            const uint32_t gi = g + t;
+            dbl_fill<K, true>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_b, &tmap_x, &tmap_a, e,
+                              o, c0, pol_e, pol_n, lane);
         }
-        __syncwarp();
-        RecvRows<K> cur, nxt;
-        const auto load = [&](RecvRows<K>& rw, int t) {
-            const int e = __shfl_sync(0xffffffffu, my_e, t);
-            const int s = __shfl_sync(0xffffffffu, my_s, t);
-            const bool ld = on && s >= 0;
-            load_rows<V>(rw.w, prm.w + (size_t)e * K::NP * C + c0 + cl, C, ld);
-            load_rows<V>(rw.b, prm.b + (size_t)e * K::NP * C + c0 + cl, C, ld);
-            load_rows<V>(rw.x, prm.x + (size_t)max(s, 0) * K::D_IN * C + c0 + cl, C, ld);
-            load_rows<V>(rw.a, prm.a + (size_t)max(s, 0) * K::D_IN * C + c0 + cl, C, ld);
-        };
-        if (DblShape<K>::PF) load(cur, 0);
-        for (int t = 0; t < nb; ++t) {
-            if (DblShape<K>::PF) {
-                if (t + 1 < nb) load(nxt, t + 1);
-            } else {
-                load(cur, t);
+        for (int b0 = 0; b0 < n && ok_all; b0 += CH) {
+            const int nb = min(CH, n - b0);
+            if (lane >= b0 && lane < b0 + nb) {
+                const float* qe = prm.q + 3 * (size_t)my_e;
+                float ux, uy, uz, il;
+                const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
+                float Y[K::D_SH], rho[K::D_SH];
+                sh_eval<K::LSH>(ok, ux, uy, uz, Y);
+                sh_jvp<K::LSH>(rx, ry, rz, qe[0], qe[1], qe[2], rho);
+                compute_A<K>(Y, AY + (lane - b0) * K::NA_PAD);
+                compute_A<K>(rho, AR + (lane - b0) * K::NA_PAD);
             }
-            if (__shfl_sync(0xffffffffu, my_s, t) >= 0)
-                dbl_recv_edge<K>(AY + t * K::NA_PAD, AR + t * K::NA_PAD, cur.x, cur.a, cur.w, cur.b, acc);
-            if (DblShape<K>::PF) cur = nxt;
+            __syncwarp();
+            for (int t = b0; t < b0 + nb; ++t) {
+                const uint32_t gi = g + t;
+                float* st = stages + (gi % S) * SF;
+                if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
+                    if (lane == 0) atomicOr(prm.status, 4u);
+                    ok_all = false;
+                    fill_from = gi;
+                    fill_to = g + (uint32_t)min(n, t + S);
+                    break;
+                }
+                float wv[K::NP][V], bv[K::NP][V], xv[K::D_IN][V], av[K::D_IN][V];
+#pragma unroll
+                for (int p = 0; p < K::NP; ++p) {
+                    lds_vec<V>(wv[p], st + p * K::TILE_C + cl);
+                    lds_vec<V>(bv[p], st + (K::NP + p) * K::TILE_C + cl);
+                }
+#pragma unroll
+                for (int d = 0; d < K::D_IN; ++d) {
+                    lds_vec<V>(xv[d], st + (2 * K::NP + d) * K::TILE_C + cl);
+                    lds_vec<V>(av[d], st + (2 * K::NP + K::D_IN + d) * K::TILE_C + cl);
+                }
+                dbl_recv_edge<K>(AY + (t - b0) * K::NA_PAD, AR + (t - b0) * K::NA_PAD, xv, av, wv, bv, acc);
+                __syncwarp();
+                if (t + S < n) {
+                    const int e = __shfl_sync(0xffffffffu, my_e, t + S), o = __shfl_sync(0xffffffffu, my_s, t + S);
+                    dbl_fill<K, true>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_b, &tmap_x, &tmap_a, e, o, c0, pol_e,
+                                      pol_n, lane);
+                }
+            }
+            __syncwarp();
         }
-        __syncwarp();
+        g += n;
+    }
+    if (!ok_all) {
+        drain_fills<S>(bars, fill_from, fill_to);
+        return;
     }
     if (on) {
         float* gi = prm.g_gy + (size_t)node * K::D_OUT * C + c0 + cl;
@@ -331,20 +357,32 @@ __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_recv_kerne
     }
 }
 
-// Sender pass: g_x, g_w and the per-tile partials of gYv, gY1.
+// Sender pass: g_x, g_w and the per-tile partials of gYv, gY1.  One warp per
+// sender and channel tile; x_j and a_j stay in registers.
 template <class K>
-__global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_send_kernel(const DblParams prm) {
-    constexpr int V = K::VEC, CH = DblShape<K>::CH, W = DblShape<K>::WARPS;
+__global__ void __launch_bounds__(DblRing<K, false>::WARPS * 32)
+    eqconv_dbl_send_kernel(const DblParams prm, const __grid_constant__ CUtensorMap tmap_w,
+                           const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_g) {
+    using L = DblRing<K, false>;
+    constexpr int V = K::VEC, S = L::S, CH = L::CH, W = L::WARPS, SF = L::SF;
     constexpr int G = K::G > 0 ? K::G : 1;
     extern __shared__ __align__(128) float4 smem4[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int node = blockIdx.x * W + warp;
     if (node >= prm.N) return;
-    float* AY = reinterpret_cast<float*>(smem4) + warp * DblShape<K>::WARP_FLOATS;   // Y, rho rows
+    float* stages = reinterpret_cast<float*>(smem4) + warp * L::TOTAL_F;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + L::ST_F);
+    float* Ys = stages + L::ST_F + L::BAR_F;   // rows of 2 D_SH: Y then rho
     const int C = prm.C;
     const int tile = blockIdx.y;
     const int c0 = tile * K::TILE_C, cl = lane * V;
     const bool on = c0 + cl < C;
+    const uint64_t pol_e = policy_evict_first(), pol_n = policy_evict_last();
+    if (lane == 0) {
+        for (int q = 0; q < S; ++q) mbar_init(&bars[2 * q], 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
     float xv[K::D_IN][V], av[K::D_IN][V], gacc[K::D_IN][V];
     load_rows<V>(xv, prm.x + (size_t)node * K::D_IN * C + c0 + cl, C, on);
     load_rows<V>(av, prm.a + (size_t)node * K::D_IN * C + c0 + cl, C, on);
@@ -352,63 +390,90 @@ __global__ void __launch_bounds__(DblShape<K>::WARPS * 32) eqconv_dbl_send_kerne
     for (int d = 0; d < K::D_IN; ++d)
 #pragma unroll
         for (int v = 0; v < V; ++v) gacc[d][v] = 0.f;
-    const int kb = prm.ptr[node], ke = prm.ptr[node + 1];
-    for (int k0 = kb; k0 < ke; k0 += CH) {
-        const int nb = min(CH, ke - k0);
-        int my_e = 0, my_i = -1;
-        if (lane < nb) {
-            my_e = prm.perm[k0 + lane];
-            if ((unsigned)my_e < (unsigned)prm.E) my_i = prm.other[my_e];
-            if ((unsigned)my_i >= (unsigned)prm.N) {
-                atomicOr(prm.status, 1u);
-                my_i = -1;
-            } else {
-                dbl_harmonics<K>(prm.r, prm.q, my_e, AY + lane * 2 * K::D_SH);
-            }
+    uint32_t g = 0;
+    bool ok_all = true;
+    uint32_t fill_from = 0, fill_to = 0;
+    int k = prm.ptr[node];
+    const int ke = prm.ptr[node + 1];
+    while (k < ke && ok_all) {
+        int my_e, my_i;
+        float rx, ry, rz;
+        const int n = gather_window(prm.perm, prm.other, prm.r, prm.N, 0, prm.N, k, ke, prm.status, lane, my_e,
+                                    my_i, rx, ry, rz);
+        if (n == 0) continue;
+        const int pre = min(S, n);
+        for (int t = 0; t < pre; ++t) {
+            const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_i, t);
+            const uint32_t gi = g + t;
+            dbl_fill<K, false>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_b, &tmap_g, nullptr, e,
+                               o, c0, pol_e, pol_n, lane);
         }
-        __syncwarp();
-        SendRows<K> cur, nxt;
-        const auto load = [&](SendRows<K>& rw, int t) {
-            const int e = __shfl_sync(0xffffffffu, my_e, t);
-            const int i = __shfl_sync(0xffffffffu, my_i, t);
-            const bool ld = on && i >= 0;
-            load_rows<V>(rw.w, prm.w + (size_t)e * K::NP * C + c0 + cl, C, ld);
-            load_rows<V>(rw.b, prm.b + (size_t)e * K::NP * C + c0 + cl, C, ld);
-            load_rows<V>(rw.g, prm.gy + (size_t)max(i, 0) * K::D_OUT * C + c0 + cl, C, ld);
-        };
-        if (DblShape<K>::PF) load(cur, 0);
-        for (int t = 0; t < nb; ++t) {
-            if (DblShape<K>::PF) {
-                if (t + 1 < nb) load(nxt, t + 1);
-            } else {
-                load(cur, t);
-            }
-            const int e = __shfl_sync(0xffffffffu, my_e, t);
-            const int i = __shfl_sync(0xffffffffu, my_i, t);
-            if (i < 0) {
-                if (DblShape<K>::PF) cur = nxt;
-                continue;
-            }
-            float gYv[G], gY1[G];
+        for (int b0 = 0; b0 < n && ok_all; b0 += CH) {
+            const int nb = min(CH, n - b0);
+            if (lane >= b0 && lane < b0 + nb) {
+                const float* qe = prm.q + 3 * (size_t)my_e;
+                float ux, uy, uz, il;
+                const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
+                float Y[K::D_SH], rho[K::D_SH];
+                sh_eval<K::LSH>(ok, ux, uy, uz, Y);
+                sh_jvp<K::LSH>(rx, ry, rz, qe[0], qe[1], qe[2], rho);
+                float* yrow = Ys + (lane - b0) * 2 * K::D_SH;
 #pragma unroll
-            for (int k = 0; k < G; ++k) gYv[k] = gY1[k] = 0.f;
-            dbl_send_edge<K>(AY + t * 2 * K::D_SH, xv, av, cur.g, cur.w, cur.b, gacc,
-                             prm.g_w + (size_t)e * K::NP * C + c0 + cl, C, on, gYv, gY1);
-            if (DblShape<K>::PF) cur = nxt;
-            if constexpr (K::G > 0) {
-                warp_sum<G>(gYv);
-                warp_sum<G>(gY1);
-                if (lane == 0) {
-                    float* pp = prm.part + ((size_t)e * prm.T + tile) * 2 * G;
-#pragma unroll
-                    for (int k = 0; k < G; ++k) {
-                        pp[k] = gYv[k];
-                        pp[G + k] = gY1[k];
-                    }
+                for (int q = 0; q < K::D_SH; ++q) {
+                    yrow[q] = Y[q];
+                    yrow[K::D_SH + q] = rho[q];
                 }
             }
+            __syncwarp();
+            for (int t = b0; t < b0 + nb; ++t) {
+                const uint32_t gi = g + t;
+                float* st = stages + (gi % S) * SF;
+                if (!mbar_wait(&bars[2 * (gi % S)], (gi / S) & 1u)) {
+                    if (lane == 0) atomicOr(prm.status, 4u);
+                    ok_all = false;
+                    fill_from = gi;
+                    fill_to = g + (uint32_t)min(n, t + S);
+                    break;
+                }
+                const int e = __shfl_sync(0xffffffffu, my_e, t);
+                float wv[K::NP][V], bv[K::NP][V], gv[K::D_OUT][V];
+#pragma unroll
+                for (int p = 0; p < K::NP; ++p) {
+                    lds_vec<V>(wv[p], st + p * K::TILE_C + cl);
+                    lds_vec<V>(bv[p], st + (K::NP + p) * K::TILE_C + cl);
+                }
+#pragma unroll
+                for (int d = 0; d < K::D_OUT; ++d) lds_vec<V>(gv[d], st + (2 * K::NP + d) * K::TILE_C + cl);
+                float gYv[G], gY1[G];
+#pragma unroll
+                for (int q = 0; q < G; ++q) gYv[q] = gY1[q] = 0.f;
+                dbl_send_edge<K>(Ys + (t - b0) * 2 * K::D_SH, xv, av, gv, wv, bv, gacc,
+                                 prm.g_w + (size_t)e * K::NP * C + c0 + cl, C, on, gYv, gY1);
+                __syncwarp();
+                if (t + S < n) {
+                    const int e2 = __shfl_sync(0xffffffffu, my_e, t + S), o2 = __shfl_sync(0xffffffffu, my_i, t + S);
+                    dbl_fill<K, false>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_b, &tmap_g, nullptr, e2, o2, c0,
+                                       pol_e, pol_n, lane);
+                }
+                if constexpr (K::G > 0) {
+                    // the 2G partials summed over the warp at once; value q lands on lanes q << SH ..
+                    constexpr int NV = pow2_at_least(2 * G), SH = transpose_sum_shift(NV);
+                    float tv[NV];
+#pragma unroll
+                    for (int q = 0; q < NV; ++q) tv[q] = q < G ? gYv[q] : (q < 2 * G ? gY1[q - G] : 0.f);
+                    const float sum = warp_transpose_sum<NV>(tv, lane);
+                    const int q = lane >> SH;
+                    if ((lane & ((1 << SH) - 1)) == 0 && q < 2 * G)
+                        prm.part[((size_t)e * prm.T + tile) * 2 * G + q] = sum;
+                }
+            }
+            __syncwarp();
         }
-        __syncwarp();
+        g += n;
+    }
+    if (!ok_all) {
+        drain_fills<S>(bars, fill_from, fill_to);
+        return;
     }
     if (on) {
         float* gj = prm.g_x + (size_t)node * K::D_IN * C + c0 + cl;

@@ -16,19 +16,34 @@ namespace eqc {
 template <class K>
 struct DblLaunch {
     static cudaError_t run(const DblParams& prm, const DblParams& send_prm, cudaStream_t st) {
-        constexpr int W = DblShape<K>::WARPS, smem = DblShape<K>::SMEM;
+        using LR = DblRing<K, true>;
+        using LS = DblRing<K, false>;
         auto recv = eqconv_dbl_recv_kernel<K>;
         auto send = eqconv_dbl_send_kernel<K>;
         static bool done_recv[64] = {}, done_send[64] = {};
-        cudaError_t err = ensure_smem(recv, smem, done_recv);
-        if (err == cudaSuccess) err = ensure_smem(send, smem, done_send);
+        cudaError_t err = ensure_smem(recv, LR::SMEM, done_recv);
+        if (err == cudaSuccess) err = ensure_smem(send, LS::SMEM, done_send);
         if (err != cudaSuccess) return err;
         if (prm.N > 0) {
-            const dim3 grid((prm.N + W - 1) / W, prm.T);
-            recv<<<grid, W * 32, smem, st>>>(prm);
+            // with no edges the edge maps are never read: give them a valid stand-in
+            const bool edges = prm.E > 0;
+            const void* wb = edges ? (const void*)prm.w : (const void*)prm.x;
+            const void* bb = edges ? (const void*)prm.b : (const void*)prm.x;
+            const uint64_t ne = edges ? (uint64_t)prm.E : (uint64_t)prm.N;
+            const int nr = edges ? K::NP : K::D_IN;
+            CUtensorMap tw, tb, tx, ta, tg;
+            if (!encode_rows_map(&tw, wb, ne, nr, prm.C, K::TILE_C) ||
+                !encode_rows_map(&tb, bb, ne, nr, prm.C, K::TILE_C) ||
+                !encode_rows_map(&tx, prm.x, (uint64_t)prm.N, K::D_IN, prm.C, K::TILE_C) ||
+                !encode_rows_map(&ta, prm.a, (uint64_t)prm.N, K::D_IN, prm.C, K::TILE_C) ||
+                !encode_rows_map(&tg, prm.gy, (uint64_t)prm.N, K::D_OUT, prm.C, K::TILE_C))
+                return cudaErrorInvalidValue;
+            recv<<<dim3((prm.N + LR::WARPS - 1) / LR::WARPS, prm.T), LR::WARPS * 32, LR::SMEM, st>>>(prm, tw, tb, tx,
+                                                                                                  ta);
             count_launch();
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
-            send<<<grid, W * 32, smem, st>>>(send_prm);
+            send<<<dim3((prm.N + LS::WARPS - 1) / LS::WARPS, prm.T), LS::WARPS * 32, LS::SMEM, st>>>(send_prm, tw, tb,
+                                                                                                  tg);
             count_launch();
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
         }

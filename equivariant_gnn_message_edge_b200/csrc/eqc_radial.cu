@@ -59,14 +59,17 @@ __global__ void __launch_bounds__(1024)
 // power of two s (H_hi / H_lo [E][64]), uscale[k] = u(d) 2^-(s_W3 + s) (so
 // that w = D * uscale) and zscale[k] = 2^-(s_W3 + s) (may be null).  hmax
 // (may be null) receives the largest |h2| of all edges (as the bits of a
-// non-negative float, by atomicMax).  One thread per edge; W1 and W2 are read
-// from shared memory by all threads at once.
+// non-negative float, by atomicMax).  rec / ids (may be null) receive the
+// position's record for the fused kernels: (r_e, uscale) and (gathered[e],
+// own[e]), so they read positions in order with no dependent loads.  One
+// thread per edge; W1 and W2 are read from shared memory by all threads.
 __global__ void __launch_bounds__(128)
     radial_hidden_kernel(const float* __restrict__ r, const int* __restrict__ perm, int E,
                          const float* __restrict__ W1, const float* __restrict__ W2, int NB, float rc,
                          const float* __restrict__ w3_inv_scale, __half* __restrict__ H_hi,
                          __half* __restrict__ H_lo, float* __restrict__ uscale, float* __restrict__ zscale,
-                         unsigned* __restrict__ hmax) {
+                         unsigned* __restrict__ hmax, const int* __restrict__ gathered,
+                         const int* __restrict__ own, float4* __restrict__ rec, int2* __restrict__ ids) {
     __shared__ __align__(16) float sW1[kMaxBasis * kH];
     __shared__ __align__(16) float sW2[kH * kH];
     for (int i = threadIdx.x; i < NB * kH; i += blockDim.x) sW1[i] = W1[i];
@@ -130,8 +133,13 @@ __global__ void __launch_bounds__(128)
             dl[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
         const float z = ldexpf(1.f, -s) * w3_inv_scale[0];
-        uscale[k] = envelope(d, rc) * z;
+        const float us = envelope(d, rc) * z;
+        uscale[k] = us;
         if (zscale) zscale[k] = z;
+        if (rec) {   // the fused kernels' per-position record, in the order they walk
+            rec[k] = make_float4(rx, ry, rz, us);
+            ids[k] = make_int2(gathered[e], own[e]);
+        }
     }
     if (hmax) {   // blockDim is a multiple of 32: every lane of the warp is here
 #pragma unroll
@@ -282,6 +290,10 @@ Workspace carve(void* ws, int E, int PC) {
     p += up256((size_t)(E > 0 ? E : 1) * 4);
     w.zscale = reinterpret_cast<float*>(p);
     p += up256((size_t)(E > 0 ? E : 1) * 4);
+    w.rec = reinterpret_cast<float4*>(p);
+    p += up256((size_t)(E > 0 ? E : 1) * 16);
+    w.ids = reinterpret_cast<int2*>(p);
+    p += up256((size_t)(E > 0 ? E : 1) * 8);
     w.bytes = (size_t)(p - static_cast<char*>(ws));
     return w;
 }
@@ -289,13 +301,15 @@ Workspace carve(void* ws, int E, int PC) {
 size_t workspace_bytes(int E, int PC) { return carve(nullptr, E, PC).bytes; }
 
 cudaError_t prepare(const Workspace& ws, const float* r, const int* perm, int E, const float* W1, const float* W2,
-                    const float* W3, int NB, float rc, int PC, cudaStream_t st, unsigned* hmax) {
+                    const float* W3, int NB, float rc, int PC, cudaStream_t st, unsigned* hmax, const int* gathered,
+                    const int* own) {
     radial_prep_w3_kernel<<<1, 1024, 0, st>>>(W3, PC, ws.a_hi, ws.a_lo, ws.inv_scale);
     count_launch();
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess || E == 0) return err;
     radial_hidden_kernel<<<(E + 127) / 128, 128, 0, st>>>(r, perm, E, W1, W2, NB, rc, ws.inv_scale, ws.h_hi,
-                                                          ws.h_lo, ws.uscale, ws.zscale, hmax);
+                                                          ws.h_lo, ws.uscale, ws.zscale, hmax, gathered, own,
+                                                          gathered ? ws.rec : nullptr, gathered ? ws.ids : nullptr);
     count_launch();
     return cudaGetLastError();
 }

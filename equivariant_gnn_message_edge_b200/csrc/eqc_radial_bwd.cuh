@@ -59,12 +59,10 @@ constexpr uint32_t kColGD = 384;    // Gd: 64 columns (M = 64 layout)
 
 struct RadBwdParams {
     const float* x;        // [N][D_in][C]
-    const float* r;        // [E][3]
     const float* gy;       // [N][D_out][C] (the plan's output layout)
     const int* ptr;        // send_ptr [N+1]
-    const int* perm;       // send_perm [E]
-    const int* receivers;  // [E]
-    const float* uscale;   // [E] by sender position
+    const float4* rec;     // [E] (r_e, uscale) by sender position
+    const int2* ids;       // [E] (receiver, sender) by sender position
     const float* scal;     // [0] 2^-sA; [1..3] bits of max|x|, max|gy|, max|u h2|
     float* dx_pp;          // [N][DX_PP][C] per-path dx blocks
     float* gy_part;        // [E][slices][SD2] per-path harmonic-gradient partials
@@ -124,20 +122,28 @@ struct RadBwdSmem {
     static constexpr int GY_SLOT = K::D_OUT * kSlice * 4;
     static constexpr int GY_OFF = G_OFF + kBwdGroupTiles * 2 * G_TILE;
     static constexpr int YS = (K::D_SH + 3) & ~3;                         // harmonics row (floats)
-    static constexpr int Y_WARP = kBatch * (YS + 4) * 4;                  // + the batch's edge factor
-    // gy ring depth: what fits beside the rest (2 .. kGySlots)
-    static constexpr int FIXED = GY_OFF + kBwdPathWarps * Y_WARP + (14 + 2 * kGySlots) * 8 + 16 + 1024;
+    // per path warp, for a batch of up to 8 positions: harmonics rows + edge factor, and w
+    static constexpr int Y_WARP8 = 8 * (YS + 4) * 4 + 8 * 32 * 4;
+    // gy ring: batches of BT receiver rows, as many (2 .. 4) as fit beside the rest;
+    // BT = 8 where two batches of 8 fit, else 4, else 2
+    static constexpr int FIXED = GY_OFF + kBwdPathWarps * Y_WARP8 + (14 + 2 * 4) * 8 + 16 + 1024;
     static constexpr int FIT = (227 * 1024 - FIXED) / GY_SLOT;
-    static constexpr int GYS = FIT > kGySlots ? kGySlots : (FIT < 2 ? 2 : FIT);
-    static constexpr int Y_OFF = GY_OFF + GYS * GY_SLOT;
-    static constexpr int BAR_OFF = Y_OFF + kBwdPathWarps * Y_WARP;
+    static constexpr int BT = FIT >= 16 ? 8 : (FIT >= 8 ? 4 : 2);
+    static constexpr int GYB = FIT / BT >= 4 ? 4 : FIT / BT;
+    static constexpr int Y_WARP = BT * (YS + 4) * 4;
+    static constexpr int WS_WARP = BT * 32 * 4;
+    static constexpr int Y_OFF = GY_OFF + GYB * BT * GY_SLOT;
+    static constexpr int WS_OFF = Y_OFF + kBwdPathWarps * Y_WARP;
+    static constexpr int BAR_OFF = WS_OFF + kBwdPathWarps * WS_WARP;
     // w3, h_full[2], h_empty[2], t_full[2], t_empty[2], g_full, g_empty, gd_full, gd_empty, gw_full,
-    // gy_full[GYS], gy_empty[GYS]
-    static constexpr int NBAR = 14 + 2 * GYS;
+    // gy_full[GYB], gy_empty[GYB]
+    static constexpr int NBAR = 14 + 2 * GYB;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int END = MISC_OFF + 16;
     static constexpr int BYTES = END + 1024;
+    static_assert(GYB >= 2, "fused radial backward: room for two gy batches");
     static_assert(BYTES <= 227 * 1024, "fused radial backward: shared memory");
+    static_assert(kEdgeTile % BT == 0, "batches tile the MMA tile");
 };
 
 // One fp16 chunk of 8 edges for G row `row` at edge chunk `q8` of a 128 x 64
@@ -152,18 +158,22 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
                                               int slices, int gexp, volatile int* abort_flag) {
     using S = RadBwdSmem<K>;
     using R = BwdRows<K>;
+    constexpr int BT = S::BT;
     constexpr int l1 = K::PL.l1[P_], l2 = K::PL.l2[P_], l3 = K::PL.l3[P_];
     constexpr int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
     constexpr int o1 = l1 * l1, o3 = K::PL.o3[P_], o2 = l2 * l2;
     constexpr int oxp = R::dx_off(P_), ogp = R::gy_off(P_);
+    constexpr int NVAL = l2 > 0 ? 1 + d2 : 1;                    // partials of one edge
+    constexpr int NV = pow2_at_least(NVAL);
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::BAR_OFF);
     uint64_t* t_full = bars + 5;
     uint64_t* t_empty = bars + 7;
     uint64_t* g_full = bars + 9;
     uint64_t* g_empty = bars + 10;
     uint64_t* gy_full = bars + 14;
-    uint64_t* gy_empty = bars + 14 + S::GYS;
-    float* ys = reinterpret_cast<float*>(base + S::Y_OFF + warp * S::Y_WARP);   // [kBatch][YS + 4]
+    uint64_t* gy_empty = bars + 14 + S::GYB;
+    float* ys = reinterpret_cast<float*>(base + S::Y_OFF + warp * S::Y_WARP);     // [BT][YS + 4]
+    float* wst = reinterpret_cast<float*>(base + S::WS_OFF + warp * S::WS_WARP);  // [BT][32]
     const float* gring = reinterpret_cast<const float*>(base + S::GY_OFF);
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int tile = warp >> 2;                    // MMA tile of this path
@@ -173,88 +183,114 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
     const float gscale0 = ldexpf(1.f, gexp);       // G / dw = 2^gexp * uscale_e
     const int C = prm.C;
     const size_t cl = (size_t)c0 + lane;
+    auto abort_now = [&]() {
+        if (lane == 0) atomicOr(prm.status, 4u);
+        *abort_flag = 1;
+    };
 
-    float xv[d1], dxa[d1];
+    // x rows of the current sender, and of the next one (prefetched)
+    float xv[d1], xn[d1], dxa[d1];
     int cur = n0;
-    int cur_end = prm.ptr[n0 + 1];
-    auto load_x = [&]() {
-        const float* xs = prm.x + ((size_t)cur * K::D_IN + o1) * C + cl;
+    auto load_x = [&](int node, float (&dst)[d1]) {
+        if (node < n1) {
+            const float* xs = prm.x + ((size_t)node * K::D_IN + o1) * C + cl;
 #pragma unroll
-        for (int m = 0; m < d1; ++m) {
-            xv[m] = __ldg(xs + (size_t)m * C);
-            dxa[m] = 0.f;
+            for (int m = 0; m < d1; ++m) dst[m] = __ldg(xs + (size_t)m * C);
         }
     };
     auto flush = [&]() {
         float* dxo = prm.dx_pp + ((size_t)cur * R::DX_PP + oxp) * C + cl;
 #pragma unroll
-        for (int m = 0; m < d1; ++m) __stcs(dxo + (size_t)m * C, dxa[m]);
+        for (int m = 0; m < d1; ++m) {
+            __stcs(dxo + (size_t)m * C, dxa[m]);
+            dxa[m] = 0.f;
+        }
     };
-    load_x();
+    auto next_sender = [&]() {   // cur -> cur + 1, x from the prefetch
+        flush();
+        ++cur;
+#pragma unroll
+        for (int m = 0; m < d1; ++m) xv[m] = xn[m];
+        load_x(cur + 1, xn);
+    };
+#pragma unroll
+    for (int m = 0; m < d1; ++m) {
+        xv[m] = 0.f;
+        xn[m] = 0.f;
+        dxa[m] = 0.f;
+    }
+    load_x(cur, xv);
+    load_x(cur + 1, xn);
 
-    uint32_t ghi[4], glo[4];   // 8 edges of fp16 G values, packed in pairs
+    // the next batch's records (lane t < BT holds position kb + t), prefetched
+    float4 nrec = make_float4(0.f, 0.f, 0.f, 0.f);
+    int nown = 0;
+    if (lane < BT && k0 + lane < k1) {
+        nrec = prm.rec[k0 + lane];
+        nown = prm.ids[k0 + lane].y;
+    }
+
+    uint32_t ghi[4] = {0u, 0u, 0u, 0u}, glo[4] = {0u, 0u, 0u, 0u};   // 8 edges of fp16 G values
     const int ntiles = (k1 - k0 + kEdgeTile - 1) / kEdgeTile;
     for (int j = 0; j < ntiles; ++j) {
         const int s = j & 1;
         if (!mbar_wait(&t_full[s], (uint32_t)(j >> 1) & 1u) || __any_sync(0xffffffffu, *abort_flag)) {
-            if (lane == 0) atomicOr(prm.status, 4u);
-            *abort_flag = 1;
+            abort_now();
             return;
         }
         tc_fence_after();
         // the G tile of the previous tile has been read by the MMAs
         if (j > 0 && !mbar_wait(g_empty, (uint32_t)(j - 1) & 1u)) {
-            if (lane == 0) atomicOr(prm.status, 4u);
-            *abort_flag = 1;
+            abort_now();
             return;
         }
         const uint32_t tcol = tmem + lane_base + kColW + (uint32_t)((s * kBwdGroupTiles + tile) * kEdgeTile);
         const int kt = k0 + j * kEdgeTile;
         const int kt_end = min(k1, kt + kEdgeTile);
-        for (int kb = kt; kb < kt + kEdgeTile; kb += kBatch) {
-            const int nb = max(0, min(kBatch, kt_end - kb));
-            if (lane < nb) {
-                const int k = kb + lane;
-                const int e = prm.perm[k];
-                float ux, uy, uz, il;
-                const bool ok = unit_dir(prm.r[(size_t)e * 3], prm.r[(size_t)e * 3 + 1], prm.r[(size_t)e * 3 + 2],
-                                         ux, uy, uz, il);
-                float Y[K::D_SH];
-                sh_eval<K::LSH>(ok, ux, uy, uz, Y);
-                float* yrow = ys + lane * (S::YS + 4);
+        for (int kb = kt; kb < kt + kEdgeTile; kb += BT) {
+            const int nb = max(0, min(BT, kt_end - kb));
+            const int b = (kb - k0) / BT;
+            int own = 0;
+            const float* gb = gring;
+            if (nb > 0) {
+                const float4 rc = nrec;
+                own = nown;
+                if (lane < BT && kb + BT + lane < k1) {   // prefetch the batch after this one
+                    nrec = prm.rec[kb + BT + lane];
+                    nown = prm.ids[kb + BT + lane].y;
+                }
+                if (lane < nb) {
+                    float ux, uy, uz, il;
+                    const bool ok = unit_dir(rc.x, rc.y, rc.z, ux, uy, uz, il);
+                    float Y[K::D_SH];
+                    sh_eval<K::LSH>(ok, ux, uy, uz, Y);
+                    float* yrow = ys + lane * (S::YS + 4);
 #pragma unroll
-                for (int q = 0; q < K::D_SH; ++q) yrow[q] = Y[q];
-                yrow[S::YS] = prm.uscale[k];
+                    for (int q = 0; q < K::D_SH; ++q) yrow[q] = Y[q];
+                    yrow[S::YS] = rc.w;
+                }
+                tmem_stash<BT>(tcol + (uint32_t)(kb - kt), wst, lane);   // z3 * 2^(sA + sB), BT positions
+                __syncwarp();
+                if (!mbar_wait(&gy_full[b % S::GYB], (uint32_t)(b / S::GYB) & 1u) ||
+                    __any_sync(0xffffffffu, *abort_flag)) {
+                    abort_now();
+                    return;
+                }
+                gb = gring + (b % S::GYB) * BT * (S::GY_SLOT / 4) + o3 * kSlice + lane;
             }
-            __syncwarp();
-            for (int t = 0; t < kBatch; ++t) {
-                const int k = kb + t;
+            for (int t = 0; t < BT; ++t) {
                 float gval = 0.f;
                 if (t < nb) {
-                    while (k >= cur_end) {   // the current sender's edges are done (empty ones too)
-                        flush();
-                        ++cur;
-                        cur_end = prm.ptr[cur + 1];
-                        load_x();
-                    }
+                    const int own_t = __shfl_sync(0xffffffffu, own, t);
+                    while (cur < own_t) next_sender();   // the current sender's edges are done (empty ones too)
                     const float* yrow = ys + t * (S::YS + 4);
                     const float us = yrow[S::YS];
-                    const float Dv = tmem_ld1(tcol + (uint32_t)(k - kt));   // z3 * 2^(sA + sB)
+                    const float Dv = wst[t * 32 + lane];
                     const float w = Dv * us;
-                    const int q = k - k0;
-                    const int slot = q % S::GYS;
-                    if (!mbar_wait(&gy_full[slot], (uint32_t)(q / S::GYS) & 1u) ||
-                        __any_sync(0xffffffffu, *abort_flag)) {
-                        if (lane == 0) atomicOr(prm.status, 4u);
-                        *abort_flag = 1;
-                        return;
-                    }
-                    const float* gs = gring + slot * (S::GY_SLOT / 4) + o3 * kSlice + lane;
+                    const float* gs = gb + t * (S::GY_SLOT / 4);
                     float gv[d3];
 #pragma unroll
                     for (int m = 0; m < d3; ++m) gv[m] = gs[m * kSlice];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&gy_empty[slot]);
                     float tv[d1];
                     [[maybe_unused]] float hG[d2];
                     if constexpr (l2 == 0) {
@@ -291,46 +327,42 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
                     gval = dw * gscale0 * us;
                     // this path's partials of the edge, summed over the 32 channels:
                     // sum dw z3 (scaled; for g_u) and the harmonic gradient
-                    float gu = dw * Dv;
+                    float v[NV];
+                    v[0] = dw * Dv;
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) gu += __shfl_xor_sync(0xffffffffu, gu, o);
+                    for (int q = 1; q < NV; ++q) v[q] = 0.f;
                     if constexpr (l2 > 0) {
 #pragma unroll
-                        for (int m = 0; m < d2; ++m) {
-                            float v = w * hG[m];
-#pragma unroll
-                            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                            hG[m] = v;
-                        }
+                        for (int m = 0; m < d2; ++m) v[1 + m] = w * hG[m];
                     }
-                    if (lane == 0) {
-                        float* gp = prm.gy_part + ((size_t)k * slices + slice) * R::SD2 + ogp;
-                        gp[0] = gu;
-                        if constexpr (l2 > 0) {
-#pragma unroll
-                            for (int m = 0; m < d2; ++m) gp[1 + m] = hG[m];
-                        }
-                    }
+                    const float sum = warp_transpose_sum<NV>(v, lane);
+                    constexpr int sh = transpose_sum_shift(NV);
+                    const int vi = lane >> sh;
+                    if ((lane & ((1 << sh) - 1)) == 0 && vi < NVAL)
+                        prm.gy_part[((size_t)(kb + t) * slices + slice) * R::SD2 + ogp + vi] = sum;
                 }
                 // pack G (zero for edges past the range) and store every 8 edges
                 __half gh, gl;
                 split_f16(gval, gh, gl);
-                const int pr = t & 7;
+                const int pos = kb - kt + t;
+                const int pr = pos & 7;
                 const uint32_t bh = __half_as_ushort(gh), bl = __half_as_ushort(gl);
-                if ((pr & 1) == 0) {
-                    ghi[pr >> 1] = bh;
-                    glo[pr >> 1] = bl;
-                } else {
-                    ghi[pr >> 1] |= bh << 16;
-                    glo[pr >> 1] |= bl << 16;
+                // 128-bit shift registers: after 8 edges edge i sits at bits 16 i
+#pragma unroll
+                for (int q = 0; q < 3; ++q) {
+                    ghi[q] = __funnelshift_r(ghi[q], ghi[q + 1], 16);
+                    glo[q] = __funnelshift_r(glo[q], glo[q + 1], 16);
                 }
+                ghi[3] = (ghi[3] >> 16) | (bh << 16);
+                glo[3] = (glo[3] >> 16) | (bl << 16);
                 if (pr == 7) {
-                    const uint32_t off = g_chunk_offset(grow, (kb - kt + t) >> 3);
+                    const uint32_t off = g_chunk_offset(grow, pos >> 3);
                     *reinterpret_cast<uint4*>(g_hi + off) = make_uint4(ghi[0], ghi[1], ghi[2], ghi[3]);
                     *reinterpret_cast<uint4*>(g_lo + off) = make_uint4(glo[0], glo[1], glo[2], glo[3]);
                 }
             }
             __syncwarp();
+            if (nb > 0 && lane == 0) mbar_arrive(&gy_empty[b % S::GYB]);
         }
         // G written (generic proxy) -> visible to the tensor cores (async proxy)
         fence_proxy_async();
@@ -342,11 +374,8 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
         }
     }
     // the last sender and any empty ones after it
-    while (true) {
-        flush();
-        if (++cur >= n1) break;
-        load_x();
-    }
+    while (cur + 1 < n1) next_sender();
+    flush();
 }
 
 template <class K>
@@ -369,7 +398,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t* gd_empty = bars + 12;
     uint64_t* gw_full = bars + 13;
     uint64_t* gy_full = bars + 14;
-    uint64_t* gy_empty = bars + 14 + S::GYS;
+    uint64_t* gy_empty = bars + 14 + S::GYB;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base + S::MISC_OFF + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -399,7 +428,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(gd_full, 1);
         mbar_init(gd_empty, 4);
         mbar_init(gw_full, 1);
-        for (int q = 0; q < S::GYS; ++q) {
+        for (int q = 0; q < S::GYB; ++q) {
             mbar_init(&gy_full[q], 1);
             mbar_init(&gy_empty[q], gp);
         }
@@ -495,24 +524,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tma_2d(dst, &map_a_hi, 0, row, w3_full);
                     tma_2d(dst + S::A_TILE, &map_a_lo, 0, row, w3_full);
                 }
+            int h_issued = 0, h_waited = 0, committed = 0, g_done = 0;
             auto load_h = [&](int j) {
                 const int s = j & 1;
                 uint8_t* dst = base + S::H_OFF + s * 2 * S::H_TILE;
                 mbar_expect_tx(&h_full[s], 2 * S::H_TILE);
                 tma_2d(dst, &map_h_hi, 0, k0 + j * kEdgeTile, &h_full[s]);
                 tma_2d(dst + S::H_TILE, &map_h_lo, 0, k0 + j * kEdgeTile, &h_full[s]);
+                h_issued = j + 1;
             };
             load_h(0);
             if (ntiles > 1) load_h(1);
-            bool ok = mbar_wait_one(w3_full, 0);
+            const bool w3_ok = mbar_wait_one(w3_full, 0);
+            bool ok = w3_ok;
             constexpr uint32_t id_w = idesc_f16(kRowTile, kEdgeTile);                 // W3^T . H^T
             constexpr uint32_t id_gw = idesc_f16(kRowTile, kH, false, true);          // G . H (B MN-major)
             constexpr uint32_t id_gd = idesc_f16(kH, kEdgeTile, true, true);          // W3 . G (both MN-major)
             for (int j = 0; j < ntiles && ok; ++j) {
                 const int s = j & 1;
-                ok = mbar_wait_one(&h_full[s], (uint32_t)(j >> 1) & 1u) &&
-                     (j < 2 || mbar_wait_one(&t_empty[s], (uint32_t)((j >> 1) - 1) & 1u));
-                if (!ok || *abort_flag) break;
+                ok = mbar_wait_one(&h_full[s], (uint32_t)(j >> 1) & 1u);
+                if (!ok) break;
+                h_waited = j + 1;
+                ok = (j < 2 || mbar_wait_one(&t_empty[s], (uint32_t)((j >> 1) - 1) & 1u)) && !*abort_flag;
+                if (!ok) break;
                 tc_fence_after();
                 const uint8_t* hs = base + S::H_OFF + s * 2 * S::H_TILE;
                 const uint64_t dbh = sw128_desc(smem_addr(hs)), dbl = sw128_desc(smem_addr(hs + S::H_TILE));
@@ -530,10 +564,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                 }
                 umma_commit(&t_full[s]);
+                committed = j + 1;
                 // the path warps' G tile of this tile, then g_W3 += G . H and Gd = W3 . G
                 ok = mbar_wait_one(g_full, (uint32_t)j & 1u) &&
-                     (j == 0 || mbar_wait_one(gd_empty, (uint32_t)(j - 1) & 1u));
-                if (!ok || *abort_flag) break;
+                     (j == 0 || mbar_wait_one(gd_empty, (uint32_t)(j - 1) & 1u)) && !*abort_flag;
+                if (!ok) break;
                 tc_fence_after();
                 for (int t = 0; t < gtiles; ++t) {
                     const uint8_t* gt = base + S::G_OFF + t * 2 * S::G_TILE;
@@ -564,6 +599,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 umma_commit(g_empty);
                 umma_commit(gd_full);
                 umma_commit(&h_empty[s]);
+                g_done = j + 1;
                 if (j + 2 < ntiles) {
                     ok = mbar_wait_one(&h_empty[s], (uint32_t)(j >> 1) & 1u);
                     if (ok) load_h(j + 2);
@@ -574,28 +610,50 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             } else {
                 atomicOr(prm.status, 4u);
                 *abort_flag = 1;
+                // let the copies and products in flight land before the CTA lets go of its memory
+                if (!w3_ok) mbar_wait_one(w3_full, 0);
+                for (int u = h_waited; u < h_issued; ++u) mbar_wait_one(&h_full[u & 1], (uint32_t)(u >> 1) & 1u);
+                for (int u = committed > 2 ? committed - 2 : 0; u < committed; ++u)
+                    mbar_wait_one(&t_full[u & 1], (uint32_t)(u >> 1) & 1u);
+                if (g_done > 0) mbar_wait_one(g_empty, (uint32_t)(g_done - 1) & 1u);
             }
         }
     } else if (warp == kBwdGyWarp) {
-        if (lane == 0) {
-            for (int k = k0; k < k1; ++k) {
-                const int q = k - k0, slot = q % S::GYS;
-                if (q >= S::GYS && !mbar_wait_one(&gy_empty[slot], (uint32_t)(q / S::GYS - 1) & 1u)) {
-                    atomicOr(prm.status, 4u);
-                    *abort_flag = 1;
-                    break;
-                }
-                if (*abort_flag) break;
-                int ridx = prm.receivers[prm.perm[k]];
-                if ((unsigned)ridx >= (unsigned)prm.N) {
+        // receiver rows of gy, batch by batch: one barrier per batch of BT
+        // positions; lane t copies the row of position kb + t
+        constexpr int BT = S::BT;
+        const int nbatch = (k1 - k0 + BT - 1) / BT;
+        int issued = 0;
+        for (int b = 0; b < nbatch; ++b) {
+            const int kb = k0 + b * BT;
+            const int nb = min(BT, k1 - kb);
+            int ridx = 0;
+            if (lane < nb) {
+                ridx = prm.ids[kb + lane].x;
+                if ((unsigned)ridx >= (unsigned)prm.N) {   // out of range: flagged, read as node 0
                     atomicOr(prm.status, 1u);
                     ridx = 0;
                 }
-                mbar_expect_tx(&gy_full[slot], S::GY_SLOT);
-                tma_rows(base + S::GY_OFF + slot * S::GY_SLOT, &map_gy, c0, ridx, &gy_full[slot],
-                         policy_evict_last());
             }
+            int go = 1;
+            if (lane == 0) {
+                if (b >= S::GYB && !mbar_wait_one(&gy_empty[b % S::GYB], (uint32_t)(b / S::GYB - 1) & 1u)) {
+                    atomicOr(prm.status, 4u);
+                    *abort_flag = 1;
+                }
+                go = *abort_flag ? 0 : 1;
+                if (go) mbar_expect_tx(&gy_full[b % S::GYB], nb * S::GY_SLOT);
+            }
+            if (!__shfl_sync(0xffffffffu, go, 0)) break;
+            if (lane < nb)
+                tma_rows(base + S::GY_OFF + ((b % S::GYB) * BT + lane) * S::GY_SLOT, &map_gy, c0, ridx,
+                         &gy_full[b % S::GYB], policy_evict_last());
+            issued = b + 1;
         }
+        // the last fills of each buffer land before the CTA lets go of its memory
+        if (lane == 0)
+            for (int b = issued > S::GYB ? issued - S::GYB : 0; b < issued; ++b)
+                mbar_wait_one(&gy_full[b % S::GYB], (uint32_t)(b / S::GYB) & 1u);
     }
     tc_fence_before();
     __syncthreads();
@@ -658,22 +716,27 @@ __global__ void radial_sum_dx_kernel(const float* __restrict__ dx_pp, float* __r
     __stcs(reinterpret_cast<float4*>(dx + ((size_t)j * K::D_IN + row) * C) + cq, s);
 }
 
-// Per sender position k (edge e = perm[k]), one thread each, 64 per CTA, the
-// CTA walking `chunks` chunks of 64 positions:
-//   Gd = sum of the (slice, group) partials, unscaled;  g_h2 = u Gd,
+// Per tile of 64 sender positions k (edge e = perm[k]); 256 threads, the CTA
+// walking `chunks` tiles in order:
+//   Gd = sum of the (slice, group) partials, unscaled;  g_z2 = u Gd silu'(z2);
 //   g_u = h2 . Gd;  back through the two SiLU layers (recomputed) to g_b;
 //   g_d = g_b . b'(d) + g_u u'(d);  gY = sum of the per-path partials;
 //   dr[e] = (dY/dr)^T gY + g_d r / d.
-// The CTA's partial sums of g_W2 = sum_e h1 (x) g_z2 and g_W1 = sum_e b (x)
-// g_z1 are accumulated in a fixed order (thread t owns row t) and written to
+// The MLP layers of a tile are small GEMMs ([64 positions] x [64] x [64]):
+// each thread owns a 4 x 4 block of every product (rows 4 tk.., columns
+// 4 tj..), operands from shared memory as float4 rows.  The CTA's partial
+// sums of g_W2 = sum_k h1 (x) g_z2 and g_W1 = sum_k b (x) g_z1 stay in the
+// threads' registers (positions in order: deterministic) and go to
 // gw2_part / gw1_part [CTA].
-constexpr int kEpiThreads = 64;
-constexpr int kEpiStride = kH + 1;   // thread-private smem rows (conflict-free)
-constexpr int kEpiSmemBytes =
-    (kMaxBasis * kH + kH * kH + 3 * kEpiThreads * kEpiStride + kEpiThreads * (kMaxBasis + 1)) * 4;
+constexpr int kEpiThreads = 256;
+constexpr int kEpiTile = 64;             // positions per tile
+constexpr int kEpiLd = kH + 4;           // padded row stride of the activation tiles
+constexpr int kEpiSmemFloats =
+    kMaxBasis * kH + 2 * kH * kH + 3 * kEpiTile * kEpiLd + 2 * kEpiTile * kMaxBasis + 3 * kEpiTile;
+constexpr int kEpiSmemBytes = kEpiSmemFloats * 4;
 
 template <class K>
-__global__ void __launch_bounds__(kEpiThreads)
+__global__ void __launch_bounds__(kEpiThreads, 2)
     radial_bwd_epilogue_kernel(const float* __restrict__ r, const int* __restrict__ perm, int E,
                                const float* __restrict__ W1, const float* __restrict__ W2, int NB, float rc,
                                const float* __restrict__ scal, const float* __restrict__ zscale,
@@ -682,127 +745,253 @@ __global__ void __launch_bounds__(kEpiThreads)
                                float* __restrict__ gw2_part) {
     using R = BwdRows<K>;
     extern __shared__ __align__(16) float epi_smem[];   // kEpiSmemBytes
-    float* sW1 = epi_smem;                               // [kMaxBasis][kH]
+    float* sW1 = epi_smem;                               // [kMaxBasis][kH], rows >= NB zero
     float* sW2 = sW1 + kMaxBasis * kH;                   // [kH][kH]
-    float* sz1 = sW2 + kH * kH;                          // z1, then g_z1 (rows of kEpiStride)
-    float* sh1 = sz1 + kEpiThreads * kEpiStride;         // h1
-    float* sg2 = sh1 + kEpiThreads * kEpiStride;         // g_z2
-    float* sb = sg2 + kEpiThreads * kEpiStride;          // Bessel values (rows of kMaxBasis + 1)
-    const int t = threadIdx.x;
-    for (int i = t; i < NB * kH; i += kEpiThreads) sW1[i] = W1[i];
-    for (int i = t; i < kH * kH; i += kEpiThreads) sW2[i] = W2[i];
+    float* sW2T = sW2 + kH * kH;                         // [kH][kH] transposed
+    float* sH1 = sW2T + kH * kH;                         // [64][kEpiLd] h1
+    float* sG2 = sH1 + kEpiTile * kEpiLd;                // [64][kEpiLd] g_z2
+    float* sG1 = sG2 + kEpiTile * kEpiLd;                // [64][kEpiLd] g_z1
+    float* sB = sG1 + kEpiTile * kEpiLd;                 // [64][kMaxBasis] Bessel values
+    float* sGb = sB + kEpiTile * kMaxBasis;              // [64][kMaxBasis] their derivatives in d
+    float* sFac = sGb + kEpiTile * kMaxBasis;            // [64] unscaling of Gd
+    float* sGud = sFac + kEpiTile;                       // [64] g_u u'(d)
+    float* sGdl = sGud + kEpiTile;                       // [64] g_b . b'(d)
+    const int t = threadIdx.x, tk = t >> 4, tj = t & 15;
+    for (int i = t; i < kMaxBasis * kH; i += kEpiThreads) sW1[i] = i < NB * kH ? W1[i] : 0.f;
+    for (int i = t; i < kH * kH; i += kEpiThreads) {
+        const float v = W2[i];
+        sW2[i] = v;
+        sW2T[(i % kH) * kH + i / kH] = v;
+    }
     const int sA = inv_pow2_exponent(scal[0]);
     const int gexp = g_scale_exponent(scal);
-    float acc2[kH];                       // g_W2 row t
-    float acc1[kMaxBasis];                // g_W1 column t
+    float gw2[4][4];   // g_W2 rows 4 tk + i, columns 4 tj + c
+    float gw1[4];      // g_W1 rows (t >> 6) + 4 i, column t & 63
 #pragma unroll
-    for (int i = 0; i < kH; ++i) acc2[i] = 0.f;
+    for (int i = 0; i < 4; ++i) {
+        gw1[i] = 0.f;
 #pragma unroll
-    for (int i = 0; i < kMaxBasis; ++i) acc1[i] = 0.f;
-    float* z1 = sz1 + t * kEpiStride;
-    float* h1 = sh1 + t * kEpiStride;
-    float* g2 = sg2 + t * kEpiStride;
-    float* bb = sb + t * (kMaxBasis + 1);
+        for (int c = 0; c < 4; ++c) gw2[i][c] = 0.f;
+    }
 
     for (int ch = 0; ch < chunks; ++ch) {
-        __syncthreads();   // weights loaded / previous chunk's rows consumed
-        const int k = (blockIdx.x * chunks + ch) * kEpiThreads + t;
-        const bool live = k < E;
-        if (live) {
-            const int e = perm[k];
-            const float rx = r[(size_t)e * 3], ry = r[(size_t)e * 3 + 1], rz = r[(size_t)e * 3 + 2];
-            const float d = sqrtf(fmaf(rx, rx, fmaf(ry, ry, rz * rz)));
-            const float inv_d = 1.f / fmaxf(d, 1e-12f);
-            const float pref = sqrtf(2.f / rc);
-            const float kd = 3.14159265358979323846f * d / rc;
-            // forward of the MLP, recomputed
-            for (int j = 0; j < kH; ++j) z1[j] = 0.f;
-            float gbd[kMaxBasis];   // b'_n(d)
-            for (int n = 0; n < NB; ++n) {
-                float sn, cn;
-                sincosf((float)(n + 1) * kd, &sn, &cn);
-                const float kn = (float)(n + 1) * 3.14159265358979323846f / rc;
-                const float b = pref * sn * inv_d;
-                bb[n] = b;
-                gbd[n] = pref * (kn * cn * inv_d - sn * inv_d * inv_d);
-                for (int j = 0; j < kH; ++j) z1[j] = fmaf(b, sW1[n * kH + j], z1[j]);
-            }
-            for (int j = 0; j < kH; ++j) h1[j] = silu(z1[j]);
-            float z2[kH];
-#pragma unroll
-            for (int j = 0; j < kH; ++j) z2[j] = 0.f;
-            for (int q = 0; q < kH; ++q) {
-                const float a = h1[q];
-#pragma unroll
-                for (int j = 0; j < kH; j += 4) {
-                    const float4 wv = *reinterpret_cast<const float4*>(&sW2[q * kH + j]);
-                    z2[j] = fmaf(a, wv.x, z2[j]);
-                    z2[j + 1] = fmaf(a, wv.y, z2[j + 1]);
-                    z2[j + 2] = fmaf(a, wv.z, z2[j + 2]);
-                    z2[j + 3] = fmaf(a, wv.w, z2[j + 3]);
+        const int kbase = (blockIdx.x * chunks + ch) * kEpiTile;
+        if (kbase >= E) break;   // uniform over the CTA
+        __syncthreads();   // weights loaded / the previous tile consumed
+        // 1. per-position terms (threads 0..63)
+        float d0 = 0.f, d1v = 0.f, d2v = 0.f, rx = 0.f, ry = 0.f, rz = 0.f, inv_d = 0.f, d = 0.f;
+        int e = -1;
+        if (t < kEpiTile) {
+            const int k = kbase + t;
+            float* bb = sB + t * kMaxBasis;
+            float* gb = sGb + t * kMaxBasis;
+            if (k < E) {
+                e = perm[k];
+                rx = r[(size_t)e * 3];
+                ry = r[(size_t)e * 3 + 1];
+                rz = r[(size_t)e * 3 + 2];
+                d = sqrtf(fmaf(rx, rx, fmaf(ry, ry, rz * rz)));
+                inv_d = 1.f / fmaxf(d, 1e-12f);
+                const float pref = sqrtf(2.f / rc);
+                const float kd = 3.14159265358979323846f * d / rc;
+                for (int n = 0; n < NB; ++n) {
+                    float sn, cn;
+                    sincosf((float)(n + 1) * kd, &sn, &cn);
+                    const float kn = (float)(n + 1) * 3.14159265358979323846f / rc;
+                    bb[n] = pref * sn * inv_d;
+                    gb[n] = pref * (kn * cn * inv_d - sn * inv_d * inv_d);
                 }
-            }
-            const float x = fminf(d / rc, 1.f);
-            // u'(d) = (-168 x^5 + 336 x^6 - 168 x^7) / rc, zero from the cutoff on
-            const float x2 = x * x, x5 = x2 * x2 * x;
-            const float du = d < rc ? x5 * fmaf(x, fmaf(-168.f, x, 336.f), -168.f) / rc : 0.f;
-            // g_h2 = u W3 . dw: with G = dw 2^gexp uscale_e = u dw 2^gexp zscale_e,
-            // D = sum_pc (W3 2^sA) G = 2^(sA + gexp) zscale_e g_h2
-            const float zs = zscale[k];
-            const float fac = ldexpf(1.f, -(sA + gexp)) / zs;
-#pragma unroll
-            for (int j = 0; j < kH; ++j) {
-                float s = 0.f;
-                for (int q = 0; q < SG; ++q) s += gd_part[((size_t)q * E + k) * kH + j];
-                g2[j] = s * fac * silu_grad(z2[j]);
-            }
-            // g_u = sum_pc dw z3: the paths' partials (each sum dw D, D = z3 2^(sA + sB) = z3 / zscale)
-            float gu = 0.f;
-            for (int s = 0; s < slices; ++s) {
-                const float* gp = gy_part + ((size_t)k * slices + s) * R::SD2;
-                static_for<K::NP>([&](auto pc) { gu += gp[R::gy_off(EQC_CV(pc))]; });
-            }
-            gu *= zs;
-            // g_h1 = W2 g_z2, g_z1 = g_h1 silu'(z1)  (z1 row then holds g_z1)
-            for (int q = 0; q < kH; ++q) {
-                float s = 0.f;
-#pragma unroll
-                for (int j = 0; j < kH; j += 4) {
-                    const float4 wv = *reinterpret_cast<const float4*>(&sW2[q * kH + j]);
-                    s = fmaf(wv.x, g2[j], s);
-                    s = fmaf(wv.y, g2[j + 1], s);
-                    s = fmaf(wv.z, g2[j + 2], s);
-                    s = fmaf(wv.w, g2[j + 3], s);
-                }
-                z1[q] = s * silu_grad(z1[q]);
-            }
-            float gd_len = gu * du;
-            for (int n = 0; n < NB; ++n) {
-                float s = 0.f;
-                for (int j = 0; j < kH; ++j) s = fmaf(sW1[n * kH + j], z1[j], s);
-                gd_len = fmaf(s, gbd[n], gd_len);
-            }
-            // harmonic gradient: the per-path partials, in (slice, path) order
-            float ux, uy, uz, il;
-            const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
-            float d0 = 0.f, d1v = 0.f, d2v = 0.f;
-            if constexpr (K::G > 0) {
-                float gY[K::G];
-#pragma unroll
-                for (int q = 0; q < K::G; ++q) gY[q] = 0.f;
+                const float x = fminf(d / rc, 1.f);
+                // u'(d) = (-168 x^5 + 336 x^6 - 168 x^7) / rc, zero from the cutoff on
+                const float x2 = x * x, x5 = x2 * x2 * x;
+                const float du = d < rc ? x5 * fmaf(x, fmaf(-168.f, x, 336.f), -168.f) / rc : 0.f;
+                // with G = dw 2^gexp uscale_e = u dw 2^gexp zscale_e, the summed partials are
+                // D = sum_pc (W3 2^sA) G = 2^(sA + gexp) zscale_e u W3 . dw
+                const float zs = zscale[k];
+                sFac[t] = ldexpf(1.f, -(sA + gexp)) / zs;
+                // g_u = sum_pc dw z3: the paths' partials (each sum dw D, D = z3 / zscale)
+                float gu = 0.f;
                 for (int s = 0; s < slices; ++s) {
                     const float* gp = gy_part + ((size_t)k * slices + s) * R::SD2;
-                    static_for<K::NP>([&](auto pc) {
-                        constexpr int p = EQC_CV(pc);
-                        constexpr int l2 = K::PL.l2[p];
-                        if constexpr (l2 > 0) {
-#pragma unroll
-                            for (int m = 0; m < 2 * l2 + 1; ++m) gY[l2 * l2 - 1 + m] += gp[R::gy_off(p) + 1 + m];
-                        }
-                    });
+                    static_for<K::NP>([&](auto pc) { gu += gp[R::gy_off(EQC_CV(pc))]; });
                 }
-                sh_grad_contract<K::LSH>(ok, ux, uy, uz, il, gY, d0, d1v, d2v);
+                sGud[t] = gu * zs * du;
+                // harmonic gradient: the per-path partials, in (slice, path) order
+                float ux, uy, uz, il;
+                const bool ok = unit_dir(rx, ry, rz, ux, uy, uz, il);
+                if constexpr (K::G > 0) {
+                    float gY[K::G];
+#pragma unroll
+                    for (int q = 0; q < K::G; ++q) gY[q] = 0.f;
+                    for (int s = 0; s < slices; ++s) {
+                        const float* gp = gy_part + ((size_t)k * slices + s) * R::SD2;
+                        static_for<K::NP>([&](auto pc) {
+                            constexpr int p = EQC_CV(pc);
+                            constexpr int l2 = K::PL.l2[p];
+                            if constexpr (l2 > 0) {
+#pragma unroll
+                                for (int m = 0; m < 2 * l2 + 1; ++m) gY[l2 * l2 - 1 + m] += gp[R::gy_off(p) + 1 + m];
+                            }
+                        });
+                    }
+                    sh_grad_contract<K::LSH>(ok, ux, uy, uz, il, gY, d0, d1v, d2v);
+                }
+            } else {
+                for (int n = 0; n < NB; ++n) bb[n] = gb[n] = 0.f;
+                sFac[t] = 0.f;
+                sGud[t] = 0.f;
             }
+        }
+        __syncthreads();
+        // 2. z1 = b . W1, h1 = silu(z1)
+        float dz1[4][4];
+        {
+            float z[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) z[i][c] = 0.f;
+            for (int n = 0; n < NB; ++n) {
+                const float4 w = *reinterpret_cast<const float4*>(sW1 + n * kH + 4 * tj);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float a = sB[(4 * tk + i) * kMaxBasis + n];
+                    z[i][0] = fmaf(a, w.x, z[i][0]);
+                    z[i][1] = fmaf(a, w.y, z[i][1]);
+                    z[i][2] = fmaf(a, w.z, z[i][2]);
+                    z[i][3] = fmaf(a, w.w, z[i][3]);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float h[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    h[c] = silu(z[i][c]);
+                    dz1[i][c] = silu_grad(z[i][c]);
+                }
+                *reinterpret_cast<float4*>(sH1 + (4 * tk + i) * kEpiLd + 4 * tj) = make_float4(h[0], h[1], h[2], h[3]);
+            }
+        }
+        __syncthreads();
+        // 3. z2 = h1 . W2, g_z2 = Gd fac silu'(z2)
+        {
+            float z[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) z[i][c] = 0.f;
+#pragma unroll 4
+            for (int q = 0; q < kH; q += 4) {
+                float4 a[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(sH1 + (4 * tk + i) * kEpiLd + q);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const float4 w = *reinterpret_cast<const float4*>(sW2 + (q + qq) * kH + 4 * tj);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float av = qq == 0 ? a[i].x : qq == 1 ? a[i].y : qq == 2 ? a[i].z : a[i].w;
+                        z[i][0] = fmaf(av, w.x, z[i][0]);
+                        z[i][1] = fmaf(av, w.y, z[i][1]);
+                        z[i][2] = fmaf(av, w.z, z[i][2]);
+                        z[i][3] = fmaf(av, w.w, z[i][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int k = kbase + 4 * tk + i;
+                float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (k < E)
+                    for (int q = 0; q < SG; ++q) {
+                        const float4 v = __ldcs(reinterpret_cast<const float4*>(gd_part + ((size_t)q * E + k) * kH + 4 * tj));
+                        g.x += v.x;
+                        g.y += v.y;
+                        g.z += v.z;
+                        g.w += v.w;
+                    }
+                const float f = sFac[4 * tk + i];
+                *reinterpret_cast<float4*>(sG2 + (4 * tk + i) * kEpiLd + 4 * tj) =
+                    make_float4(g.x * f * silu_grad(z[i][0]), g.y * f * silu_grad(z[i][1]),
+                                g.z * f * silu_grad(z[i][2]), g.w * f * silu_grad(z[i][3]));
+            }
+        }
+        __syncthreads();
+        // 4. g_z1 = (g_z2 . W2^T) silu'(z1);  g_W2 += h1^T g_z2
+        {
+            float z[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) z[i][c] = 0.f;
+#pragma unroll 4
+            for (int j = 0; j < kH; j += 4) {
+                float4 a[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(sG2 + (4 * tk + i) * kEpiLd + j);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const float4 w = *reinterpret_cast<const float4*>(sW2T + (j + jj) * kH + 4 * tj);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float av = jj == 0 ? a[i].x : jj == 1 ? a[i].y : jj == 2 ? a[i].z : a[i].w;
+                        z[i][0] = fmaf(av, w.x, z[i][0]);
+                        z[i][1] = fmaf(av, w.y, z[i][1]);
+                        z[i][2] = fmaf(av, w.z, z[i][2]);
+                        z[i][3] = fmaf(av, w.w, z[i][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4*>(sG1 + (4 * tk + i) * kEpiLd + 4 * tj) =
+                    make_float4(z[i][0] * dz1[i][0], z[i][1] * dz1[i][1], z[i][2] * dz1[i][2], z[i][3] * dz1[i][3]);
+#pragma unroll 4
+            for (int k = 0; k < kEpiTile; ++k) {
+                const float4 h = *reinterpret_cast<const float4*>(sH1 + k * kEpiLd + 4 * tk);
+                const float4 g = *reinterpret_cast<const float4*>(sG2 + k * kEpiLd + 4 * tj);
+                const float hv[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    gw2[i][0] = fmaf(hv[i], g.x, gw2[i][0]);
+                    gw2[i][1] = fmaf(hv[i], g.y, gw2[i][1]);
+                    gw2[i][2] = fmaf(hv[i], g.z, gw2[i][2]);
+                    gw2[i][3] = fmaf(hv[i], g.w, gw2[i][3]);
+                }
+            }
+        }
+        __syncthreads();
+        // 5. g_b . b'(d) per position (4 threads each, fixed order);  g_W1 += b^T g_z1
+        {
+            const int kk = t >> 2, ng = t & 3;
+            float part = 0.f;
+            for (int n = ng; n < NB; n += 4) {
+                float sdot = 0.f;
+#pragma unroll 4
+                for (int j = 0; j < kH; j += 4) {
+                    const float4 g = *reinterpret_cast<const float4*>(sG1 + kk * kEpiLd + j);
+                    const float4 w = *reinterpret_cast<const float4*>(sW1 + n * kH + j);
+                    sdot = fmaf(g.x, w.x, fmaf(g.y, w.y, fmaf(g.z, w.z, fmaf(g.w, w.w, sdot))));
+                }
+                part = fmaf(sdot, sGb[kk * kMaxBasis + n], part);
+            }
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            if (ng == 0) sGdl[kk] = part;
+            const int jc = t & 63, n0 = t >> 6;
+#pragma unroll 4
+            for (int k = 0; k < kEpiTile; ++k) {
+                const float g = sG1[k * kEpiLd + jc];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (n0 + 4 * i < NB) gw1[i] = fmaf(sB[k * kMaxBasis + n0 + 4 * i], g, gw1[i]);
+            }
+        }
+        __syncthreads();
+        // 6. dr
+        if (t < kEpiTile && e >= 0) {
+            const float gd_len = sGdl[t] + sGud[t];
             if (d > 1e-12f) {
                 d0 = fmaf(gd_len, rx * inv_d, d0);
                 d1v = fmaf(gd_len, ry * inv_d, d1v);
@@ -811,31 +1000,16 @@ __global__ void __launch_bounds__(kEpiThreads)
             dr[(size_t)e * 3] = d0;
             dr[(size_t)e * 3 + 1] = d1v;
             dr[(size_t)e * 3 + 2] = d2v;
-        } else {
-            for (int j = 0; j < kH; ++j) {
-                h1[j] = 0.f;
-                g2[j] = 0.f;
-                z1[j] = 0.f;
-            }
-            for (int n = 0; n < NB; ++n) bb[n] = 0.f;
-        }
-        __syncthreads();
-        // this chunk's terms of the weight gradients, edges in order
-        for (int i = 0; i < kEpiThreads; ++i) {
-            const float h = sh1[i * kEpiStride + t];
-            const float* gz2 = sg2 + i * kEpiStride;
-#pragma unroll
-            for (int j = 0; j < kH; ++j) acc2[j] = fmaf(h, gz2[j], acc2[j]);
-            const float gz1 = sz1[i * kEpiStride + t];
-            const float* bi = sb + i * (kMaxBasis + 1);
-            for (int n = 0; n < NB; ++n) acc1[n] = fmaf(bi[n], gz1, acc1[n]);
         }
     }
-    float* o2 = gw2_part + ((size_t)blockIdx.x * kH + t) * kH;
+    float* o2 = gw2_part + (size_t)blockIdx.x * kH * kH;
 #pragma unroll
-    for (int j = 0; j < kH; ++j) o2[j] = acc2[j];
+    for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4*>(o2 + (4 * tk + i) * kH + 4 * tj) = make_float4(gw2[i][0], gw2[i][1], gw2[i][2], gw2[i][3]);
     float* o1 = gw1_part + (size_t)blockIdx.x * kMaxBasis * kH;
-    for (int n = 0; n < NB; ++n) o1[n * kH + t] = acc1[n];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if ((t >> 6) + 4 * i < NB) o1[((t >> 6) + 4 * i) * kH + (t & 63)] = gw1[i];
 }
 
 // out[i] = sum_{b < nb} part[b * stride + i], in order of b (i < n).

@@ -43,17 +43,15 @@ constexpr int kGroupTiles = 3;
 constexpr int kPathWarps = 12;
 constexpr int kMmaWarp = 12, kXWarp = 13;
 constexpr int kConvThreads = 14 * 32;
-constexpr int kXSlots = 16;        // sender-row ring depth (positions in flight)
-constexpr int kBatch = 16;         // edges per harmonics / coupling batch of a path warp
+constexpr int kXBatches = 2;       // sender-row batches in flight (double buffer)
+constexpr int kBatch = 16;         // edges per harmonics / coupling batch of a path warp (at most)
 constexpr int kTmemCols = 512;     // 2 buffers x 3 tiles x 64 columns, rounded to a power of two
 
 struct RadFwdParams {
     const float* x;      // [N][D_in][C]
-    const float* r;      // [E][3]
     const int* ptr;      // recv_ptr [N+1]
-    const int* perm;     // recv_perm [E]
-    const int* senders;  // [E]
-    const float* uscale; // [E] by receiver position
+    const float4* rec;   // [E] (r_e, uscale) by receiver position
+    const int2* ids;     // [E] (sender, receiver) by receiver position
     float* y_pp;         // [N][D_pp][C] per-path output blocks
     int N, C, E;
     int nodes_per_cta;
@@ -73,22 +71,27 @@ constexpr int max_coupling_floats() {
 // Shared-memory layout of the fused forward (bytes; tiles 1024-aligned).
 template <class K>
 struct RadFwdSmem {
+    static constexpr int BT = K::D_IN >= 16 ? 8 : kBatch;                 // positions per batch
     static constexpr int A_TILE = kRowTile * kTileRowBytes;                 // 16 KB: 128 rows of W3^T
     static constexpr int H_TILE = kEdgeTile * kTileRowBytes;                // 8 KB: 64 rows of h2
     static constexpr int W3_OFF = 0;                                        // [tile][hi, lo]
     static constexpr int H_OFF = W3_OFF + kGroupTiles * 2 * A_TILE;         // [stage][hi, lo]
     static constexpr int X_SLOT = K::D_IN * kSlice * 4;
-    static constexpr int X_OFF = H_OFF + 2 * 2 * H_TILE;
+    static constexpr int X_OFF = H_OFF + 2 * 2 * H_TILE;                    // [batch buffer][BT slots]
     static constexpr int NA = max_coupling_floats<K>();
-    static constexpr int CPL_OFF = X_OFF + kXSlots * X_SLOT;
-    static constexpr int CPL_WARP = kBatch * NA * 4;
-    static constexpr int US_OFF = CPL_OFF + kPathWarps * CPL_WARP;          // per path warp: batch uscale
-    static constexpr int BAR_OFF = US_OFF + kPathWarps * kBatch * 4;
-    // barriers: w3, h_full[2], h_empty[2], t_full[2], t_empty[2], x_full[R], x_empty[R]
-    static constexpr int NBAR = 9 + 2 * kXSlots;
+    static constexpr int CPL_OFF = X_OFF + kXBatches * BT * X_SLOT;
+    static constexpr int CPL_WARP = BT * NA * 4;
+    static constexpr int WS_OFF = CPL_OFF + kPathWarps * CPL_WARP;          // per path warp: w of the batch
+    static constexpr int WS_WARP = BT * 32 * 4;
+    static constexpr int US_OFF = WS_OFF + kPathWarps * WS_WARP;            // per path warp: uscale of the batch
+    static constexpr int BAR_OFF = US_OFF + kPathWarps * BT * 4;
+    // barriers: w3, h_full[2], h_empty[2], t_full[2], t_empty[2], x_full[2], x_empty[2]
+    static constexpr int NBAR = 9 + 2 * kXBatches;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int END = MISC_OFF + 16;
     static constexpr int BYTES = END + 1024;                               // + alignment slack
+    static_assert(BYTES <= 227 * 1024, "fused radial forward: shared memory");
+    static_assert(kEdgeTile % BT == 0, "batches tile the MMA tile");
 };
 
 // Per-edge coupling of one path: Arow[m3 * d1 + m1] = sum_m2 C_p[m1,m2,m3] Y[l2^2 + m2].
@@ -123,17 +126,39 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
     return __uint_as_float(v);
 }
 
+// BT consecutive columns of this warp's lanes into `dst` [BT][32] (shared).
+template <int BT>
+__device__ __forceinline__ void tmem_stash(uint32_t taddr, float* dst, int lane) {
+    if constexpr (BT == 16) {
+        float v[16];
+        tmem_ld16(taddr, v);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) dst[t * 32 + lane] = v[t];
+    } else if constexpr (BT == 8) {
+        float v[8];
+        tmem_ld8(taddr, v);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) dst[t * 32 + lane] = v[t];
+    } else {
+#pragma unroll
+        for (int t = 0; t < BT; ++t) dst[t * 32 + lane] = tmem_ld1(taddr + (uint32_t)t);
+    }
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // The path warp's whole run for path P_ (compile-time), over the CTA's
-// positions [k0, k1) and receivers [n0, n1).
+// positions [k0, k1) and receivers [n0, n1), batch by batch: one wait for
+// the batch's sender rows, one tensor-memory read of its w, per-edge
+// records read in position order (prefetched one batch ahead).
 template <class K, int P_>
 __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* base, uint32_t tmem, int warp,
                                               int lane, int n0, int n1, int k0, int k1, int c0,
                                               volatile int* abort_flag) {
     using S = RadFwdSmem<K>;
+    constexpr int BT = S::BT;
     constexpr int l1 = K::PL.l1[P_], l2 = K::PL.l2[P_], l3 = K::PL.l3[P_];
     constexpr int d1 = 2 * l1 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o3 = K::PL.o3[P_];
     constexpr int NA = S::NA;
@@ -141,9 +166,10 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
     uint64_t* t_full = bars + 5;
     uint64_t* t_empty = bars + 7;
     uint64_t* x_full = bars + 9;
-    uint64_t* x_empty = bars + 9 + kXSlots;
+    uint64_t* x_empty = bars + 9 + kXBatches;
     float* cpl = reinterpret_cast<float*>(base + S::CPL_OFF + warp * S::CPL_WARP);
-    float* us_s = reinterpret_cast<float*>(base + S::US_OFF) + warp * kBatch;
+    float* ws = reinterpret_cast<float*>(base + S::WS_OFF + warp * S::WS_WARP);
+    float* us_s = reinterpret_cast<float*>(base + S::US_OFF) + warp * BT;
     const float* xring = reinterpret_cast<const float*>(base + S::X_OFF);
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tile_col = (uint32_t)(64 * (warp >> 2));
@@ -153,8 +179,7 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
 #pragma unroll
     for (int m = 0; m < d3; ++m) acc[m] = 0.f;
     int cur = n0;
-    int cur_end = prm.ptr[n0 + 1];
-    auto flush = [&]() {
+    auto flush = [&]() {   // the current receiver's block, then reset
         float* yo = prm.y_pp + ((size_t)cur * K::D_OUT + o3) * C + c0 + lane;
 #pragma unroll
         for (int m = 0; m < d3; ++m) {
@@ -162,6 +187,13 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
             acc[m] = 0.f;
         }
     };
+    // the next batch's records (lane t < BT holds position kb + t), prefetched
+    float4 nrec = make_float4(0.f, 0.f, 0.f, 0.f);
+    int nown = 0;
+    if (lane < BT && k0 + lane < k1) {
+        nrec = prm.rec[k0 + lane];
+        nown = prm.ids[k0 + lane].y;
+    }
 
     const int ntiles = (k1 - k0 + kEdgeTile - 1) / kEdgeTile;
     for (int j = 0; j < ntiles; ++j) {
@@ -175,43 +207,45 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
         const uint32_t tcol = tmem + lane_base + (uint32_t)(s * kGroupTiles * kEdgeTile) + tile_col;
         const int kt = k0 + j * kEdgeTile;
         const int kt_end = min(k1, kt + kEdgeTile);
-        for (int kb = kt; kb < kt_end; kb += kBatch) {
-            const int nb = min(kBatch, kt_end - kb);
+        for (int kb = kt; kb < kt_end; kb += BT) {
+            const int nb = min(BT, kt_end - kb);
+            const int b = (kb - k0) / BT;
+            const float4 rc = nrec;
+            const int own = nown;
+            if (lane < BT && kb + BT + lane < k1) {   // prefetch the batch after this one
+                nrec = prm.rec[kb + BT + lane];
+                nown = prm.ids[kb + BT + lane].y;
+            }
             if (lane < nb) {
-                const int k = kb + lane;
-                const int e = prm.perm[k];
-                float ux, uy, uz, il;
-                const bool ok = unit_dir(prm.r[(size_t)e * 3], prm.r[(size_t)e * 3 + 1], prm.r[(size_t)e * 3 + 2],
-                                         ux, uy, uz, il);
                 if constexpr (l2 > 0) {
+                    float ux, uy, uz, il;
+                    const bool ok = unit_dir(rc.x, rc.y, rc.z, ux, uy, uz, il);
                     float Y[K::D_SH];
                     sh_eval<K::LSH>(ok, ux, uy, uz, Y);
                     path_coupling<l1, l2, l3>(Y, cpl + lane * NA);
                 }
-                us_s[lane] = prm.uscale[k];
+                us_s[lane] = rc.w;
             }
+            tmem_stash<BT>(tcol + (uint32_t)(kb - kt), ws, lane);
             __syncwarp();
+            if (!mbar_wait(&x_full[b % kXBatches], (uint32_t)(b / kXBatches) & 1u) ||
+                __any_sync(0xffffffffu, *abort_flag)) {
+                if (lane == 0) atomicOr(prm.status, 4u);
+                *abort_flag = 1;
+                return;
+            }
+            const float* xb = xring + (b % kXBatches) * BT * (S::X_SLOT / 4) + o1 * kSlice + lane;
             for (int t = 0; t < nb; ++t) {
-                const int k = kb + t;
-                while (k >= cur_end) {   // the current receiver's edges are done (empty ones too)
+                const int own_t = __shfl_sync(0xffffffffu, own, t);
+                while (cur < own_t) {   // receivers done (and any without edges)
                     flush();
                     ++cur;
-                    cur_end = prm.ptr[cur + 1];
                 }
-                const float w = tmem_ld1(tcol + (uint32_t)(k - kt)) * us_s[t];
-                const int q = k - k0;
-                const int slot = q % kXSlots;
-                if (!mbar_wait(&x_full[slot], (uint32_t)(q / kXSlots) & 1u) || __any_sync(0xffffffffu, *abort_flag)) {
-                    if (lane == 0) atomicOr(prm.status, 4u);
-                    *abort_flag = 1;
-                    return;
-                }
-                const float* xs = xring + slot * (S::X_SLOT / 4) + o1 * kSlice + lane;
+                const float w = ws[t * 32 + lane] * us_s[t];
+                const float* xs = xb + t * (S::X_SLOT / 4);
                 float xv[d1];
 #pragma unroll
                 for (int m = 0; m < d1; ++m) xv[m] = xs[m * kSlice];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&x_empty[slot]);
                 if constexpr (l2 == 0) {
 #pragma unroll
                     for (int m = 0; m < d1; ++m) acc[m] = fmaf(w, xv[m], acc[m]);
@@ -227,6 +261,7 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
                 }
             }
             __syncwarp();
+            if (lane == 0) mbar_arrive(&x_empty[b % kXBatches]);
         }
         tc_fence_before();
         __syncwarp();
@@ -244,6 +279,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
                            const __grid_constant__ CUtensorMap map_a_lo, const __grid_constant__ CUtensorMap map_h_hi,
                            const __grid_constant__ CUtensorMap map_h_lo, const __grid_constant__ CUtensorMap map_x) {
     using S = RadFwdSmem<K>;
+    constexpr int BT = S::BT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + S::BAR_OFF);
@@ -253,7 +289,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     uint64_t* t_full = bars + 5;
     uint64_t* t_empty = bars + 7;
     uint64_t* x_full = bars + 9;
-    uint64_t* x_empty = bars + 9 + kXSlots;
+    uint64_t* x_empty = bars + 9 + kXBatches;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + S::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base + S::MISC_OFF + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -275,7 +311,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
             mbar_init(&t_full[s], 1);
             mbar_init(&t_empty[s], gp);
         }
-        for (int q = 0; q < kXSlots; ++q) {
+        for (int q = 0; q < kXBatches; ++q) {
             mbar_init(&x_full[q], 1);
             mbar_init(&x_empty[q], gp);
         }
@@ -307,22 +343,27 @@ __global__ void __launch_bounds__(kConvThreads, 1)
                     tma_2d(dst, &map_a_hi, 0, row, w3_full);
                     tma_2d(dst + S::A_TILE, &map_a_lo, 0, row, w3_full);
                 }
+            int h_issued = 0, h_waited = 0, committed = 0;
             auto load_h = [&](int j) {
                 const int s = j & 1;
                 uint8_t* dst = base + S::H_OFF + s * 2 * S::H_TILE;
                 mbar_expect_tx(&h_full[s], 2 * S::H_TILE);
                 tma_2d(dst, &map_h_hi, 0, k0 + j * kEdgeTile, &h_full[s]);
                 tma_2d(dst + S::H_TILE, &map_h_lo, 0, k0 + j * kEdgeTile, &h_full[s]);
+                h_issued = j + 1;
             };
             load_h(0);
             if (ntiles > 1) load_h(1);
-            bool ok = mbar_wait_one(w3_full, 0);
+            const bool w3_ok = mbar_wait_one(w3_full, 0);
+            bool ok = w3_ok;
             constexpr uint32_t id = idesc_f16(kRowTile, kEdgeTile);
             for (int j = 0; j < ntiles && ok; ++j) {
                 const int s = j & 1;
-                ok = mbar_wait_one(&h_full[s], (uint32_t)(j >> 1) & 1u) &&
-                     (j < 2 || mbar_wait_one(&t_empty[s], (uint32_t)((j >> 1) - 1) & 1u));
-                if (!ok || *abort_flag) break;
+                ok = mbar_wait_one(&h_full[s], (uint32_t)(j >> 1) & 1u);
+                if (!ok) break;
+                h_waited = j + 1;
+                ok = (j < 2 || mbar_wait_one(&t_empty[s], (uint32_t)((j >> 1) - 1) & 1u)) && !*abort_flag;
+                if (!ok) break;
                 tc_fence_after();
                 const uint8_t* hs = base + S::H_OFF + s * 2 * S::H_TILE;
                 const uint64_t dbh = sw128_desc(smem_addr(hs)), dbl = sw128_desc(smem_addr(hs + S::H_TILE));
@@ -340,6 +381,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
                 }
                 umma_commit(&t_full[s]);
                 umma_commit(&h_empty[s]);
+                committed = j + 1;
                 if (j + 2 < ntiles) {
                     ok = mbar_wait_one(&h_empty[s], (uint32_t)(j >> 1) & 1u);
                     if (ok) load_h(j + 2);
@@ -348,28 +390,50 @@ __global__ void __launch_bounds__(kConvThreads, 1)
             if (!ok) {
                 atomicOr(prm.status, 4u);
                 *abort_flag = 1;
+                // let the copies and products in flight land before the CTA lets go of its memory
+                if (!w3_ok) mbar_wait_one(w3_full, 0);
+                for (int u = h_waited; u < h_issued; ++u) mbar_wait_one(&h_full[u & 1], (uint32_t)(u >> 1) & 1u);
+                for (int u = committed > 2 ? committed - 2 : 0; u < committed; ++u)
+                    mbar_wait_one(&t_full[u & 1], (uint32_t)(u >> 1) & 1u);
             }
         }
     } else if (warp == kXWarp) {
-        if (lane == 0) {
-            for (int k = k0; k < k1; ++k) {
-                const int q = k - k0, slot = q % kXSlots;
-                if (q >= kXSlots && !mbar_wait_one(&x_empty[slot], (uint32_t)(q / kXSlots - 1) & 1u)) {
-                    atomicOr(prm.status, 4u);
-                    *abort_flag = 1;
-                    break;
-                }
-                if (*abort_flag) break;
-                int sidx = prm.senders[prm.perm[k]];
+        // sender rows, batch by batch: one barrier per batch of BT positions;
+        // lane t copies the row of position kb + t
+        const int nbatch = (k1 - k0 + BT - 1) / BT;
+        int issued = 0;
+        for (int b = 0; b < nbatch; ++b) {
+            const int kb = k0 + b * BT;
+            const int nb = min(BT, k1 - kb);
+            int sidx = 0;
+            if (lane < nb) {
+                sidx = prm.ids[kb + lane].x;
                 if ((unsigned)sidx >= (unsigned)prm.N) {   // out of range: flagged, read as node 0
                     atomicOr(prm.status, 1u);
                     sidx = 0;
                 }
-                mbar_expect_tx(&x_full[slot], S::X_SLOT);
-                tma_rows(base + S::X_OFF + slot * S::X_SLOT, &map_x, c0, sidx, &x_full[slot],
-                         policy_evict_last());
             }
+            int go = 1;
+            if (lane == 0) {
+                if (b >= kXBatches &&
+                    !mbar_wait_one(&x_empty[b % kXBatches], (uint32_t)(b / kXBatches - 1) & 1u)) {
+                    atomicOr(prm.status, 4u);
+                    *abort_flag = 1;
+                }
+                go = *abort_flag ? 0 : 1;
+                if (go) mbar_expect_tx(&x_full[b % kXBatches], nb * S::X_SLOT);
+            }
+            if (!__shfl_sync(0xffffffffu, go, 0)) break;
+            if (lane < nb)
+                tma_rows(base + S::X_OFF + ((b % kXBatches) * BT + lane) * S::X_SLOT, &map_x, c0, sidx,
+                         &x_full[b % kXBatches], policy_evict_last());
+            issued = b + 1;
         }
+        // the last fills of each buffer land before the CTA lets go of its memory
+        // (immediate when their consumers already saw them)
+        if (lane == 0)
+            for (int b = issued > kXBatches ? issued - kXBatches : 0; b < issued; ++b)
+                mbar_wait_one(&x_full[b % kXBatches], (uint32_t)(b / kXBatches) & 1u);
     }
     tc_fence_before();
     __syncthreads();

@@ -14,6 +14,7 @@ struct RadFwdArgs {
     const int* recv_ptr;
     const int* recv_perm;
     const int* senders;
+    const int* receivers;
     const float* W1;         // [NB][64]
     const float* W2;         // [64][64]
     const float* W3;         // [64][P*C]
@@ -33,6 +34,7 @@ struct RadBwdArgs {
     const float* gy;         // [N][D_out][C] of the plan (summed or per-path layout)
     const int* send_ptr;
     const int* send_perm;
+    const int* senders;
     const int* receivers;
     const float* W1;
     const float* W2;

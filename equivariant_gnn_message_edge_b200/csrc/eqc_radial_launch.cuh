@@ -39,7 +39,8 @@ struct RadLaunch {
         float* y_pp = a.per_path ? a.y
                                  : reinterpret_cast<float*>(static_cast<char*>(a.workspace) +
                                                             up256(workspace_bytes(a.E, PC)));
-        cudaError_t err = prepare(ws, a.r, a.recv_perm, a.E, a.W1, a.W2, a.W3, a.NB, a.rc, PC, st);
+        cudaError_t err = prepare(ws, a.r, a.recv_perm, a.E, a.W1, a.W2, a.W3, a.NB, a.rc, PC, st, nullptr,
+                                  a.senders, a.receivers);
         if (err != cudaSuccess) return err;
         if (a.E > 0) {
             CUtensorMap ma_hi, ma_lo, mh_hi, mh_lo, mx;
@@ -63,8 +64,7 @@ struct RadLaunch {
             const long long want = 148LL * 4;
             int npc = (int)(((long long)a.N * slices * groups + want - 1) / want);
             if (npc < 1) npc = 1;
-            RadFwdParams prm{a.x, a.r, a.recv_ptr, a.recv_perm, a.senders, ws.uscale, y_pp, a.N, a.C, a.E, npc,
-                             a.status};
+            RadFwdParams prm{a.x, a.recv_ptr, ws.rec, ws.ids, y_pp, a.N, a.C, a.E, npc, a.status};
             const dim3 grid((a.N + npc - 1) / npc, slices, groups);
             radial_conv_fwd_kernel<KP><<<grid, kConvThreads, S::BYTES, st>>>(prm, ma_hi, ma_lo, mh_hi, mh_lo, mx);
             count_launch();
@@ -93,7 +93,7 @@ struct RadLaunch {
         return npc < 1 ? 1 : npc;
     }
     static constexpr int kEpiChunks = 16;   // 64-position chunks per epilogue CTA
-    static int epi_ctas(int E) { return (E + kEpiThreads * kEpiChunks - 1) / (kEpiThreads * kEpiChunks); }
+    static int epi_ctas(int E) { return (E + kEpiTile * kEpiChunks - 1) / (kEpiTile * kEpiChunks); }
 
     struct BwdWs {
         Workspace rad;
@@ -152,7 +152,8 @@ struct RadLaunch {
         radial_absmax_kernel<<<296, 256, 0, st>>>(a.gy, ng4, sbits + 2);
         count_launch();
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
-        err = prepare(b.rad, a.r, a.send_perm, a.E, a.W1, a.W2, a.W3, a.NB, a.rc, PC, st, sbits + 3);
+        err = prepare(b.rad, a.r, a.send_perm, a.E, a.W1, a.W2, a.W3, a.NB, a.rc, PC, st, sbits + 3, a.receivers,
+                      a.senders);
         if (err != cudaSuccess) return err;
         CUtensorMap ma_hi, ma_lo, mh_hi, mh_lo, mg;
         if (!encode_f16_rows(&ma_hi, b.rad.a_hi, (uint64_t)PC, 32) ||
@@ -175,8 +176,8 @@ struct RadLaunch {
         }
         const int slices = bwd_slices(a.C), groups = bwd_groups(), npc = bwd_nodes_per_cta(a.N, a.C);
         const int ranges = (a.N + npc - 1) / npc;
-        RadBwdParams prm{a.x, a.r, a.gy, a.send_ptr, a.send_perm, a.receivers, b.rad.uscale, scal, b.dx_pp,
-                         b.gy_part, b.gd_part, b.gw3_part, a.N, a.C, a.E, npc, a.status};
+        RadBwdParams prm{a.x, a.gy, a.send_ptr, b.rad.rec, b.rad.ids, scal, b.dx_pp, b.gy_part, b.gd_part,
+                         b.gw3_part, a.N, a.C, a.E, npc, a.status};
         radial_conv_bwd_kernel<KG><<<dim3(ranges, slices, groups), kBwdThreads, S::BYTES, st>>>(prm, ma_hi, ma_lo,
                                                                                                mh_hi, mh_lo, mg);
         count_launch();
