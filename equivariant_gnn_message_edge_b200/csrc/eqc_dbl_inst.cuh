@@ -59,7 +59,7 @@ struct DblLaunch {
 };
 
 #ifndef EQC_DBL_VEC
-#define EQC_DBL_VEC 1   // channel width of every instance (0: 1 where an l = 3 block is present, else 2)
+#define EQC_DBL_VEC 0   // channel width of every instance (0: 1 where an l = 3 block is present, else 2)
 #endif
 constexpr int dbl_vec(int lin, int lsh, int lout) { return EQC_DBL_VEC > 0 ? EQC_DBL_VEC : mode_vec(lin, lsh, lout); }
 
