@@ -136,6 +136,57 @@ def time_node_product(W, Nn, dev, stream, reps, reduce=lambda t: t):
                      "and read, dw written"}
 
 
+def time_symmetric_contraction(W, Nn, dev, stream, reps, reduce=lambda t: t, n_species=4):
+    """Median device time and GB/s of the symmetric contraction of correlation
+    order 2 (A (x) A with per-species weights; irreps of the workload's
+    features in and out) on Nn nodes, forward and backward; bytes = each
+    tensor read or written once per kernel (A, species, W1, W2, B; A,
+    species, W1, W2, gB, dA, the weight-gradient partials written and read,
+    dW1, dW2)."""
+    import torch
+
+    from equivariant_gnn_message_edge_b200 import binding as B
+    from equivariant_gnn_message_edge_b200.conv import SymmetricContraction
+    op = SymmetricContraction(W.irreps_in, W.irreps_out, W.C, n_species)
+    gen = torch.Generator(device=dev).manual_seed(wl.SEED_X + 11)
+    C, P, S = W.C, op.P, n_species
+    with torch.cuda.stream(stream):
+        A = torch.randn((Nn, op.D_A, C), generator=gen, device=dev)
+        z = torch.randint(0, S, (Nn,), generator=gen, device=dev, dtype=torch.int32)
+        W1 = torch.randn((S, op.L1N, C), generator=gen, device=dev)
+        W2 = torch.randn((S, P, C), generator=gen, device=dev)
+        gB = torch.randn((Nn, op.D_out, C), generator=gen, device=dev)
+        out = torch.empty_like(gB)
+        dA, dW1, dW2 = torch.empty_like(A), torch.empty_like(W1), torch.empty_like(W2)
+        nws = B.eqconv_symmetric_contraction_workspace_bytes(op.plan, Nn)
+        ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev)
+    h = stream.cuda_stream
+    fe = []
+    for _ in range(reps + 1):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        B.eqconv_symmetric_contraction(op.plan, Nn, A, z, W1, W2, out, h)
+        ev[1].record(stream)
+        B.eqconv_symmetric_contraction_backward(op.plan, Nn, A, z, W1, W2, gB, dA, dW1, dW2, ws, nws, h)
+        ev[2].record(stream)
+        fe.append(ev)
+    stream.synchronize()
+    assert B.eqconv_get_device_error(op.plan, h) == B.EQCONV_OK
+    f_ms = reduce(statistics.median([e[0].elapsed_time(e[1]) for e in fe[1:]]))     # max over ranks
+    b_ms = reduce(statistics.median([e[1].elapsed_time(e[2]) for e in fe[1:]]))
+    row = 4 * C * Nn
+    wbytes = 4 * S * (op.L1N + P) * C
+    fb = row * (op.D_A + op.D_out) + 4 * Nn + wbytes
+    bb = row * (2 * op.D_A + op.D_out) + 4 * Nn + 2 * wbytes + 2 * nws
+    peak = measured_peak()[0]
+    return {"nodes": Nn, "species": S, "paths": P, "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
+            "fwd_gbps": round(fb / (f_ms * 1e-3) / 1e9, 1), "bwd_gbps": round(bb / (b_ms * 1e-3) / 1e9, 1),
+            "fwd_frac_of_measured_hbm": round(fb / (f_ms * 1e-3) / 1e9 / peak, 4),
+            "bwd_frac_of_measured_hbm": round(bb / (b_ms * 1e-3) / 1e9 / peak, 4),
+            "bytes": "fwd: A, species, W1, W2 read, B written; bwd: A, species, W1, W2, gB read, dA written, "
+                     "weight-gradient partials written and read, dW1, dW2 written"}
+
+
 def device_inputs(W, D_in, D_out, P, dev, seed_offset=0):
     """Graph of workload W from the seeded NumPy generators; features, weights
     and output gradients drawn on the device by a seeded torch generator with
@@ -706,6 +757,11 @@ def run_native(args, rank, world, local_rank):
     if not W.all_parity and not args.no_node_product:
         nprod = time_node_product(W, 4 * N, dev, stream, max(3, args.steps // 2),
                                   lambda t: reduce_max(t, world, dev))
+    # symmetric contraction of correlation order 2 (4 species) on 4N nodes
+    symc = None
+    if not W.all_parity and not W.per_path and not args.no_node_product:
+        symc = time_symmetric_contraction(W, 4 * N, dev, stream, max(3, args.steps // 2),
+                                          lambda t: reduce_max(t, world, dev))
 
     # End to end through the public API with host buffers (pinned), copies
     # timed: every step uploads its inputs and downloads its results.  Steps
@@ -822,6 +878,7 @@ def run_native(args, rank, world, local_rank):
                          "algorithmic_bytes": bc["fwd"]},
         "double_backward": dbl,
         "node_product": nprod,
+        "symmetric_contraction": symc,
         "workloads": legs,
         "gpu_launches": int(launches),
         "clocks": clk.summary((w0, w1)),
