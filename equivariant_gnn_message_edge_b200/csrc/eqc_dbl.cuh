@@ -59,7 +59,7 @@ struct DblParams {
 
 template <class K>
 struct DblShape {
-    static constexpr int CH = K::NA_PAD > 128 ? 4 : 8;        // edges per coupling batch
+    static constexpr int CH = 8;   // edges whose harmonics (Y, rho) one batch evaluates
 };
 
 template <int V>
@@ -93,16 +93,20 @@ __device__ __forceinline__ void load_rows(float (&d)[R][V], const float* base, i
     }
 }
 
-// acc[o3] += w_p (A_p(Y) a + A_p(rho) x) + b_p A_p(Y) x for every path.
+// acc[o3] += w_p (A_p(Y) a + A_p(rho) x) + b_p A_p(Y) x for every path, in
+// the form that needs no coupling matrices: with s1 = w a + b x and s2 = w x
+// (per channel), acc[m3] += sum_{m1, m2} C_p[m1, m2, m3] (Y[m2] s1[m1] +
+// rho[m2] s2[m1]), one product per nonzero (m1, m2) row of C_p.  Yrow holds
+// the edge's Y, then rho.
 template <class K>
-__device__ __forceinline__ void dbl_recv_edge(const float* AY, const float* AR, const float (&xv)[K::D_IN][K::VEC],
+__device__ __forceinline__ void dbl_recv_edge(const float* Yrow, const float (&xv)[K::D_IN][K::VEC],
                                               const float (&av)[K::D_IN][K::VEC], const float (&wv)[K::NP][K::VEC],
                                               const float (&bv)[K::NP][K::VEC], float (&acc)[K::D_OUT][K::VEC]) {
     constexpr int V = K::VEC;
     static_for<K::NP>([&](auto pc) {
         constexpr int p = EQC_CV(pc);
         constexpr int l1 = K::PL.l1[p], l2 = K::PL.l2[p], l3 = K::PL.l3[p];
-        constexpr int d1 = 2 * l1 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o3 = K::PL.o3[p];
+        constexpr int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o2 = l2 * l2, o3 = K::PL.o3[p];
         if constexpr (l2 == 0) {       // A(Y) = I, A(rho) = 0
 #pragma unroll
             for (int m = 0; m < d1; ++m)
@@ -110,28 +114,32 @@ __device__ __forceinline__ void dbl_recv_edge(const float* AY, const float* AR, 
                 for (int v = 0; v < V; ++v)
                     acc[o3 + m][v] = fmaf(wv[p][v], av[o1 + m][v], fmaf(bv[p][v], xv[o1 + m][v], acc[o3 + m][v]));
         } else {
-            constexpr int n4 = (d1 * d3 + 3) / 4;
-            constexpr int aoff = K::AO.off[p];
-            float ay[n4 * 4], ar[n4 * 4];
-            load_A<n4>(AY + aoff, ay);
-            load_A<n4>(AR + aoff, ar);
+            float s1[d1][V], s2[d1][V];
 #pragma unroll
-            for (int m3 = 0; m3 < d3; ++m3) {
-                float ta[V], tx[V], tr[V];
+            for (int m = 0; m < d1; ++m)
 #pragma unroll
-                for (int v = 0; v < V; ++v) ta[v] = tx[v] = tr[v] = 0.f;
+                for (int v = 0; v < V; ++v) {
+                    s1[m][v] = fmaf(wv[p][v], av[o1 + m][v], bv[p][v] * xv[o1 + m][v]);
+                    s2[m][v] = wv[p][v] * xv[o1 + m][v];
+                }
+            static_for<d2>([&](auto m2c) {
+                constexpr int m2 = EQC_CV(m2c);
+                const float y2 = Yrow[o2 + m2], r2 = Yrow[K::D_SH + o2 + m2];
+                static_for<d1>([&](auto m1c) {
+                    constexpr int m1 = EQC_CV(m1c);
+                    if constexpr (cg_row_nonzero<l1, l2, l3>(m1, m2)) {
 #pragma unroll
-                for (int m1 = 0; m1 < d1; ++m1)
-#pragma unroll
-                    for (int v = 0; v < V; ++v) {
-                        ta[v] = fmaf(ay[m3 * d1 + m1], av[o1 + m1][v], ta[v]);
-                        tx[v] = fmaf(ay[m3 * d1 + m1], xv[o1 + m1][v], tx[v]);
-                        tr[v] = fmaf(ar[m3 * d1 + m1], xv[o1 + m1][v], tr[v]);
+                        for (int v = 0; v < V; ++v) {
+                            const float z = fmaf(y2, s1[m1][v], r2 * s2[m1][v]);
+                            static_for<d3>([&](auto m3c) {
+                                constexpr int m3 = EQC_CV(m3c);
+                                constexpr double c = RealCG<l1, l2, l3>::t.v[m1][m2][m3];
+                                if constexpr (c != 0.0) acc[o3 + m3][v] = fmaf((float)c, z, acc[o3 + m3][v]);
+                            });
+                        }
                     }
-#pragma unroll
-                for (int v = 0; v < V; ++v)
-                    acc[o3 + m3][v] = fmaf(wv[p][v], ta[v] + tr[v], fmaf(bv[p][v], tx[v], acc[o3 + m3][v]));
-            }
+                });
+            });
         }
     });
 }
@@ -229,7 +237,7 @@ struct DblRing {
     static constexpr uint32_t STAGE_BYTES = SF * 4;
     static constexpr int ST_F = S * SF;
     static constexpr int BAR_F = up32(4 * S);
-    static constexpr int ROW_F = up32(RECV ? 2 * CH * K::NA_PAD : CH * 2 * K::D_SH);
+    static constexpr int ROW_F = up32(CH * 2 * K::D_SH);   // per edge of a batch: Y, then rho
     static constexpr int TOTAL_F = ST_F + BAR_F + ROW_F;
     static constexpr int WARPS = best_warps(TOTAL_F * 4);
     static constexpr int SMEM = WARPS * TOTAL_F * 4;
@@ -266,8 +274,7 @@ __global__ void __launch_bounds__(DblRing<K, true>::WARPS * 32)
     if (node >= prm.N) return;
     float* stages = reinterpret_cast<float*>(smem4) + warp * L::TOTAL_F;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + L::ST_F);
-    float* AY = stages + L::ST_F + L::BAR_F;
-    float* AR = AY + CH * K::NA_PAD;
+    float* Ys = stages + L::ST_F + L::BAR_F;   // rows of 2 D_SH: Y then rho
     const int C = prm.C;
     const int c0 = blockIdx.y * K::TILE_C, cl = lane * V;
     const bool on = c0 + cl < C;
@@ -309,8 +316,12 @@ __global__ void __launch_bounds__(DblRing<K, true>::WARPS * 32)
                 float Y[K::D_SH], rho[K::D_SH];
                 sh_eval<K::LSH>(ok, ux, uy, uz, Y);
                 sh_jvp<K::LSH>(rx, ry, rz, qe[0], qe[1], qe[2], rho);
-                compute_A<K>(Y, AY + (lane - b0) * K::NA_PAD);
-                compute_A<K>(rho, AR + (lane - b0) * K::NA_PAD);
+                float* yrow = Ys + (lane - b0) * 2 * K::D_SH;
+#pragma unroll
+                for (int q = 0; q < K::D_SH; ++q) {
+                    yrow[q] = Y[q];
+                    yrow[K::D_SH + q] = rho[q];
+                }
             }
             __syncwarp();
             for (int t = b0; t < b0 + nb; ++t) {
@@ -334,7 +345,7 @@ __global__ void __launch_bounds__(DblRing<K, true>::WARPS * 32)
                     lds_vec<V>(xv[d], st + (2 * K::NP + d) * K::TILE_C + cl);
                     lds_vec<V>(av[d], st + (2 * K::NP + K::D_IN + d) * K::TILE_C + cl);
                 }
-                dbl_recv_edge<K>(AY + (t - b0) * K::NA_PAD, AR + (t - b0) * K::NA_PAD, xv, av, wv, bv, acc);
+                dbl_recv_edge<K>(Ys + (t - b0) * 2 * K::D_SH, xv, av, wv, bv, acc);
                 __syncwarp();
                 if (t + S < n) {
                     const int e = __shfl_sync(0xffffffffu, my_e, t + S), o = __shfl_sync(0xffffffffu, my_s, t + S);
