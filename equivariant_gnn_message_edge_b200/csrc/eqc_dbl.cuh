@@ -20,11 +20,13 @@
 //
 // Three launches, all deterministic (no atomics):
 //   * receiver pass (receiver CSR): g_gy, one warp per receiver and channel
-//     tile, sums in registers;
+//     tile, sums in registers; it contracts C directly with
+//     Y (w a + b x) + rho (w x), one product per nonzero CG row;
 //   * sender pass (sender CSR): g_x in registers, g_w stored per edge, the
-//     per-tile partials of gYv and gY1 (warp butterfly, fixed order) to a
-//     workspace [E][T][2G]; it contracts through h = C.gy and needs only
-//     each edge's Y and rho, not its coupling matrices;
+//     per-tile partials of gYv and gY1 (one warp transpose-sum, fixed order)
+//     to a workspace [E][T][2G]; it contracts through h = C.gy;
+//   so neither pass builds coupling matrices: each needs only the edge's Y
+//   and rho;
 //   * r epilogue (one thread per edge): sums the tiles in order and applies
 //     the gradient and the Hessian-vector product of the harmonics.
 // Each warp stages its edges' rows through a ring of shared-memory stages
@@ -93,34 +95,78 @@ __device__ __forceinline__ void load_rows(float (&d)[R][V], const float* base, i
     }
 }
 
+// This lane's V channels of stage row `row` (zeros when the lane is past C;
+// the predicate also keeps the compiler from hoisting every row load of the
+// edge into registers).
+template <class K>
+__device__ __forceinline__ void stage_row(float (&d)[K::VEC], const float* st, int row, int cl, bool rd) {
+    if (rd) {
+        lds_vec<K::VEC>(d, st + row * K::TILE_C + cl);
+    } else {
+#pragma unroll
+        for (int v = 0; v < K::VEC; ++v) d[v] = 0.f;
+    }
+}
+
 // acc[o3] += w_p (A_p(Y) a + A_p(rho) x) + b_p A_p(Y) x for every path, in
 // the form that needs no coupling matrices: with s1 = w a + b x and s2 = w x
 // (per channel), acc[m3] += sum_{m1, m2} C_p[m1, m2, m3] (Y[m2] s1[m1] +
 // rho[m2] s2[m1]), one product per nonzero (m1, m2) row of C_p.  Yrow holds
 // the edge's Y, then rho.
+// The edge's rows: read from its stage path by path (PRE = false: fewer live
+// registers, for wide channel tiles) or taken from arrays the caller loaded
+// up front (PRE = true).
 template <class K>
-__device__ __forceinline__ void dbl_recv_edge(const float* Yrow, const float (&xv)[K::D_IN][K::VEC],
-                                              const float (&av)[K::D_IN][K::VEC], const float (&wv)[K::NP][K::VEC],
-                                              const float (&bv)[K::NP][K::VEC], float (&acc)[K::D_OUT][K::VEC]) {
+struct DblRecvRows {
+    float w[K::NP][K::VEC], b[K::NP][K::VEC], x[K::D_IN][K::VEC], a[K::D_IN][K::VEC];
+};
+template <class K, bool PRE>
+__device__ __forceinline__ void dbl_recv_edge(const float* st, int cl, bool rd, const DblRecvRows<K>& pre,
+                                              const float* Yrow, float (&acc)[K::D_OUT][K::VEC]) {
     constexpr int V = K::VEC;
     static_for<K::NP>([&](auto pc) {
         constexpr int p = EQC_CV(pc);
         constexpr int l1 = K::PL.l1[p], l2 = K::PL.l2[p], l3 = K::PL.l3[p];
         constexpr int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1, o1 = l1 * l1, o2 = l2 * l2, o3 = K::PL.o3[p];
+        float w[V], b[V];
+        float xv[d1][V], av[d1][V];
+        if constexpr (PRE) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                w[v] = pre.w[p][v];
+                b[v] = pre.b[p][v];
+            }
+#pragma unroll
+            for (int m = 0; m < d1; ++m)
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    xv[m][v] = pre.x[o1 + m][v];
+                    av[m][v] = pre.a[o1 + m][v];
+                }
+        } else {
+            constexpr int XR = 2 * K::NP + o1, AR = 2 * K::NP + K::D_IN + o1;   // stage rows of x_l1, a_l1
+            stage_row<K>(w, st, p, cl, rd);
+            stage_row<K>(b, st, K::NP + p, cl, rd);
+#pragma unroll
+            for (int m = 0; m < d1; ++m) {
+                stage_row<K>(xv[m], st, XR + m, cl, rd);
+                stage_row<K>(av[m], st, AR + m, cl, rd);
+            }
+        }
         if constexpr (l2 == 0) {       // A(Y) = I, A(rho) = 0
 #pragma unroll
             for (int m = 0; m < d1; ++m)
 #pragma unroll
                 for (int v = 0; v < V; ++v)
-                    acc[o3 + m][v] = fmaf(wv[p][v], av[o1 + m][v], fmaf(bv[p][v], xv[o1 + m][v], acc[o3 + m][v]));
+                    acc[o3 + m][v] = fmaf(w[v], av[m][v], fmaf(b[v], xv[m][v], acc[o3 + m][v]));
         } else {
             float s1[d1][V], s2[d1][V];
 #pragma unroll
             for (int m = 0; m < d1; ++m)
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    s1[m][v] = fmaf(wv[p][v], av[o1 + m][v], bv[p][v] * xv[o1 + m][v]);
-                    s2[m][v] = wv[p][v] * xv[o1 + m][v];
+                    s1[m][v] = fmaf(w[v], av[m][v], b[v] * xv[m][v]);
+                    s2[m][v] = w[v] * xv[m][v];
                 }
             static_for<d2>([&](auto m2c) {
                 constexpr int m2 = EQC_CV(m2c);
@@ -150,11 +196,16 @@ __device__ __forceinline__ void dbl_recv_edge(const float* Yrow, const float (&x
 // contractions: A_p(Y)^T gy = sum_m2 Y[m2] h, A_p(rho)^T gy = sum_m2 rho[m2] h,
 // G_p(a, gy) = sum_m1 a[m1] h and G_p(x, gy) = sum_m1 x[m1] h; so the pass
 // needs only each edge's Y and rho, not its coupling matrices.
+// The edge's rows (w, b, gy): from its stage path by path, or (PRE) from
+// arrays the caller loaded up front.
 template <class K>
-__device__ __forceinline__ void dbl_send_edge(const float* Yrow, const float (&xv)[K::D_IN][K::VEC],
+struct DblSendRows {
+    float w[K::NP][K::VEC], b[K::NP][K::VEC], g[K::D_OUT][K::VEC];
+};
+template <class K, bool PRE>
+__device__ __forceinline__ void dbl_send_edge(const float* st, int cl, bool rd, const DblSendRows<K>& pre,
+                                              const float* Yrow, const float (&xv)[K::D_IN][K::VEC],
                                               const float (&av)[K::D_IN][K::VEC],
-                                              const float (&gv)[K::D_OUT][K::VEC],
-                                              const float (&wv)[K::NP][K::VEC], const float (&bv)[K::NP][K::VEC],
                                               float (&gacc)[K::D_IN][K::VEC], float* gw_row, int C, bool on,
                                               float* gYv, float* gY1) {
     constexpr int V = K::VEC;
@@ -163,13 +214,30 @@ __device__ __forceinline__ void dbl_send_edge(const float* Yrow, const float (&x
         constexpr int l1 = K::PL.l1[p], l2 = K::PL.l2[p], l3 = K::PL.l3[p];
         constexpr int d1 = 2 * l1 + 1, d2 = 2 * l2 + 1, d3 = 2 * l3 + 1;
         constexpr int o1 = l1 * l1, o2 = l2 * l2, o3 = K::PL.o3[p];
+        float wv[V], bv[V], gv[d3][V];
+        if constexpr (PRE) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                wv[v] = pre.w[p][v];
+                bv[v] = pre.b[p][v];
+            }
+#pragma unroll
+            for (int m = 0; m < d3; ++m)
+#pragma unroll
+                for (int v = 0; v < V; ++v) gv[m][v] = pre.g[o3 + m][v];
+        } else {
+            stage_row<K>(wv, st, p, cl, rd);
+            stage_row<K>(bv, st, K::NP + p, cl, rd);
+#pragma unroll
+            for (int m = 0; m < d3; ++m) stage_row<K>(gv[m], st, 2 * K::NP + o3 + m, cl, rd);
+        }
         float uY[d1][V], uR[d1][V];
         if constexpr (l2 == 0) {       // A(Y) = I, A(rho) = 0
 #pragma unroll
             for (int m = 0; m < d1; ++m)
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    uY[m][v] = gv[o3 + m][v];
+                    uY[m][v] = gv[m][v];
                     uR[m][v] = 0.f;
                 }
         } else {
@@ -192,7 +260,7 @@ __device__ __forceinline__ void dbl_send_edge(const float* Yrow, const float (&x
                             static_for<d3>([&](auto m3c) {
                                 constexpr int m3 = EQC_CV(m3c);
                                 constexpr double c = RealCG<l1, l2, l3>::t.v[m1][m2][m3];
-                                if constexpr (c != 0.0) h = fmaf((float)c, gv[o3 + m3][v], h);
+                                if constexpr (c != 0.0) h = fmaf((float)c, gv[m3][v], h);
                             });
                             uY[m1][v] = fmaf(y2, h, uY[m1][v]);
                             uR[m1][v] = fmaf(r2, h, uR[m1][v]);
@@ -203,8 +271,8 @@ __device__ __forceinline__ void dbl_send_edge(const float* Yrow, const float (&x
                 });
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    gYv[o2 + m2 - 1] = fmaf(wv[p][v], Ga[v], fmaf(bv[p][v], Gx[v], gYv[o2 + m2 - 1]));
-                    gY1[o2 + m2 - 1] = fmaf(wv[p][v], Gx[v], gY1[o2 + m2 - 1]);
+                    gYv[o2 + m2 - 1] = fmaf(wv[v], Ga[v], fmaf(bv[v], Gx[v], gYv[o2 + m2 - 1]));
+                    gY1[o2 + m2 - 1] = fmaf(wv[v], Gx[v], gY1[o2 + m2 - 1]);
                 }
             });
         }
@@ -215,7 +283,7 @@ __device__ __forceinline__ void dbl_send_edge(const float* Yrow, const float (&x
         for (int m1 = 0; m1 < d1; ++m1)
 #pragma unroll
             for (int v = 0; v < V; ++v) {
-                gacc[o1 + m1][v] = fmaf(bv[p][v], uY[m1][v], fmaf(wv[p][v], uR[m1][v], gacc[o1 + m1][v]));
+                gacc[o1 + m1][v] = fmaf(bv[v], uY[m1][v], fmaf(wv[v], uR[m1][v], gacc[o1 + m1][v]));
                 gw[v] = fmaf(av[o1 + m1][v], uY[m1][v], fmaf(xv[o1 + m1][v], uR[m1][v], gw[v]));
             }
         if (on) st_stream<V>(gw_row + (size_t)p * C, gw);
@@ -224,9 +292,8 @@ __device__ __forceinline__ void dbl_send_edge(const float* Yrow, const float (&x
 
 // Per-warp shared memory of the two passes (floats, regions 128-byte
 // aligned): [stages: S x ROWS x TILE_C] [mbarriers] [per-batch rows].
-// Receiver pass: rows w (NP), b (NP), x (D_IN), a (D_IN) per stage and the
-// batch's coupling matrices A(Y), A(rho); sender pass: rows w, b, gy (D_OUT)
-// and the batch's harmonics Y, rho.
+// Receiver pass: rows w (NP), b (NP), x (D_IN), a (D_IN) per stage; sender
+// pass: rows w, b, gy (D_OUT); both keep the batch's harmonics Y, rho.
 template <class K, bool RECV>
 struct DblRing {
     static constexpr int S = K::STAGES;
@@ -334,18 +401,22 @@ __global__ void __launch_bounds__(DblRing<K, true>::WARPS * 32)
                     fill_to = g + (uint32_t)min(n, t + S);
                     break;
                 }
-                float wv[K::NP][V], bv[K::NP][V], xv[K::D_IN][V], av[K::D_IN][V];
+                // 32-channel tiles take every row up front, wider ones read them on demand
+                constexpr bool PRE = V == 1;
+                DblRecvRows<K> rows;
+                if constexpr (PRE) {
 #pragma unroll
-                for (int p = 0; p < K::NP; ++p) {
-                    lds_vec<V>(wv[p], st + p * K::TILE_C + cl);
-                    lds_vec<V>(bv[p], st + (K::NP + p) * K::TILE_C + cl);
-                }
+                    for (int p = 0; p < K::NP; ++p) {
+                        lds_vec<V>(rows.w[p], st + p * K::TILE_C + cl);
+                        lds_vec<V>(rows.b[p], st + (K::NP + p) * K::TILE_C + cl);
+                    }
 #pragma unroll
-                for (int d = 0; d < K::D_IN; ++d) {
-                    lds_vec<V>(xv[d], st + (2 * K::NP + d) * K::TILE_C + cl);
-                    lds_vec<V>(av[d], st + (2 * K::NP + K::D_IN + d) * K::TILE_C + cl);
+                    for (int d = 0; d < K::D_IN; ++d) {
+                        lds_vec<V>(rows.x[d], st + (2 * K::NP + d) * K::TILE_C + cl);
+                        lds_vec<V>(rows.a[d], st + (2 * K::NP + K::D_IN + d) * K::TILE_C + cl);
+                    }
                 }
-                dbl_recv_edge<K>(Ys + (t - b0) * 2 * K::D_SH, xv, av, wv, bv, acc);
+                dbl_recv_edge<K, PRE>(st, cl, on, rows, Ys + (t - b0) * 2 * K::D_SH, acc);
                 __syncwarp();
                 if (t + S < n) {
                     const int e = __shfl_sync(0xffffffffu, my_e, t + S), o = __shfl_sync(0xffffffffu, my_s, t + S);
@@ -447,19 +518,22 @@ __global__ void __launch_bounds__(DblRing<K, false>::WARPS * 32)
                     break;
                 }
                 const int e = __shfl_sync(0xffffffffu, my_e, t);
-                float wv[K::NP][V], bv[K::NP][V], gv[K::D_OUT][V];
-#pragma unroll
-                for (int p = 0; p < K::NP; ++p) {
-                    lds_vec<V>(wv[p], st + p * K::TILE_C + cl);
-                    lds_vec<V>(bv[p], st + (K::NP + p) * K::TILE_C + cl);
-                }
-#pragma unroll
-                for (int d = 0; d < K::D_OUT; ++d) lds_vec<V>(gv[d], st + (2 * K::NP + d) * K::TILE_C + cl);
                 float gYv[G], gY1[G];
 #pragma unroll
                 for (int q = 0; q < G; ++q) gYv[q] = gY1[q] = 0.f;
-                dbl_send_edge<K>(Ys + (t - b0) * 2 * K::D_SH, xv, av, gv, wv, bv, gacc,
-                                 prm.g_w + (size_t)e * K::NP * C + c0 + cl, C, on, gYv, gY1);
+                constexpr bool PRE = V == 1;
+                DblSendRows<K> rows;
+                if constexpr (PRE) {
+#pragma unroll
+                    for (int p = 0; p < K::NP; ++p) {
+                        lds_vec<V>(rows.w[p], st + p * K::TILE_C + cl);
+                        lds_vec<V>(rows.b[p], st + (K::NP + p) * K::TILE_C + cl);
+                    }
+#pragma unroll
+                    for (int d = 0; d < K::D_OUT; ++d) lds_vec<V>(rows.g[d], st + (2 * K::NP + d) * K::TILE_C + cl);
+                }
+                dbl_send_edge<K, PRE>(st, cl, on, rows, Ys + (t - b0) * 2 * K::D_SH, xv, av, gacc,
+                                      prm.g_w + (size_t)e * K::NP * C + c0 + cl, C, on, gYv, gY1);
                 __syncwarp();
                 if (t + S < n) {
                     const int e2 = __shfl_sync(0xffffffffu, my_e, t + S), o2 = __shfl_sync(0xffffffffu, my_i, t + S);

@@ -83,8 +83,12 @@ struct RadFwdSmem {
     static constexpr int CPL_WARP = BT * NA * 4;
     static constexpr int WS_OFF = CPL_OFF + kPathWarps * CPL_WARP;          // per path warp: w of the batch
     static constexpr int WS_WARP = BT * 32 * 4;
-    static constexpr int US_OFF = WS_OFF + kPathWarps * WS_WARP;            // per path warp: uscale of the batch
-    static constexpr int BAR_OFF = US_OFF + kPathWarps * BT * 4;
+    // per batch buffer, written by the sender-row warp: each position's harmonics
+    // (rows of YS floats), edge factor and receiver
+    static constexpr int YS = (K::D_SH + 3) & ~3;
+    static constexpr int YB_OFF = WS_OFF + kPathWarps * WS_WARP;
+    static constexpr int YB_BATCH = BT * (YS + 4) * 4;                      // Y row + (us, own) per position
+    static constexpr int BAR_OFF = YB_OFF + kXBatches * YB_BATCH;
     // barriers: w3, h_full[2], h_empty[2], t_full[2], t_empty[2], x_full[2], x_empty[2]
     static constexpr int NBAR = 9 + 2 * kXBatches;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
@@ -169,7 +173,6 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
     uint64_t* x_empty = bars + 9 + kXBatches;
     float* cpl = reinterpret_cast<float*>(base + S::CPL_OFF + warp * S::CPL_WARP);
     float* ws = reinterpret_cast<float*>(base + S::WS_OFF + warp * S::WS_WARP);
-    float* us_s = reinterpret_cast<float*>(base + S::US_OFF) + warp * BT;
     const float* xring = reinterpret_cast<const float*>(base + S::X_OFF);
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tile_col = (uint32_t)(64 * (warp >> 2));
@@ -187,13 +190,6 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
             acc[m] = 0.f;
         }
     };
-    // the next batch's records (lane t < BT holds position kb + t), prefetched
-    float4 nrec = make_float4(0.f, 0.f, 0.f, 0.f);
-    int nown = 0;
-    if (lane < BT && k0 + lane < k1) {
-        nrec = prm.rec[k0 + lane];
-        nown = prm.ids[k0 + lane].y;
-    }
 
     const int ntiles = (k1 - k0 + kEdgeTile - 1) / kEdgeTile;
     for (int j = 0; j < ntiles; ++j) {
@@ -210,38 +206,28 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
         for (int kb = kt; kb < kt_end; kb += BT) {
             const int nb = min(BT, kt_end - kb);
             const int b = (kb - k0) / BT;
-            const float4 rc = nrec;
-            const int own = nown;
-            if (lane < BT && kb + BT + lane < k1) {   // prefetch the batch after this one
-                nrec = prm.rec[kb + BT + lane];
-                nown = prm.ids[kb + BT + lane].y;
-            }
-            if (lane < nb) {
-                if constexpr (l2 > 0) {
-                    float ux, uy, uz, il;
-                    const bool ok = unit_dir(rc.x, rc.y, rc.z, ux, uy, uz, il);
-                    float Y[K::D_SH];
-                    sh_eval<K::LSH>(ok, ux, uy, uz, Y);
-                    path_coupling<l1, l2, l3>(Y, cpl + lane * NA);
-                }
-                us_s[lane] = rc.w;
-            }
             tmem_stash<BT>(tcol + (uint32_t)(kb - kt), ws, lane);
-            __syncwarp();
+            // the batch's sender rows, harmonics, edge factors and receivers
             if (!mbar_wait(&x_full[b % kXBatches], (uint32_t)(b / kXBatches) & 1u) ||
                 __any_sync(0xffffffffu, *abort_flag)) {
                 if (lane == 0) atomicOr(prm.status, 4u);
                 *abort_flag = 1;
                 return;
             }
+            const float* yb = reinterpret_cast<const float*>(base + S::YB_OFF + (b % kXBatches) * S::YB_BATCH);
+            if constexpr (l2 > 0) {
+                if (lane < nb) path_coupling<l1, l2, l3>(yb + lane * (S::YS + 4), cpl + lane * NA);
+                __syncwarp();
+            }
             const float* xb = xring + (b % kXBatches) * BT * (S::X_SLOT / 4) + o1 * kSlice + lane;
             for (int t = 0; t < nb; ++t) {
-                const int own_t = __shfl_sync(0xffffffffu, own, t);
+                const float* yt = yb + t * (S::YS + 4);
+                const int own_t = __float_as_int(yt[S::YS + 1]);
                 while (cur < own_t) {   // receivers done (and any without edges)
                     flush();
                     ++cur;
                 }
-                const float w = ws[t * 32 + lane] * us_s[t];
+                const float w = ws[t * 32 + lane] * yt[S::YS];
                 const float* xs = xb + t * (S::X_SLOT / 4);
                 float xv[d1];
 #pragma unroll
@@ -312,7 +298,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
             mbar_init(&t_empty[s], gp);
         }
         for (int q = 0; q < kXBatches; ++q) {
-            mbar_init(&x_full[q], 1);
+            mbar_init(&x_full[q], 2);   // the copies' bytes + the batch info
             mbar_init(&x_empty[q], gp);
         }
         *abort_flag = 0;
@@ -405,9 +391,13 @@ __global__ void __launch_bounds__(kConvThreads, 1)
         for (int b = 0; b < nbatch; ++b) {
             const int kb = k0 + b * BT;
             const int nb = min(BT, k1 - kb);
-            int sidx = 0;
+            int sidx = 0, own = 0;
+            float4 rc = make_float4(0.f, 0.f, 0.f, 0.f);
             if (lane < nb) {
-                sidx = prm.ids[kb + lane].x;
+                const int2 id = prm.ids[kb + lane];
+                rc = prm.rec[kb + lane];
+                sidx = id.x;
+                own = id.y;
                 if ((unsigned)sidx >= (unsigned)prm.N) {   // out of range: flagged, read as node 0
                     atomicOr(prm.status, 1u);
                     sidx = 0;
@@ -428,6 +418,21 @@ __global__ void __launch_bounds__(kConvThreads, 1)
                 tma_rows(base + S::X_OFF + ((b % kXBatches) * BT + lane) * S::X_SLOT, &map_x, c0, sidx,
                          &x_full[b % kXBatches], policy_evict_last());
             issued = b + 1;
+            // each position's harmonics, edge factor and receiver for the path warps
+            if (lane < nb) {
+                float* yrow = reinterpret_cast<float*>(base + S::YB_OFF + (b % kXBatches) * S::YB_BATCH) +
+                              lane * (S::YS + 4);
+                float ux, uy, uz, il;
+                const bool okd = unit_dir(rc.x, rc.y, rc.z, ux, uy, uz, il);
+                float Y[K::D_SH];
+                sh_eval<K::LSH>(okd, ux, uy, uz, Y);
+#pragma unroll
+                for (int q = 0; q < K::D_SH; ++q) yrow[q] = Y[q];
+                yrow[S::YS] = rc.w;
+                yrow[S::YS + 1] = __int_as_float(own);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&x_full[b % kXBatches]);
         }
         // the last fills of each buffer land before the CTA lets go of its memory
         // (immediate when their consumers already saw them)
