@@ -46,16 +46,16 @@
 namespace eqc {
 namespace radial {
 
-constexpr int kBwdGroupPaths = 8;
-constexpr int kBwdGroupTiles = 2;
-constexpr int kBwdPathWarps = 8;
-constexpr int kBwdReaderWarp0 = 8;
-constexpr int kBwdMmaWarp = 12, kBwdGyWarp = 13;
-constexpr int kBwdThreads = 14 * 32;
+constexpr int kBwdGroupPaths = 4;
+constexpr int kBwdGroupTiles = 1;
+constexpr int kBwdPathWarps = 4;
+constexpr int kBwdMmaWarp = 4, kBwdGyWarp = 5;
+constexpr int kBwdThreads = 6 * 32;
+constexpr int kBwdTmemCols = 256;   // two CTAs share an SM's tensor memory
 constexpr int kGySlots = 16;
-constexpr uint32_t kColW = 0;       // w: [2 buffers][2 tiles][64]
-constexpr uint32_t kColGW = 256;    // g_W3 accumulators: [2 tiles][64 (k)]
-constexpr uint32_t kColGD = 384;    // Gd: 64 columns (M = 64 layout)
+constexpr uint32_t kColW = 0;       // w: [2 buffers][1 tile][64]
+constexpr uint32_t kColGW = 128;    // g_W3 accumulators: [1 tile][64 (k)]
+constexpr uint32_t kColGD = 192;    // Gd: 64 columns (M = 64 layout)
 
 struct RadBwdParams {
     const float* x;        // [N][D_in][C]
@@ -125,9 +125,11 @@ struct RadBwdSmem {
     // per path warp, for a batch of up to 8 positions: harmonics rows + edge factor, and w
     static constexpr int Y_WARP8 = 8 * (YS + 4) * 4 + 8 * 32 * 4;
     // gy ring: batches of BT receiver rows, as many (2 .. 4) as fit beside the rest;
-    // BT = 8 where two batches of 8 fit, else 4, else 2
+    // BT = 8 where two batches of 8 fit, else 4, else 2.  Two CTAs share an SM
+    // (113 KB each) when a ring of two 4-position batches fits, else one (227 KB).
     static constexpr int FIXED = GY_OFF + kBwdPathWarps * Y_WARP8 + (14 + 2 * 4) * 8 + 16 + 1024;
-    static constexpr int FIT = (227 * 1024 - FIXED) / GY_SLOT;
+    static constexpr bool TWO = (113 * 1024 - FIXED) / GY_SLOT >= 8;
+    static constexpr int FIT = ((TWO ? 113 : 227) * 1024 - FIXED) / GY_SLOT;
     static constexpr int BT = FIT >= 16 ? 8 : (FIT >= 8 ? 4 : 2);
     static constexpr int GYB = FIT / BT >= 4 ? 4 : FIT / BT;
     static constexpr int Y_WARP = BT * (YS + 4) * 4;
@@ -142,7 +144,7 @@ struct RadBwdSmem {
     static constexpr int END = MISC_OFF + 16;
     static constexpr int BYTES = END + 1024;
     static_assert(GYB >= 2, "fused radial backward: room for two gy batches");
-    static_assert(BYTES <= 227 * 1024, "fused radial backward: shared memory");
+    static_assert(BYTES <= (TWO ? 113 : 227) * 1024, "fused radial backward: shared memory");
     static_assert(kEdgeTile % BT == 0, "batches tile the MMA tile");
 };
 
@@ -152,10 +154,50 @@ __device__ __forceinline__ uint32_t g_chunk_offset(int row, int q8) {
     return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((q8 ^ (row & 7)) << 4));
 }
 
+// Gd of the tile starting at position kt (tensor-memory lanes 16 q .. +15 of
+// subpartition q hold rows k = 16 q + lane of the M = 64 layout) to the
+// workspace, positions below k1.
+__device__ __noinline__ void copy_gd(const RadBwdParams& prm, uint32_t tmem, int q, int lane, int kt, int k1,
+                                        int sg) {
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    float* dst = prm.gd_part + ((size_t)sg * prm.E + kt) * kH + 16 * q + lane;
+    const int n = k1 - kt;   // positions of the tile below k1
+#pragma unroll 1
+    for (int c16 = 0; c16 < kEdgeTile; c16 += 16) {
+        float v[16];
+        tmem_ld16(tmem + lane_base + kColGD + (uint32_t)c16, v);
+        if (lane < 16) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (c16 + i < n) dst[(size_t)(c16 + i) * kH] = v[i];
+        }
+    }
+}
+
+// The CTA's g_W3 rows of path p (row 32 q + lane = channel c0 + lane) out of
+// tensor memory, or zeros for a range without edges.
+__device__ __noinline__ void copy_gw3(const RadBwdParams& prm, uint32_t tmem, int q, int lane, int p, int NP,
+                                         int c0, bool zero) {
+    float* dst = prm.gw3_part + ((size_t)blockIdx.x * NP * prm.C + (size_t)p * prm.C + c0 + lane) * kH;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+#pragma unroll 1
+    for (int c16 = 0; c16 < kH; c16 += 16) {
+        float v[16];
+        if (zero) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        } else {
+            tmem_ld16(tmem + lane_base + kColGW + (uint32_t)c16, v);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) *reinterpret_cast<float4*>(dst + c16 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    }
+}
+
 template <class K, int P_>
 __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* base, uint32_t tmem, int warp,
                                               int lane, int n0, int n1, int k0, int k1, int c0, int slice,
-                                              int slices, int gexp, volatile int* abort_flag) {
+                                              int slices, int sg, int gexp, volatile int* abort_flag) {
     using S = RadBwdSmem<K>;
     using R = BwdRows<K>;
     constexpr int BT = S::BT;
@@ -170,6 +212,9 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
     uint64_t* t_empty = bars + 7;
     uint64_t* g_full = bars + 9;
     uint64_t* g_empty = bars + 10;
+    uint64_t* gd_full = bars + 11;
+    uint64_t* gd_empty = bars + 12;
+    uint64_t* gw_full = bars + 13;
     uint64_t* gy_full = bars + 14;
     uint64_t* gy_empty = bars + 14 + S::GYB;
     float* ys = reinterpret_cast<float*>(base + S::Y_OFF + warp * S::Y_WARP);     // [BT][YS + 4]
@@ -239,10 +284,18 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
             return;
         }
         tc_fence_after();
-        // the G tile of the previous tile has been read by the MMAs
-        if (j > 0 && !mbar_wait(g_empty, (uint32_t)(j - 1) & 1u)) {
-            abort_now();
-            return;
+        // the G tile of the previous tile has been read by the MMAs; that
+        // tile's Gd (same products) goes to the workspace
+        if (j > 0) {
+            if (!mbar_wait(g_empty, (uint32_t)(j - 1) & 1u)) {
+                abort_now();
+                return;
+            }
+            tc_fence_after();
+            copy_gd(prm, tmem, warp & 3, lane, k0 + (j - 1) * kEdgeTile, k1, sg);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(gd_empty);
         }
         const uint32_t tcol = tmem + lane_base + kColW + (uint32_t)((s * kBwdGroupTiles + tile) * kEdgeTile);
         const int kt = k0 + j * kEdgeTile;
@@ -373,13 +426,28 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
             mbar_arrive(&t_empty[s]);
         }
     }
+    // the last tile's Gd, then the CTA's g_W3 rows of this path
+    if (ntiles > 0) {
+        if (!mbar_wait(gd_full, (uint32_t)(ntiles - 1) & 1u) || !mbar_wait(gw_full, 0u)) {
+            abort_now();
+            return;
+        }
+        tc_fence_after();
+        copy_gd(prm, tmem, warp & 3, lane, k0 + (ntiles - 1) * kEdgeTile, k1, sg);
+        copy_gw3(prm, tmem, warp & 3, lane, P_, K::NP, c0, false);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(gd_empty);
+    } else {
+        copy_gw3(prm, tmem, warp & 3, lane, P_, K::NP, c0, true);
+    }
     // the last sender and any empty ones after it
     while (cur + 1 < n1) next_sender();
     flush();
 }
 
 template <class K>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 2)
     radial_conv_bwd_kernel(const RadBwdParams prm, const __grid_constant__ CUtensorMap map_a_hi,
                            const __grid_constant__ CUtensorMap map_a_lo, const __grid_constant__ CUtensorMap map_h_hi,
                            const __grid_constant__ CUtensorMap map_h_lo, const __grid_constant__ CUtensorMap map_gy) {
@@ -439,7 +507,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int i = tid; i < kBwdGroupTiles * 2 * S::G_TILE / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(base + S::G_OFF)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async();
-    if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+    if (warp == 0) tmem_alloc(tmem_slot, kBwdTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -451,67 +519,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             static_for<K::NP>([&](auto pc) {
                 if (EQC_CV(pc) == p)
                     path_warp_bwd<K, EQC_CV(pc)>(prm, base, tmem, warp, lane, n0, n1, k0, k1, c0, slice, slices,
-                                                 gexp, abort_flag);
+                                                 sg, gexp, abort_flag);
             });
-        }
-    } else if (warp < kBwdMmaWarp) {
-        // reader warp of subpartition q: Gd rows k = 16 q + lane (lanes < 16) of every tile
-        const int q = warp & 3;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        for (int j = 0; j < ntiles; ++j) {
-            if (!mbar_wait(gd_full, (uint32_t)j & 1u) || __any_sync(0xffffffffu, *abort_flag)) {
-                if (lane == 0) atomicOr(prm.status, 4u);
-                *abort_flag = 1;
-                break;
-            }
-            tc_fence_after();
-            const int kt = k0 + j * kEdgeTile;
-            const int kk = 16 * q + lane;
-#pragma unroll
-            for (int c16 = 0; c16 < kEdgeTile; c16 += 16) {
-                float v[16];
-                tmem_ld16(tmem + lane_base + kColGD + (uint32_t)c16, v);
-                if (lane < 16) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int k = kt + c16 + i;
-                        if (k < k1) prm.gd_part[((size_t)sg * prm.E + k) * kH + kk] = v[i];
-                    }
+        } else {
+            // a subpartition without a path still copies its rows of every tile's Gd
+            for (int j = 0; j < ntiles; ++j) {
+                if (!mbar_wait(gd_full, (uint32_t)j & 1u) || __any_sync(0xffffffffu, *abort_flag)) {
+                    if (lane == 0) atomicOr(prm.status, 4u);
+                    *abort_flag = 1;
+                    break;
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(gd_empty);
-        }
-        // the CTA's g_W3 rows: tile t, row 32 q + lane = (path g0 + 4 t + q, channel c0 + lane);
-        // a range without edges contributes zeros
-        if (ntiles == 0) {
-            for (int t = 0; t < gtiles; ++t) {
-                const int p = g0 + 4 * t + q;
-                if (p < K::NP) {
-                    float* dst = prm.gw3_part +
-                                 ((size_t)blockIdx.x * K::NP * prm.C + (size_t)p * prm.C + c0 + lane) * kH;
-                    for (int i = 0; i < kH; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-        } else if (!*abort_flag) {
-            if (mbar_wait(gw_full, 0)) {
                 tc_fence_after();
-                for (int t = 0; t < gtiles; ++t) {
-                    const int p = g0 + 4 * t + q;
-                    float* dst = prm.gw3_part + ((size_t)blockIdx.x * K::NP * prm.C + (size_t)p * prm.C + c0 + lane) * kH;
-#pragma unroll
-                    for (int c16 = 0; c16 < kH; c16 += 16) {
-                        float v[16];
-                        tmem_ld16(tmem + lane_base + kColGW + (uint32_t)(t * kH + c16), v);
-                        if (p < K::NP)
-#pragma unroll
-                            for (int i = 0; i < 16; i += 4)
-                                *reinterpret_cast<float4*>(dst + c16 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                    }
-                }
-            } else if (lane == 0) {
-                atomicOr(prm.status, 4u);
+                copy_gd(prm, tmem, warp & 3, lane, k0 + j * kEdgeTile, k1, sg);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(gd_empty);
             }
         }
     } else if (warp == kBwdMmaWarp) {
@@ -659,7 +681,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, kBwdTmemCols);
     }
 }
 

@@ -88,7 +88,7 @@ struct RadLaunch {
     static int bwd_slices(int C) { return C / kSlice; }
     static constexpr int bwd_groups() { return (KP::NP + kBwdGroupPaths - 1) / kBwdGroupPaths; }
     static int bwd_nodes_per_cta(int N, int C) {
-        const long long want = 148LL * 4;   // about 4 waves of one CTA per SM
+        const long long want = 148LL * 2 * 4;   // about 4 waves of two CTAs per SM
         const int npc = (int)(((long long)N * bwd_slices(C) * bwd_groups() + want - 1) / want);
         return npc < 1 ? 1 : npc;
     }
