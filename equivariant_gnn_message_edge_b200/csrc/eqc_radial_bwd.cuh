@@ -14,21 +14,24 @@
 // routes of r count).
 //
 // radial_conv_bwd_kernel: one CTA per sender range x 32-channel slice x
-// group of up to 8 paths (2 MMA tiles of 4 paths x 32 channels).  Warps:
-//   * 0..7 (path warps): warp w owns path 8 g + w, its lanes the 32 channels.
-//     For every out-edge of the current sender (positions of the sender
-//     CSR) it reads w from tensor memory, the receiver's gy rows from the
-//     ring, the edge's harmonics, and with h[m1][m2] = sum_m3 C_p gy[m3]:
+// group of up to 4 paths (one MMA tile of 4 paths x 32 channels); two CTAs
+// share an SM where their shared memory allows.  Warps:
+//   * 0..3 (path warps): warp w owns path 4 g + w, its lanes the 32 channels
+//     and tensor-memory subpartition w.  For every out-edge of the current
+//     sender (positions of the sender CSR) it reads w from tensor memory,
+//     the receiver's gy rows from the ring, the edge's harmonics, and with
+//     h[m1][m2] = sum_m3 C_p gy[m3]:
 //       t[m1] = sum_m2 Y[m2] h,  dw = x . t,  dx += w t,
 //       gY[m2] += w sum_m1 x[m1] h      (summed over the 32 lanes)
 //     u dw goes, scaled and split into fp16 halves, into the G tile
-//     [(path, channel) rows][64 edges] in shared memory;
-//   * 8..11 (reader warps, one per tensor-memory subpartition): copy Gd of
-//     every tile and, at the end, the CTA's g_W3 rows out of tensor memory;
-//   * 12 (one thread): stages W3^T and h2 tiles with TMA and issues the
+//     [(path, channel) rows][64 edges] in shared memory.  Each also copies
+//     its subpartition's rows of Gd per tile and its path's g_W3 rows at the
+//     end out of tensor memory (a warp without a path copies only Gd);
+//   * 4 (one thread): stages W3^T and h2 tiles with TMA and issues the
 //     MMAs: w = W3^T . h2^T, then per tile g_W3 += G . h2 and Gd = W3 . G
 //     (K over the tile's edges / the group's rows), G the tile of u dw;
-//   * 13 (one thread): copies each position's receiver row gy[i, :, slice].
+//   * 5: copies each batch's receiver rows gy[i, :, slice] (one lane per
+//     position).
 // Per-path dx blocks, per-edge gY partials, Gd partials and g_W3 partials go
 // to the workspace; radial_bwd_epilogue_kernel and the reductions finish dr,
 // dx and the weight gradients in a fixed order (deterministic).

@@ -10,20 +10,25 @@
 //
 // One CTA takes a range of receivers (their in-edges are consecutive
 // positions of the receiver CSR), one slice of 32 channels and a group of up
-// to 12 paths.  Its 448 threads are 14 warps with fixed roles:
-//   * warp 12 (one thread): stages the group's W3^T rows (3 tiles of 4
+// to 4 paths.  Its 192 threads are 6 warps with fixed roles (two CTAs share
+// an SM; grouping 4 paths per CTA keeps the distinct per-path code an SM runs
+// small and lets a light path's CTA finish early instead of waiting on the
+// heaviest path of a larger group):
+//   * warp 4 (one thread): stages the group's W3^T rows (one tile of 4
 //     paths x 32 channels, fp16 hi/lo, resident for the whole CTA) and the
 //     h2 tiles of 64 positions (TMA, 2 stages), and issues the MMAs
 //       D[(path, channel), edge] = W3^T . h2^T      (M = 128, N = 64, K = 64)
-//     into one of two tensor-memory buffers (3 x 64 columns each);
-//   * warp 13 (one thread): copies each position's sender row x[s, :, slice]
-//     into a ring of shared-memory slots (TMA, one box of D_in x 32 floats);
-//   * warps 0..11 (the path warps): warp w owns path p = 12 g + w.  Its lanes
-//     are the slice's 32 channels, and tensor-memory lanes 32 (w % 4) .. +31
-//     of tile w / 4 hold exactly that path's 32 channels, so each lane reads
-//     its own w[e, p, c] with tcgen05.ld.  Per edge it forms the path's
-//     coupling A_p = C_p . Y(r_e) (lane t for edge t of a batch, into shared
-//     memory), reads its input block of the x slot and accumulates
+//     into one of two tensor-memory buffers (64 columns each);
+//   * warp 5: copies the sender rows x[s, :, slice] of each batch of 8
+//     positions into a ring of shared-memory slots (TMA, one box of
+//     D_in x 32 floats per position) and publishes each position's
+//     harmonics, edge factor and receiver beside them;
+//   * warps 0..3 (the path warps): warp w owns path p = 4 g + w.  Its lanes
+//     are the slice's 32 channels, and tensor-memory lanes 32 w .. +31 hold
+//     exactly that path's 32 channels, so each lane reads its own
+//     w[e, p, c] with tcgen05.ld.  Per batch it forms the path's coupling
+//     A_p = C_p . Y(r_e) (lane t for position t, into shared memory), and per
+//     edge accumulates
 //       acc[m3] += w * sum_m1 A_p[m3][m1] x[m1]
 //     for the current receiver, writing the path's output block of a
 //     receiver when its edges end.
@@ -38,14 +43,13 @@ namespace eqc {
 namespace radial {
 
 constexpr int kSlice = 32;         // channels per CTA: one per lane of a path warp
-constexpr int kGroupPaths = 12;    // paths per CTA: 3 MMA tiles of 4 paths x 32 channels
-constexpr int kGroupTiles = 3;
-constexpr int kPathWarps = 12;
-constexpr int kMmaWarp = 12, kXWarp = 13;
-constexpr int kConvThreads = 14 * 32;
+constexpr int kGroupPaths = 4;     // paths per CTA: one MMA tile of 4 paths x 32 channels
+constexpr int kGroupTiles = 1;
+constexpr int kPathWarps = 4;
+constexpr int kMmaWarp = 4, kXWarp = 5;
+constexpr int kConvThreads = 6 * 32;
 constexpr int kXBatches = 2;       // sender-row batches in flight (double buffer)
-constexpr int kBatch = 16;         // edges per harmonics / coupling batch of a path warp (at most)
-constexpr int kTmemCols = 512;     // 2 buffers x 3 tiles x 64 columns, rounded to a power of two
+constexpr int kTmemCols = 128;     // 2 buffers x 1 tile x 64 columns (several CTAs share an SM)
 
 struct RadFwdParams {
     const float* x;      // [N][D_in][C]
@@ -71,7 +75,7 @@ constexpr int max_coupling_floats() {
 // Shared-memory layout of the fused forward (bytes; tiles 1024-aligned).
 template <class K>
 struct RadFwdSmem {
-    static constexpr int BT = K::D_IN >= 16 ? 8 : kBatch;                 // positions per batch
+    static constexpr int BT = 8;                                            // positions per batch
     static constexpr int A_TILE = kRowTile * kTileRowBytes;                 // 16 KB: 128 rows of W3^T
     static constexpr int H_TILE = kEdgeTile * kTileRowBytes;                // 8 KB: 64 rows of h2
     static constexpr int W3_OFF = 0;                                        // [tile][hi, lo]
@@ -260,7 +264,7 @@ __device__ __forceinline__ void path_warp_fwd(const RadFwdParams& prm, uint8_t* 
 }
 
 template <class K>
-__global__ void __launch_bounds__(kConvThreads, 1)
+__global__ void __launch_bounds__(kConvThreads, 2)
     radial_conv_fwd_kernel(const RadFwdParams prm, const __grid_constant__ CUtensorMap map_a_hi,
                            const __grid_constant__ CUtensorMap map_a_lo, const __grid_constant__ CUtensorMap map_h_hi,
                            const __grid_constant__ CUtensorMap map_h_lo, const __grid_constant__ CUtensorMap map_x) {

@@ -60,8 +60,8 @@ struct RadLaunch {
                 attr_done[dev] = true;
             }
             const int slices = a.C / kSlice, groups = (KP::NP + kGroupPaths - 1) / kGroupPaths;
-            // about 4 waves of one CTA per SM
-            const long long want = 148LL * 4;
+            // about 4 waves of two CTAs per SM
+            const long long want = 148LL * 2 * 4;
             int npc = (int)(((long long)a.N * slices * groups + want - 1) / want);
             if (npc < 1) npc = 1;
             RadFwdParams prm{a.x, a.recv_ptr, ws.rec, ws.ids, y_pp, a.N, a.C, a.E, npc, a.status};
