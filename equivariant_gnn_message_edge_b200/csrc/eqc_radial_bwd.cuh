@@ -119,19 +119,29 @@ struct RadBwdSmem {
     static constexpr int A_TILE = kRowTile * kTileRowBytes;               // 16 KB
     static constexpr int H_TILE = kEdgeTile * kTileRowBytes;              // 8 KB
     static constexpr int G_TILE = kRowTile * kEdgeTile * 2;               // 16 KB: 128 rows x 64 edges fp16
-    static constexpr int W3_OFF = 0;                                      // [tile][hi, lo]
-    static constexpr int H_OFF = W3_OFF + kBwdGroupTiles * 2 * A_TILE;    // [stage][hi, lo]
-    static constexpr int G_OFF = H_OFF + 2 * 2 * H_TILE;                  // [tile][hi, lo]
     static constexpr int GY_SLOT = K::D_OUT * kSlice * 4;
-    static constexpr int GY_OFF = G_OFF + kBwdGroupTiles * 2 * G_TILE;
     static constexpr int YS = (K::D_SH + 3) & ~3;                         // harmonics row (floats)
     // per path warp, for a batch of up to 8 positions: harmonics rows + edge factor, and w
     static constexpr int Y_WARP8 = 8 * (YS + 4) * 4 + 8 * 32 * 4;
-    // gy ring: batches of BT receiver rows, as many (2 .. 4) as fit beside the rest;
-    // BT = 8 where two batches of 8 fit, else 4, else 2.  Two CTAs share an SM
-    // (113 KB each) when a ring of two 4-position batches fits, else one (227 KB).
-    static constexpr int FIXED = GY_OFF + kBwdPathWarps * Y_WARP8 + (14 + 2 * 4) * 8 + 16 + 1024;
-    static constexpr bool TWO = (113 * 1024 - FIXED) / GY_SLOT >= 8;
+    // everything but the gy ring, with hs stages of h2
+    static constexpr int fixed_for(int hs) {
+        return kBwdGroupTiles * 2 * A_TILE + hs * 2 * H_TILE + kBwdGroupTiles * 2 * G_TILE +
+               kBwdPathWarps * Y_WARP8 + (14 + 2 * 4) * 8 + 16 + 1024;
+    }
+    static constexpr bool two_for(int hs) { return (113 * 1024 - fixed_for(hs)) / GY_SLOT >= 8; }
+    // Two CTAs share an SM (113 KB each) when a gy ring of two 4-position
+    // batches fits beside the rest, else one (227 KB).  Two h2 stages: with
+    // one, the next tile's h2 waits for this tile's products (measured slower
+    // at lmax3 even with two CTAs per SM).
+    static constexpr int HS = 2;
+    static constexpr bool TWO = two_for(HS);
+    static constexpr int W3_OFF = 0;                                      // [tile][hi, lo]
+    static constexpr int H_OFF = W3_OFF + kBwdGroupTiles * 2 * A_TILE;    // [stage][hi, lo]
+    static constexpr int G_OFF = H_OFF + HS * 2 * H_TILE;                 // [tile][hi, lo]
+    static constexpr int GY_OFF = G_OFF + kBwdGroupTiles * 2 * G_TILE;
+    // gy ring: batches of BT receiver rows, as many (2 .. 4) as fit beside the
+    // rest; BT = 8 where two batches of 8 fit, else 4, else 2
+    static constexpr int FIXED = fixed_for(HS);
     static constexpr int FIT = ((TWO ? 113 : 227) * 1024 - FIXED) / GY_SLOT;
     static constexpr int BT = FIT >= 16 ? 8 : (FIT >= 8 ? 4 : 2);
     static constexpr int GYB = FIT / BT >= 4 ? 4 : FIT / BT;
@@ -550,30 +560,31 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
                     tma_2d(dst + S::A_TILE, &map_a_lo, 0, row, w3_full);
                 }
             int h_issued = 0, h_waited = 0, committed = 0, g_done = 0;
+            // h2 tile j sits in stage j % HS, phase (j / HS) & 1
             auto load_h = [&](int j) {
-                const int s = j & 1;
-                uint8_t* dst = base + S::H_OFF + s * 2 * S::H_TILE;
-                mbar_expect_tx(&h_full[s], 2 * S::H_TILE);
-                tma_2d(dst, &map_h_hi, 0, k0 + j * kEdgeTile, &h_full[s]);
-                tma_2d(dst + S::H_TILE, &map_h_lo, 0, k0 + j * kEdgeTile, &h_full[s]);
+                const int hs = j % S::HS;
+                uint8_t* dst = base + S::H_OFF + hs * 2 * S::H_TILE;
+                mbar_expect_tx(&h_full[hs], 2 * S::H_TILE);
+                tma_2d(dst, &map_h_hi, 0, k0 + j * kEdgeTile, &h_full[hs]);
+                tma_2d(dst + S::H_TILE, &map_h_lo, 0, k0 + j * kEdgeTile, &h_full[hs]);
                 h_issued = j + 1;
             };
             load_h(0);
-            if (ntiles > 1) load_h(1);
+            if (S::HS > 1 && ntiles > 1) load_h(1);
             const bool w3_ok = mbar_wait_one(w3_full, 0);
             bool ok = w3_ok;
             constexpr uint32_t id_w = idesc_f16(kRowTile, kEdgeTile);                 // W3^T . H^T
             constexpr uint32_t id_gw = idesc_f16(kRowTile, kH, false, true);          // G . H (B MN-major)
             constexpr uint32_t id_gd = idesc_f16(kH, kEdgeTile, true, true);          // W3 . G (both MN-major)
             for (int j = 0; j < ntiles && ok; ++j) {
-                const int s = j & 1;
-                ok = mbar_wait_one(&h_full[s], (uint32_t)(j >> 1) & 1u);
+                const int s = j & 1, hst = j % S::HS;
+                ok = mbar_wait_one(&h_full[hst], (uint32_t)(j / S::HS) & 1u);
                 if (!ok) break;
                 h_waited = j + 1;
                 ok = (j < 2 || mbar_wait_one(&t_empty[s], (uint32_t)((j >> 1) - 1) & 1u)) && !*abort_flag;
                 if (!ok) break;
                 tc_fence_after();
-                const uint8_t* hs = base + S::H_OFF + s * 2 * S::H_TILE;
+                const uint8_t* hs = base + S::H_OFF + hst * 2 * S::H_TILE;
                 const uint64_t dbh = sw128_desc(smem_addr(hs)), dbl = sw128_desc(smem_addr(hs + S::H_TILE));
                 // w of this tile
                 for (int t = 0; t < gtiles; ++t) {
@@ -623,11 +634,11 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
                 }
                 umma_commit(g_empty);
                 umma_commit(gd_full);
-                umma_commit(&h_empty[s]);
+                umma_commit(&h_empty[hst]);
                 g_done = j + 1;
-                if (j + 2 < ntiles) {
-                    ok = mbar_wait_one(&h_empty[s], (uint32_t)(j >> 1) & 1u);
-                    if (ok) load_h(j + 2);
+                if (j + S::HS < ntiles) {
+                    ok = mbar_wait_one(&h_empty[hst], (uint32_t)(j / S::HS) & 1u);
+                    if (ok) load_h(j + S::HS);
                 }
             }
             if (ok && !*abort_flag) {
@@ -637,7 +648,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
                 *abort_flag = 1;
                 // let the copies and products in flight land before the CTA lets go of its memory
                 if (!w3_ok) mbar_wait_one(w3_full, 0);
-                for (int u = h_waited; u < h_issued; ++u) mbar_wait_one(&h_full[u & 1], (uint32_t)(u >> 1) & 1u);
+                for (int u = h_waited; u < h_issued; ++u)
+                    mbar_wait_one(&h_full[u % S::HS], (uint32_t)(u / S::HS) & 1u);
                 for (int u = committed > 2 ? committed - 2 : 0; u < committed; ++u)
                     mbar_wait_one(&t_full[u & 1], (uint32_t)(u >> 1) & 1u);
                 if (g_done > 0) mbar_wait_one(g_empty, (uint32_t)(g_done - 1) & 1u);
