@@ -289,6 +289,16 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
     }
 
     uint32_t ghi[4] = {0u, 0u, 0u, 0u}, glo[4] = {0u, 0u, 0u, 0u};   // 8 edges of fp16 G values
+    // partials of the last edge, summed over the warp one edge later
+    float vp[NV];
+    int kp = -1;
+    auto reduce_store = [&]() {
+        const float sum = warp_transpose_sum<NV>(vp, lane);
+        constexpr int sh = transpose_sum_shift(NV);
+        const int vi = lane >> sh;
+        if ((lane & ((1 << sh) - 1)) == 0 && vi < NVAL)
+            prm.gy_part[((size_t)kp * slices + slice) * R::SD2 + ogp + vi] = sum;
+    };
     const int ntiles = (k1 - k0 + kEdgeTile - 1) / kEdgeTile;
     for (int j = 0; j < ntiles; ++j) {
         const int s = j & 1;
@@ -401,11 +411,12 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
 #pragma unroll
                         for (int m = 0; m < d2; ++m) v[1 + m] = w * hG[m];
                     }
-                    const float sum = warp_transpose_sum<NV>(v, lane);
-                    constexpr int sh = transpose_sum_shift(NV);
-                    const int vi = lane >> sh;
-                    if ((lane & ((1 << sh) - 1)) == 0 && vi < NVAL)
-                        prm.gy_part[((size_t)(kb + t) * slices + slice) * R::SD2 + ogp + vi] = sum;
+                    // the previous edge's partials are summed now, so their shuffle
+                    // chain overlaps this edge's arithmetic
+                    if (kp >= 0) reduce_store();
+#pragma unroll
+                    for (int q = 0; q < NV; ++q) vp[q] = v[q];
+                    kp = kb + t;
                 }
                 // pack G (zero for edges past the range) and store every 8 edges
                 __half gh, gl;
@@ -439,6 +450,7 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
             mbar_arrive(&t_empty[s]);
         }
     }
+    if (kp >= 0) reduce_store();
     // the last tile's Gd, then the CTA's g_W3 rows of this path
     if (ntiles > 0) {
         if (!mbar_wait(gd_full, (uint32_t)(ntiles - 1) & 1u) || !mbar_wait(gw_full, 0u)) {
