@@ -121,14 +121,16 @@ struct RadBwdSmem {
     static constexpr int G_TILE = kRowTile * kEdgeTile * 2;               // 16 KB: 128 rows x 64 edges fp16
     static constexpr int GY_SLOT = K::D_OUT * kSlice * 4;
     static constexpr int YS = (K::D_SH + 3) & ~3;                         // harmonics row (floats)
-    // per path warp, for a batch of up to 8 positions: harmonics rows + edge factor, and w
-    static constexpr int Y_WARP8 = 8 * (YS + 4) * 4 + 8 * 32 * 4;
+    // per path warp, for a batch of up to 8 positions: w
+    static constexpr int WS_WARP8 = 8 * 32 * 4;
+    // per ring position: the gy rows, then the harmonics row, edge factor and sender
+    static constexpr int POS_BYTES = GY_SLOT + (YS + 4) * 4;
     // everything but the gy ring, with hs stages of h2
     static constexpr int fixed_for(int hs) {
         return kBwdGroupTiles * 2 * A_TILE + hs * 2 * H_TILE + kBwdGroupTiles * 2 * G_TILE +
-               kBwdPathWarps * Y_WARP8 + (14 + 2 * 4) * 8 + 16 + 1024;
+               kBwdPathWarps * WS_WARP8 + (14 + 2 * 4) * 8 + 16 + 1024;
     }
-    static constexpr bool two_for(int hs) { return (113 * 1024 - fixed_for(hs)) / GY_SLOT >= 8; }
+    static constexpr bool two_for(int hs) { return (113 * 1024 - fixed_for(hs)) / POS_BYTES >= 8; }
     // Two CTAs share an SM (113 KB each) when a gy ring of two 4-position
     // batches fits beside the rest, else one (227 KB).  Two h2 stages: with
     // one, the next tile's h2 waits for this tile's products (measured slower
@@ -142,13 +144,15 @@ struct RadBwdSmem {
     // gy ring: batches of BT receiver rows, as many (2 .. 4) as fit beside the
     // rest; BT = 8 where two batches of 8 fit, else 4, else 2
     static constexpr int FIXED = fixed_for(HS);
-    static constexpr int FIT = ((TWO ? 113 : 227) * 1024 - FIXED) / GY_SLOT;
+    static constexpr int FIT = ((TWO ? 113 : 227) * 1024 - FIXED) / POS_BYTES;
     static constexpr int BT = FIT >= 16 ? 8 : (FIT >= 8 ? 4 : 2);
     static constexpr int GYB = FIT / BT >= 4 ? 4 : FIT / BT;
-    static constexpr int Y_WARP = BT * (YS + 4) * 4;
+    // per gy batch buffer, written by the gy warp: each position's harmonics
+    // (rows of YS floats), edge factor and sender
+    static constexpr int YB_BATCH = BT * (YS + 4) * 4;
     static constexpr int WS_WARP = BT * 32 * 4;
     static constexpr int Y_OFF = GY_OFF + GYB * BT * GY_SLOT;
-    static constexpr int WS_OFF = Y_OFF + kBwdPathWarps * Y_WARP;
+    static constexpr int WS_OFF = Y_OFF + GYB * YB_BATCH;
     static constexpr int BAR_OFF = WS_OFF + kBwdPathWarps * WS_WARP;
     // w3, h_full[2], h_empty[2], t_full[2], t_empty[2], g_full, g_empty, gd_full, gd_empty, gw_full,
     // gy_full[GYB], gy_empty[GYB]
@@ -230,7 +234,6 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
     uint64_t* gw_full = bars + 13;
     uint64_t* gy_full = bars + 14;
     uint64_t* gy_empty = bars + 14 + S::GYB;
-    float* ys = reinterpret_cast<float*>(base + S::Y_OFF + warp * S::Y_WARP);     // [BT][YS + 4]
     float* wst = reinterpret_cast<float*>(base + S::WS_OFF + warp * S::WS_WARP);  // [BT][32]
     const float* gring = reinterpret_cast<const float*>(base + S::GY_OFF);
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
@@ -280,14 +283,6 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
     load_x(cur, xv);
     load_x(cur + 1, xn);
 
-    // the next batch's records (lane t < BT holds position kb + t), prefetched
-    float4 nrec = make_float4(0.f, 0.f, 0.f, 0.f);
-    int nown = 0;
-    if (lane < BT && k0 + lane < k1) {
-        nrec = prm.rec[k0 + lane];
-        nown = prm.ids[k0 + lane].y;
-    }
-
     uint32_t ghi[4] = {0u, 0u, 0u, 0u}, glo[4] = {0u, 0u, 0u, 0u};   // 8 edges of fp16 G values
     // partials of the last edge, summed over the warp one edge later
     float vp[NV];
@@ -326,40 +321,25 @@ __device__ __forceinline__ void path_warp_bwd(const RadBwdParams& prm, uint8_t* 
         for (int kb = kt; kb < kt + kEdgeTile; kb += BT) {
             const int nb = max(0, min(BT, kt_end - kb));
             const int b = (kb - k0) / BT;
-            int own = 0;
             const float* gb = gring;
+            const float* ys = gring;   // the batch's harmonics rows (written by the gy warp)
             if (nb > 0) {
-                const float4 rc = nrec;
-                own = nown;
-                if (lane < BT && kb + BT + lane < k1) {   // prefetch the batch after this one
-                    nrec = prm.rec[kb + BT + lane];
-                    nown = prm.ids[kb + BT + lane].y;
-                }
-                if (lane < nb) {
-                    float ux, uy, uz, il;
-                    const bool ok = unit_dir(rc.x, rc.y, rc.z, ux, uy, uz, il);
-                    float Y[K::D_SH];
-                    sh_eval<K::LSH>(ok, ux, uy, uz, Y);
-                    float* yrow = ys + lane * (S::YS + 4);
-#pragma unroll
-                    for (int q = 0; q < K::D_SH; ++q) yrow[q] = Y[q];
-                    yrow[S::YS] = rc.w;
-                }
                 tmem_stash<BT>(tcol + (uint32_t)(kb - kt), wst, lane);   // z3 * 2^(sA + sB), BT positions
-                __syncwarp();
+                // the batch's receiver rows, harmonics, edge factors and senders
                 if (!mbar_wait(&gy_full[b % S::GYB], (uint32_t)(b / S::GYB) & 1u) ||
                     __any_sync(0xffffffffu, *abort_flag)) {
                     abort_now();
                     return;
                 }
                 gb = gring + (b % S::GYB) * BT * (S::GY_SLOT / 4) + o3 * kSlice + lane;
+                ys = reinterpret_cast<const float*>(base + S::Y_OFF + (b % S::GYB) * S::YB_BATCH);
             }
             for (int t = 0; t < BT; ++t) {
                 float gval = 0.f;
                 if (t < nb) {
-                    const int own_t = __shfl_sync(0xffffffffu, own, t);
-                    while (cur < own_t) next_sender();   // the current sender's edges are done (empty ones too)
                     const float* yrow = ys + t * (S::YS + 4);
+                    const int own_t = __float_as_int(yrow[S::YS + 1]);
+                    while (cur < own_t) next_sender();   // the current sender's edges are done (empty ones too)
                     const float us = yrow[S::YS];
                     const float Dv = wst[t * 32 + lane];
                     const float w = Dv * us;
@@ -522,7 +502,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
         mbar_init(gd_empty, 4);
         mbar_init(gw_full, 1);
         for (int q = 0; q < S::GYB; ++q) {
-            mbar_init(&gy_full[q], 1);
+            mbar_init(&gy_full[q], 2);   // the copies' bytes + the batch info
             mbar_init(&gy_empty[q], gp);
         }
         *abort_flag = 0;
@@ -676,9 +656,13 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
         for (int b = 0; b < nbatch; ++b) {
             const int kb = k0 + b * BT;
             const int nb = min(BT, k1 - kb);
-            int ridx = 0;
+            int ridx = 0, own = 0;
+            float4 rc = make_float4(0.f, 0.f, 0.f, 0.f);
             if (lane < nb) {
-                ridx = prm.ids[kb + lane].x;
+                const int2 id = prm.ids[kb + lane];
+                rc = prm.rec[kb + lane];
+                ridx = id.x;
+                own = id.y;
                 if ((unsigned)ridx >= (unsigned)prm.N) {   // out of range: flagged, read as node 0
                     atomicOr(prm.status, 1u);
                     ridx = 0;
@@ -698,6 +682,21 @@ __global__ void __launch_bounds__(kBwdThreads, 2)
                 tma_rows(base + S::GY_OFF + ((b % S::GYB) * BT + lane) * S::GY_SLOT, &map_gy, c0, ridx,
                          &gy_full[b % S::GYB], policy_evict_last());
             issued = b + 1;
+            // each position's harmonics, edge factor and sender for the path warps
+            if (lane < nb) {
+                float* yrow = reinterpret_cast<float*>(base + S::Y_OFF + (b % S::GYB) * S::YB_BATCH) +
+                              lane * (S::YS + 4);
+                float ux, uy, uz, il;
+                const bool okd = unit_dir(rc.x, rc.y, rc.z, ux, uy, uz, il);
+                float Y[K::D_SH];
+                sh_eval<K::LSH>(okd, ux, uy, uz, Y);
+#pragma unroll
+                for (int q = 0; q < K::D_SH; ++q) yrow[q] = Y[q];
+                yrow[S::YS] = rc.w;
+                yrow[S::YS + 1] = __int_as_float(own);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&gy_full[b % S::GYB]);
         }
         // the last fills of each buffer land before the CTA lets go of its memory
         if (lane == 0)
