@@ -147,6 +147,11 @@ __device__ __forceinline__ void tmem_stash(uint32_t taddr, float* dst, int lane)
         tmem_ld8(taddr, v);
 #pragma unroll
         for (int t = 0; t < 8; ++t) dst[t * 32 + lane] = v[t];
+    } else if constexpr (BT == 4) {
+        float v[4];
+        tmem_ld4(taddr, v);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) dst[t * 32 + lane] = v[t];
     } else {
 #pragma unroll
         for (int t = 0; t < BT; ++t) dst[t * 32 + lane] = tmem_ld1(taddr + (uint32_t)t);
