@@ -908,9 +908,8 @@ constexpr int transpose_sum_shift(int nv) { return nv >= 32 ? 0 : nv >= 16 ? 1 :
 // !DET: node = receiver i, resident gy_i, dx scattered with atomic adds.
 // FUSED: the tile covers every channel (T == 1): dr is finished in-kernel.
 template <class K, bool DET, bool FUSED>
-__global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
-    eqconv_bwd_kernel(const BwdParams prm, const __grid_constant__ CUtensorMap tmap_w,
-                      const __grid_constant__ CUtensorMap tmap_g) {
+__device__ __forceinline__ void eqconv_bwd_body(const BwdParams& prm, const CUtensorMap* tmap_w,
+                                                const CUtensorMap* tmap_g) {
     constexpr int V = K::VEC;
     constexpr int S = K::STAGES;
     constexpr int GG = K::G > 0 ? K::G : 1;
@@ -986,7 +985,7 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
         for (int t = 0; t < pre; ++t) {
             const int e = __shfl_sync(0xffffffffu, my_e, t), o = __shfl_sync(0xffffffffu, my_o, t);
             const uint32_t gi = g + t;
-            stage_fill<K, DL>(stages + (gi % S) * SF, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e, o, c0, pol_stream,
+            stage_fill<K, DL>(stages + (gi % S) * SF, &bars[2 * (gi % S)], tmap_w, tmap_g, e, o, c0, pol_stream,
                               pol_keep, lane);
         }
         for (int b0 = 0; b0 < n && ok_all; b0 += CH) {
@@ -1074,7 +1073,7 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
                 __syncwarp();
                 if (t + S < n) {
                     const int e2 = __shfl_sync(0xffffffffu, my_e, t + S), o2 = __shfl_sync(0xffffffffu, my_o, t + S);
-                    stage_fill<K, DL>(st, &bars[2 * (gi % S)], &tmap_w, &tmap_g, e2, o2, c0, pol_stream, pol_keep,
+                    stage_fill<K, DL>(st, &bars[2 * (gi % S)], tmap_w, tmap_g, e2, o2, c0, pol_stream, pol_keep,
                                       lane);
                 }
             }
@@ -1116,6 +1115,24 @@ __global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
             }
         }
     }
+}
+
+template <class K, bool DET, bool FUSED>
+__global__ void __launch_bounds__(BwdShape<K, DET>::WARPS * 32)
+    eqconv_bwd_kernel(const BwdParams prm, const __grid_constant__ CUtensorMap tmap_w,
+                      const __grid_constant__ CUtensorMap tmap_g) {
+    eqconv_bwd_body<K, DET, FUSED>(prm, &tmap_w, &tmap_g);
+}
+
+// The deterministic kernel that leaves dr to the epilogue (several channel
+// tiles) at 128-channel tiles, capped at 168 registers (shared memory then
+// allows 3 CTAs of 3 warps per SM): left to its own heuristic it takes 232
+// and holds 2 CTAs, with no spill either way.
+template <class K>
+__global__ void __launch_bounds__(BwdShape<K, true>::WARPS * 32, 4)
+    eqconv_bwd_tiles_kernel(const BwdParams prm, const __grid_constant__ CUtensorMap tmap_w,
+                            const __grid_constant__ CUtensorMap tmap_g) {
+    eqconv_bwd_body<K, true, false>(prm, &tmap_w, &tmap_g);
 }
 
 // dr for edges whose gY is split over T channel tiles: fixed-order sum, then

@@ -57,6 +57,7 @@ struct Launch {
     static cudaError_t bwd_one(const BwdParams& prm_in, int bands, cudaStream_t st) {
         BwdParams prm = prm_in;
         auto kern = eqconv_bwd_kernel<K, DET, FUSED>;
+        if constexpr (DET && !FUSED && K::VEC == 4) kern = eqconv_bwd_tiles_kernel<K>;
         static bool done[64] = {};
         constexpr int W = BwdShape<K, DET>::WARPS;
         constexpr int smem = W * BwdShape<K, DET>::L::BYTES;
